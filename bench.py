@@ -1,0 +1,634 @@
+#!/usr/bin/env python
+"""ReSA decode hot-path benchmark on B200.
+
+One step = one ReSA cycle of f = 32 tokens through every layer: f-1 sparse
+decode steps (append + block selection + group block-sparse split-KV
+attention) followed by one dense rectification of the last f tokens
+(write-back + descriptor refresh + causal chunk attention), per layer, as in
+Algorithm 1 of the Rectified Sparse Attention summary.  Each cycle is one CUDA
+graph of libresa launches; inputs are seeded synthetic tensors resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long256k]
+    python bench.py --impl reference ...     # the CPU oracle on the same workload
+
+Multi-GPU: one process per GPU (torchrun); the path does not shard, so every
+rank runs an independent replica (weak scaling) and the time is the maximum
+over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-decode attn tokens/s & µs/step at 256K ctx; achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+WORKLOADS = {
+    "long256k": dict(layers=28, batch=1, hq=28, hkv=4, d=128, ctx=[262144], f=32, paged=False,
+                     text="long-context decode: 28 layers x (28 q / 4 kv heads, d 128), batch 1, "
+                          "262144-token bf16 cache, block 16, top-k 10% (1638) + current block, "
+                          "ReSA cycle f=32 (31 sparse decode steps + 1 dense rectification)"),
+    "loop64k": dict(layers=1, batch=4, hq=28, hkv=4, d=128, ctx=[65536] * 4, f=32, paged=False,
+                    text="ReSA decode loop: 1 layer (28 q / 4 kv, d 128), batch 4, 65536-token "
+                         "cache, top-k 10%, 31 sparse decode steps + 1 rectification of 32"),
+    "cbatch": dict(layers=1, batch=32, hq=28, hkv=4, d=128, ctx=None, f=32, paged=True,
+                   text="continuous batching: 1 layer, 32 sequences with lengths uniform in "
+                        "[8192, 131072], random page order, top-k 10% per sequence"),
+    "tiny": dict(layers=1, batch=1, hq=4, hkv=2, d=64, ctx=[2048], f=32, paged=False,
+                 text="tiny: 1 layer (4 q / 2 kv, d 64), 2048-token cache, top-k 16"),
+}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["resa", "reference"], default="resa")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="long256k")
+    ap.add_argument("--seed", type=int, default=1234)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--breakdown-reps", type=int, default=5)
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (replicas only: no collective on the data path)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_setup(backend: str, world: int):
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    return dist
+
+
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity with one rank)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist=None, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# Workload construction
+# ---------------------------------------------------------------------------
+
+def topk_rule(L: int, bs: int = 16, n_min: int = 16) -> int:
+    """top-k of a decode step: max(n_min, round(M / 10)) capped at M, M = (L-1)//bs."""
+    M = (L - 1) // bs
+    return min(M, max(n_min, (M + 5) // 10))
+
+
+def workload_lengths(wl, seed):
+    from block_sparse_long_resa_b200 import inputs
+    if wl["ctx"] is None:
+        return inputs.continuous_batch_lengths(seed, wl["batch"], 8192, 131072)
+    return list(wl["ctx"])
+
+
+class Schedule:
+    """Sequence lengths and top-k per global step (decode steps and rectifications)."""
+
+    def __init__(self, ctx, f, cycles):
+        self.ctx, self.f, self.cycles = ctx, f, cycles
+        self.B = len(ctx)
+        self.Bpad = (self.B + 3) // 4 * 4  # 16-byte aligned rows
+
+    def decode_L(self, c, s):
+        return [L0 + c * self.f + s + 1 for L0 in self.ctx]
+
+    def rect_L(self, c):
+        return [L0 + (c + 1) * self.f for L0 in self.ctx]
+
+    def max_topk(self):
+        return max(topk_rule(L0 + self.cycles * self.f) for L0 in self.ctx)
+
+    def total_tokens(self):
+        return max(self.ctx) + self.cycles * self.f
+
+
+class GpuWorkload:
+    def __init__(self, wl, cycles, seed, device):
+        import torch
+        from block_sparse_long_resa_b200 import inputs
+        from block_sparse_long_resa_b200 import resa as R
+        self.wl, self.dev, self.cycles = wl, device, cycles
+        self.R = R
+        B, hq, hkv, d, f, nl = wl["batch"], wl["hq"], wl["hkv"], wl["d"], wl["f"], wl["layers"]
+        self.B, self.hq, self.hkv, self.d, self.f, self.layers = B, hq, hkv, d, f, nl
+        ctx = workload_lengths(wl, seed)
+        self.sched = Schedule(ctx, f, cycles)
+        self.cfg = R.make_config(hq, hkv, d, 16)
+        reserve = cycles * f + 16
+        # one paged cache per layer (K, V, descriptors); the page table is shared
+        self.k, self.v, self.desc, self.k_scale = [], [], [], []
+        for layer in range(nl):
+            p = inputs.make_decode_problem(seed + 1000 * layer, B, hq, hkv, d, 16, ctx,
+                                           reserve_tokens=reserve, paged=wl["paged"],
+                                           device=device, topk=[1] * B)
+            self.k.append(p.k_cache)
+            self.v.append(p.v_cache)
+            self.desc.append(torch.zeros(p.num_pages, hkv, 2, d, dtype=torch.bfloat16,
+                                         device=device))
+            self.k_scale.append(p.k_scale)
+            self.page_table = p.page_table
+            del p
+        self.max_pages = int(self.page_table.shape[1])
+        self.num_pages = int(self.k[0].shape[0])
+        self.max_topk = self.sched.max_topk()
+        self.ws = torch.empty(R.resa_workspace_size(self.cfg, B, self.max_pages, f),
+                              dtype=torch.uint8, device=device)
+        R.resa_workspace_init(self.ws)
+        # per-step sequence lengths / top-k rows (16-byte aligned rows)
+        nsteps = cycles * f
+        Bp = self.sched.Bpad
+        sl = torch.zeros(nsteps + 1, Bp, dtype=torch.int32)
+        tk = torch.zeros(nsteps + 1, Bp, dtype=torch.int32)
+        sl[nsteps, :B] = torch.tensor(ctx)
+        for c in range(cycles):
+            for s in range(f - 1):
+                Ls = self.sched.decode_L(c, s)
+                sl[c * f + s, :B] = torch.tensor(Ls)
+                tk[c * f + s, :B] = torch.tensor([topk_rule(x) for x in Ls])
+            sl[c * f + f - 1, :B] = torch.tensor(self.sched.rect_L(c))
+        self.seq_len = sl.to(device)
+        self.topk = tk.to(device)
+        # build the block key cache of the prefilled context (row nsteps = ctx)
+        for layer in range(nl):
+            R.resa_build_descriptors(self.cfg, self.cache(layer, nsteps), None, self.ws)
+        # inputs of every cycle, resident in HBM
+        g = torch.Generator(device=device)
+        g.manual_seed(seed + 77)
+        self.q = torch.randn(cycles, f - 1, nl, B, hq, d, generator=g, device=device).to(torch.bfloat16)
+        kk = torch.randn(cycles, f - 1, nl, B, hkv, d, generator=g, device=device)
+        for layer in range(nl):
+            kk[:, :, layer] *= self.k_scale[layer][None, None, None]
+        self.kn = kk.to(torch.bfloat16)
+        del kk
+        self.vn = torch.randn(cycles, f - 1, nl, B, hkv, d, generator=g, device=device).to(torch.bfloat16)
+        self.qc = torch.randn(cycles, nl, B, f, hq, d, generator=g, device=device).to(torch.bfloat16)
+        self.kc = torch.randn(cycles, nl, B, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
+        self.vc = torch.randn(cycles, nl, B, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
+        # outputs
+        self.out = torch.empty(nl, B, hq, d, device=device)
+        self.rout = torch.empty(nl, B, f, hq, d, device=device)
+        # separate allocations keep every layer's selection buffers 16-byte aligned
+        self.idx = [torch.empty(B, hkv, self.max_topk + 1, dtype=torch.int32, device=device)
+                    for _ in range(nl)]
+        self.cnt = [torch.empty(B, hkv, dtype=torch.int32, device=device) for _ in range(nl)]
+        torch.cuda.synchronize(device)
+
+    def cache(self, layer, step_row):
+        ptr = self.seq_len.data_ptr() + 4 * self.sched.Bpad * step_row
+        return self.R.make_cache(self.k[layer], self.v[layer], self.desc[layer], self.page_table,
+                                 ptr)
+
+    def topk_ptr(self, step_row):
+        return self.topk.data_ptr() + 4 * self.sched.Bpad * step_row
+
+    def launch_cycle(self, c):
+        """Enqueue one ReSA cycle (all layers) on the current stream."""
+        R, f = self.R, self.f
+        for s in range(f - 1):
+            row = c * f + s
+            for layer in range(self.layers):
+                R.resa_decode_step(self.cfg, self.cache(layer, row), self.q[c, s, layer],
+                                   self.kn[c, s, layer], self.vn[c, s, layer], self.topk_ptr(row),
+                                   self.max_topk, self.out[layer], None, self.idx[layer],
+                                   self.cnt[layer], self.ws)
+        row = c * f + f - 1
+        for layer in range(self.layers):
+            R.resa_rectify_attention(self.cfg, self.cache(layer, row), f, self.qc[c, layer],
+                                     self.kc[c, layer], self.vc[c, layer], self.rout[layer], None,
+                                     self.ws)
+
+    def launches_per_cycle(self):
+        R = self.R
+        return self.layers * ((self.f - 1) * R.resa_kernels_per_call("resa_decode_step") +
+                              R.resa_kernels_per_call("resa_rectify_attention"))
+
+    # algorithmic bytes / flops ---------------------------------------------
+    def decode_kernel_bytes(self, Ls):
+        """q + K/V of the selected blocks and the current block + fp32 output."""
+        B, hq, hkv, d = self.B, self.hq, self.hkv, self.d
+        kv = sum(hkv * (min(topk_rule(L), (L - 1) // 16) + 1) * 16 * d * 2 * 2 for L in Ls)
+        return B * hq * d * 2 + kv + B * hq * d * 4
+
+    def step_bytes(self, Ls):
+        """One sparse decode step of one layer: q + descriptors of the complete
+        blocks + selected K/V + output (the per-unit figure of the design notes)."""
+        hkv, d = self.hkv, self.d
+        desc = sum(((L - 1) // 16) * hkv * 2 * d * 2 for L in Ls)
+        return self.decode_kernel_bytes(Ls) + desc
+
+    def rectify_bytes_flops(self, Ls):
+        hkv, hq, d, f = self.hkv, self.hq, self.d, self.f
+        byts = sum(L * hkv * d * 2 * 2 for L in Ls) + len(Ls) * f * (hq * d * 2 + hq * d * 4)
+        flops = sum(sum(4 * hq * d * (L - f + r + 1) for r in range(f)) for L in Ls)
+        return byts, flops
+
+
+# ---------------------------------------------------------------------------
+# Clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = max((num(r[2]) for r in rows if num(r[2]) is not None), default=None)
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        loaded = [s for s, p in zip(sm, power) if p is not None and p > 250] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained",
+                                                                          d["bf16_tflops"])), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """One layer of the workload held by the CPU oracle.  A sample = one sparse
+    decode step + one rectification row (of f), extrapolated to a full cycle of
+    every layer: layers * ((f-1) * t_decode + f * t_row)."""
+
+    def __init__(self, wl, seed, layer_state=None):
+        from block_sparse_long_resa_b200 import inputs
+        from oracle import oracle as O
+        self.O, self.wl = O, wl
+        ctx = workload_lengths(wl, seed)
+        self.ctx = ctx
+        B, hq, hkv, d = wl["batch"], wl["hq"], wl["hkv"], wl["d"]
+        if layer_state is None:
+            p = inputs.make_decode_problem(seed, B, hq, hkv, d, 16, ctx,
+                                           reserve_tokens=4 * wl["f"] + 16, paged=wl["paged"],
+                                           topk=[1] * B)
+            self.cache = O.OracleCache(p.k_cache, p.v_cache, p.page_table, hq, hkv, d, 16)
+            self.cache.build_descriptors(p.ctx_len)
+            self.L0 = list(ctx)
+        else:
+            k, v, desc, pt, L0 = layer_state
+            self.cache = O.OracleCache(k, v, pt, hq, hkv, d, 16, desc=desc)
+            self.L0 = list(L0)
+        self.step = 0
+
+    def run(self):
+        import numpy as np
+        from block_sparse_long_resa_b200 import inputs
+        wl, f, B = self.wl, self.wl["f"], self.wl["batch"]
+        hq, hkv, d = wl["hq"], wl["hkv"], wl["d"]
+        self.step += 1
+        L = np.array([x + self.step for x in self.L0], dtype=np.int32)
+        q, kn, vn = inputs.make_step_tokens(99, self.step, B, hq, hkv, d)
+        topk = [topk_rule(int(x)) for x in L]
+        t0 = time.perf_counter()
+        self.cache.decode_step(q, kn, vn, topk, L, max(topk))
+        t_dec = time.perf_counter() - t0
+        qc, kc, vc = inputs.make_rectify_chunk(99 + self.step, B, f, hq, hkv, d)
+        t0 = time.perf_counter()
+        self.cache.rectify_rows(qc, kc, vc, L, f, [f - 1])
+        t_row = time.perf_counter() - t0
+        cycle_s = wl["layers"] * ((f - 1) * t_dec + f * t_row)
+        return cycle_s, t_dec, t_row
+
+    def describe(self):
+        wl = self.wl
+        return (f"1 of {wl['layers']} layers: one sparse decode step (append, pooling, scores, "
+                f"top-k, attention) + one of {wl['f']} rectification rows, extrapolated to a "
+                f"{wl['layers']}-layer cycle of {wl['f'] - 1} decode steps + 1 rectification")
+
+
+def cpu_baseline(wl, seed, layer_state, samples=2):
+    from oracle import oracle as O
+    s = OracleSample(wl, seed, layer_state)
+    cyc = [s.run()[0] for _ in range(samples)]
+    t = statistics.median(cyc)
+    return {"value": wl["f"] * wl["batch"] / t, "unit": "tokens/s", "cores": O.num_threads(),
+            "kind": "oracle", "sample": s.describe(), "s_per_cycle_extrapolated": t}
+
+
+# ---------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from oracle import oracle as O
+    wl = WORKLOADS[args.workload]
+    s = OracleSample(wl, args.seed)
+    for _ in range(args.warmup):
+        s.run()
+    times = [s.run()[0] for _ in range(args.steps)]
+    total = sum(times)
+    value = args.steps * wl["f"] * wl["batch"] / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 K/V, fp32 scores, fp64 attention (CPU oracle)",
+        "data": "synthetic (seeded N(0,1) q/K/V, LogNormal K channel scale, needle blocks)",
+        "config": {"workload": args.workload, "description": wl["text"],
+                   "step": f"one ReSA cycle of {wl['f']} tokens through {wl['layers']} layers",
+                   "note": "each step is a bounded sample extrapolated to a full cycle"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.num_threads(),
+                         "kind": "oracle", "sample": s.describe()},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_resa(args):
+    import torch
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA library has no CPU path)")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist = dist_setup("nccl", world)
+    wl = WORKLOADS[args.workload]
+    K, W = args.steps, args.warmup
+    cycles = K + W
+    t_setup = time.perf_counter()
+    w = GpuWorkload(wl, cycles, args.seed + rank, device)
+    stream = torch.cuda.Stream(device)
+    graphs = []
+    with torch.cuda.stream(stream):
+        # one eager cycle-0 dry run is not needed: capture directly (no host syncs inside)
+        for c in range(cycles):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                w.launch_cycle(c)
+            graphs.append(g)
+    torch.cuda.synchronize(device)
+    setup_s = time.perf_counter() - t_setup
+
+    for c in range(W):
+        graphs[c].replay()
+    torch.cuda.synchronize(device)
+    code = w.R.resa_check_device_status(w.ws, raise_on_error=False)
+    if code:
+        raise SystemExit(f"device error word 0x{code:x} after warm-up")
+
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for c in range(W, cycles):
+            graphs[c].replay()
+        ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    clk = clocks.stop()
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, dist, device)
+    tokens = K * wl["f"] * wl["batch"] * world
+    value = tokens / (ms / 1e3)
+
+    # end to end: pinned host inputs -> device, cycle graph, outputs -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t[W:].cpu().pin_memory() for t in (w.q, w.kn, w.vn, w.qc, w.kc, w.vc)]
+        dev_in = [w.q, w.kn, w.vn, w.qc, w.kc, w.vc]
+        host_out = [torch.empty_like(w.out, device="cpu").pin_memory(),
+                    torch.empty_like(w.rout, device="cpu").pin_memory()]
+        h2d = sum(t[0].numel() * t.element_size() for t in host_in)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i, c in enumerate(range(W, cycles)):
+                for hsrc, ddst in zip(host_in, dev_in):
+                    ddst[c].copy_(hsrc[i], non_blocking=True)
+                graphs[c].replay()
+                host_out[0].copy_(w.out, non_blocking=True)
+                host_out[1].copy_(w.rout, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+        e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / K}
+
+    code = w.R.resa_check_device_status(w.ws, raise_on_error=False)
+
+    # live per-kernel timing on the same data (last decode step's block lists)
+    bd = kernel_breakdown(w, stream, device, args.breakdown_reps)
+
+    hbm_peak, bf16_peak, bf16_sus, peak_src = measured_peaks()
+    last_dec_L = w.sched.decode_L(cycles - 1, wl["f"] - 2)
+    dec_bytes = w.decode_kernel_bytes(last_dec_L)
+    dec_gbs = dec_bytes / (bd["sparse_decode_us"] * 1e-6) / 1e9
+    roofline = {"kernel": "sparse_decode_kernel (resa_sparse_decode)", "bound": "hbm",
+                "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": dec_gbs / hbm_peak, "traffic": None,
+                "algorithmic_bytes_per_launch": dec_bytes,
+                "launch_us": bd["sparse_decode_us"], "peak_source": peak_src}
+    # whole-step roofline: algorithmic bytes of every kernel in the cycle
+    cyc_bytes = 0
+    for c in range(W, cycles):
+        for s in range(wl["f"] - 1):
+            cyc_bytes += wl["layers"] * w.step_bytes(w.sched.decode_L(c, s))
+        rb, _ = w.rectify_bytes_flops(w.sched.rect_L(c))
+        cyc_bytes += wl["layers"] * rb
+    step_gbs = cyc_bytes / (ms_local / 1e3) / 1e9
+    rb, rflops = w.rectify_bytes_flops(w.sched.rect_L(cycles - 1))
+    rect = {"us_per_layer": bd["rectify_us"],
+            "tflops": rflops / (bd["rectify_us"] * 1e-6) / 1e12,
+            "hbm_gbs": rb / (bd["rectify_us"] * 1e-6) / 1e9}
+    rect["frac_of_bf16_peak"] = rect["tflops"] / bf16_peak
+    rect["frac_of_hbm_peak"] = rect["hbm_gbs"] / hbm_peak
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        L_state = w.sched.decode_L(cycles - 1, wl["f"] - 2)
+        state = (w.k[0].cpu(), w.v[0].cpu(), w.desc[0].cpu(), w.page_table.cpu(),
+                 [x for x in L_state])
+        cpu = cpu_baseline(wl, args.seed, state)
+
+    per_token_us = ms / K / wl["f"] if world == 1 else ms_local / K / wl["f"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 (K/V/q), fp32 accumulate and output",
+        "data": "synthetic (seeded N(0,1) q/K/V, LogNormal K channel scale, needle blocks)",
+        "config": {"workload": args.workload, "description": wl["text"],
+                   "step": f"one ReSA cycle of {wl['f']} tokens through {wl['layers']} layers",
+                   "l2": "working set larger than L2 (cache > 126 MB per layer set); no flush",
+                   "parallelism": f"replicas x{world}", "graph": "one CUDA graph per cycle"},
+        "us_per_token": per_token_us,
+        "roofline": roofline,
+        "step_roofline": {"algorithmic_bytes_per_step": cyc_bytes / K, "achieved": step_gbs,
+                          "peak": hbm_peak, "unit": "GB/s", "frac": step_gbs / hbm_peak},
+        "rectify": rect,
+        "kernel_breakdown_us": bd,
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": K * w.launches_per_cycle(),
+        "cpu_baseline": cpu,
+        "device_error_word": code,
+        "setup_s": setup_s,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graphs
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def kernel_breakdown(w, stream, device, reps):
+    """Average device time per call of each entry point, on the workload's own
+    data, from CUDA-graph replays of one call per layer timed with events."""
+    import torch
+    R = w.R
+    c = w.cycles - 1
+    row = c * w.f + w.f - 2          # last decode step of the last cycle
+    rrow = c * w.f + w.f - 1
+
+    def timed(enqueue, calls):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                enqueue()
+            g.replay()
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        return 1e3 * e0.elapsed_time(e1) / (reps * calls)
+
+    n = w.layers
+    res = {}
+    res["sparse_decode_us"] = timed(lambda: [R.resa_sparse_decode(
+        w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.idx[l], w.cnt[l], w.max_topk, w.out[l],
+        None, w.ws) for l in range(n)], n)
+    scratch_idx = [torch.empty_like(t) for t in w.idx]
+    scratch_cnt = [torch.empty_like(t) for t in w.cnt]
+    res["select_blocks_us"] = timed(lambda: [R.resa_select_blocks(
+        w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.topk_ptr(row), w.max_topk, scratch_idx[l],
+        scratch_cnt[l], None, w.ws) for l in range(n)], n)
+    res["append_us"] = timed(lambda: [R.resa_append_token(
+        w.cfg, w.cache(l, row), w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l], w.ws)
+        for l in range(n)], n)
+    res["decode_step_us"] = timed(lambda: [R.resa_decode_step(
+        w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
+        w.topk_ptr(row), w.max_topk, w.out[l], None, w.idx[l], w.cnt[l], w.ws)
+        for l in range(n)], n)
+    res["rectify_us"] = timed(lambda: [R.resa_rectify_attention(
+        w.cfg, w.cache(l, rrow), w.f, w.qc[c, l], w.kc[c, l], w.vc[c, l], w.rout[l], None, w.ws)
+        for l in range(n)], n)
+    return res
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_resa(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,226 @@
+// Block key cache kernels: descriptor build / refresh, decode-token append and
+// rectification write-back (ReSA summary §3.2 "Block Key Cache", Eq. 3;
+// Algorithm 1 incremental update; §3.4.2 descriptor recomputation).
+//
+// One thread owns 8 consecutive channels (one 16-byte vector) of one
+// (page, kv head) row and scans the block's tokens in position order, so the
+// min / max keep the same bit pattern a sequential scan keeps.  A warp reads
+// whole 256-byte key rows: every load is a coalesced 16-byte vector.
+#include "resa_common.cuh"
+
+namespace resa {
+namespace {
+
+struct Bf16x8 {
+    uint16_t v[8];
+};
+
+__device__ __forceinline__ Bf16x8 unpack(uint4 x) {
+    Bf16x8 r;
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        r.v[2 * i] = (uint16_t)(w[i] & 0xffffu);
+        r.v[2 * i + 1] = (uint16_t)(w[i] >> 16);
+    }
+    return r;
+}
+__device__ __forceinline__ uint4 pack(const Bf16x8 &r) {
+    uint4 x;
+    x.x = (uint32_t)r.v[0] | ((uint32_t)r.v[1] << 16);
+    x.y = (uint32_t)r.v[2] | ((uint32_t)r.v[3] << 16);
+    x.z = (uint32_t)r.v[4] | ((uint32_t)r.v[5] << 16);
+    x.w = (uint32_t)r.v[6] | ((uint32_t)r.v[7] << 16);
+    return x;
+}
+__device__ __forceinline__ void fold(Bf16x8 &mn, Bf16x8 &mx, const Bf16x8 &x) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        mn.v[i] = bf_min(mn.v[i], x.v[i]);
+        mx.v[i] = bf_max(mx.v[i], x.v[i]);
+    }
+}
+
+__device__ __forceinline__ size_t kv_off(int page, int h, int slot, int c, int hkv, int d) {
+    return ((((size_t)page * hkv + h) * kBlock + slot) * d) / 8 + c;  // in uint4 units
+}
+__device__ __forceinline__ size_t desc_off(int page, int h, int which, int c, int hkv, int d) {
+    return ((((size_t)page * hkv + h) * 2 + which) * d) / 8 + c;  // in uint4 units
+}
+
+// grid (batch), block (hkv * d/8)
+__global__ void append_kernel(uint4 *__restrict__ K, uint4 *__restrict__ V,
+                              uint4 *__restrict__ desc, const int32_t *__restrict__ page_table,
+                              const int32_t *__restrict__ seq_len, const uint4 *__restrict__ k_new,
+                              const uint4 *__restrict__ v_new, int hkv, int d, int max_pages,
+                              int num_pages, uint32_t *err) {
+    const int b = blockIdx.x;
+    const int cpr = d / 8;  // 16-byte chunks per row
+    const int h = threadIdx.x / cpr, c = threadIdx.x % cpr;
+    if (h >= hkv) return;
+    const int L = seq_len[b];
+    if (L < 1 || L > max_pages * kBlock) {
+        if (threadIdx.x == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
+        return;
+    }
+    const int pos = L - 1;
+    const int page = page_table[(size_t)b * max_pages + pos / kBlock];
+    if (page < 0 || page >= num_pages) {
+        if (threadIdx.x == 0) set_error(err, RESA_DEVERR_PAGE);
+        return;
+    }
+    const int slot = pos % kBlock;
+    const size_t src = (((size_t)b * hkv + h) * d) / 8 + c;
+    const uint4 kx = k_new[src];
+    const uint4 vx = v_new[src];
+    K[kv_off(page, h, slot, c, hkv, d)] = kx;
+    V[kv_off(page, h, slot, c, hkv, d)] = vx;
+    uint4 *pmn = &desc[desc_off(page, h, 0, c, hkv, d)];
+    uint4 *pmx = &desc[desc_off(page, h, 1, c, hkv, d)];
+    if (slot == 0) {
+        *pmn = kx;
+        *pmx = kx;
+    } else {
+        Bf16x8 mn = unpack(*pmn), mx = unpack(*pmx);
+        fold(mn, mx, unpack(kx));
+        *pmn = pack(mn);
+        *pmx = pack(mx);
+    }
+}
+
+constexpr int kBuildThreads = 256;
+constexpr int kBuildPagesPerCta = 16;
+
+// grid (ceil(max_pages / kBuildPagesPerCta), batch), block kBuildThreads.
+// Rebuilds blocks [first, ceil(L / b)) of each sequence.
+__global__ void __launch_bounds__(kBuildThreads)
+    build_desc_kernel(const uint4 *__restrict__ K, uint4 *__restrict__ desc,
+                      const int32_t *__restrict__ page_table, const int32_t *__restrict__ seq_len,
+                      const int32_t *__restrict__ first_block, int hkv, int d, int max_pages,
+                      int num_pages, uint32_t *err) {
+    const int b = blockIdx.y;
+    const int cpr = d / 8;
+    const int tpp = hkv * cpr;                 // threads per page
+    const int ppp = kBuildThreads / tpp;       // pages per pass
+    const int sub = threadIdx.x / tpp;
+    const int h = (threadIdx.x % tpp) / cpr, c = threadIdx.x % cpr;
+    if (sub >= ppp) return;
+    const int L = seq_len[b];
+    if (L < 0 || L > max_pages * kBlock) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
+        return;
+    }
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int first = first_block ? max(0, first_block[b]) : 0;
+    const int blk0 = blockIdx.x * kBuildPagesPerCta;
+    for (int blk = blk0 + sub; blk < blk0 + kBuildPagesPerCta; blk += ppp) {
+        if (blk < first || blk >= nblk) continue;
+        const int page = page_table[(size_t)b * max_pages + blk];
+        if (page < 0 || page >= num_pages) {
+            if (h == 0 && c == 0) set_error(err, RESA_DEVERR_PAGE);
+            continue;
+        }
+        const int nt = min(kBlock, L - blk * kBlock);
+        uint4 x[kBlock];
+#pragma unroll
+        for (int t = 0; t < kBlock; ++t)
+            if (t < nt) x[t] = K[kv_off(page, h, t, c, hkv, d)];
+        Bf16x8 mn = unpack(x[0]), mx = mn;
+#pragma unroll
+        for (int t = 1; t < kBlock; ++t)
+            if (t < nt) fold(mn, mx, unpack(x[t]));
+        desc[desc_off(page, h, 0, c, hkv, d)] = pack(mn);
+        desc[desc_off(page, h, 1, c, hkv, d)] = pack(mx);
+    }
+}
+
+// grid (f / b + 2, batch), block (hkv * d/8).  Block (L-f)/b + blockIdx.x:
+// writes the chunk's fresh K/V into its positions >= L-f and rebuilds its
+// descriptor from the updated keys in the same pass.
+__global__ void rectify_writeback_kernel(uint4 *__restrict__ K, uint4 *__restrict__ V,
+                                         uint4 *__restrict__ desc,
+                                         const int32_t *__restrict__ page_table,
+                                         const int32_t *__restrict__ seq_len, int f,
+                                         const uint4 *__restrict__ k_new,
+                                         const uint4 *__restrict__ v_new, int hkv, int d,
+                                         int max_pages, int num_pages, uint32_t *err) {
+    const int b = blockIdx.y;
+    const int cpr = d / 8;
+    const int h = threadIdx.x / cpr, c = threadIdx.x % cpr;
+    if (h >= hkv) return;
+    const int L = seq_len[b];
+    if (L < 1 || L > max_pages * kBlock) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
+        return;
+    }
+    if (f > L) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) set_error(err, RESA_DEVERR_CHUNK);
+        return;
+    }
+    const int start = L - f;
+    const int blk = start / kBlock + blockIdx.x;
+    if (blk > (L - 1) / kBlock) return;
+    const int page = page_table[(size_t)b * max_pages + blk];
+    if (page < 0 || page >= num_pages) {
+        if (threadIdx.x == 0) set_error(err, RESA_DEVERR_PAGE);
+        return;
+    }
+    const int nt = min(kBlock, L - blk * kBlock);
+    Bf16x8 mn, mx;
+    for (int t = 0; t < nt; ++t) {
+        const int pos = blk * kBlock + t;
+        uint4 kx;
+        const size_t o = kv_off(page, h, t, c, hkv, d);
+        if (pos >= start) {
+            const size_t src = ((((size_t)b * f + (pos - start)) * hkv + h) * d) / 8 + c;
+            kx = k_new[src];
+            K[o] = kx;
+            V[o] = v_new[src];
+        } else {
+            kx = K[o];
+        }
+        const Bf16x8 x = unpack(kx);
+        if (t == 0) {
+            mn = x;
+            mx = x;
+        } else {
+            fold(mn, mx, x);
+        }
+    }
+    desc[desc_off(page, h, 0, c, hkv, d)] = pack(mn);
+    desc[desc_off(page, h, 1, c, hkv, d)] = pack(mx);
+}
+
+}  // namespace
+
+cudaError_t launch_append(const Shape &s, void *k, void *v, void *desc, const int32_t *page_table,
+                          const int32_t *seq_len, const void *k_new, const void *v_new,
+                          uint32_t *err, cudaStream_t st) {
+    append_kernel<<<s.batch, s.hkv * (s.d / 8), 0, st>>>(
+        (uint4 *)k, (uint4 *)v, (uint4 *)desc, page_table, seq_len, (const uint4 *)k_new,
+        (const uint4 *)v_new, s.hkv, s.d, s.max_pages, s.num_pages, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_build_descriptors(const Shape &s, const void *k, void *desc,
+                                     const int32_t *page_table, const int32_t *seq_len,
+                                     const int32_t *first_block, uint32_t *err, cudaStream_t st) {
+    dim3 grid((s.max_pages + kBuildPagesPerCta - 1) / kBuildPagesPerCta, s.batch);
+    build_desc_kernel<<<grid, kBuildThreads, 0, st>>>((const uint4 *)k, (uint4 *)desc, page_table,
+                                                      seq_len, first_block, s.hkv, s.d,
+                                                      s.max_pages, s.num_pages, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rectify_writeback(const Shape &s, void *k, void *v, void *desc,
+                                     const int32_t *page_table, const int32_t *seq_len, int f,
+                                     const void *k_new, const void *v_new, uint32_t *err,
+                                     cudaStream_t st) {
+    dim3 grid(f / kBlock + 2, s.batch);
+    rectify_writeback_kernel<<<grid, s.hkv * (s.d / 8), 0, st>>>(
+        (uint4 *)k, (uint4 *)v, (uint4 *)desc, page_table, seq_len, f, (const uint4 *)k_new,
+        (const uint4 *)v_new, s.hkv, s.d, s.max_pages, s.num_pages, err);
+    return cudaGetLastError();
+}
+
+}  // namespace resa

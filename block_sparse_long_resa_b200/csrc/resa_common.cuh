@@ -1,0 +1,252 @@
+// Internal definitions shared by the libresa translation units (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/resa.h"
+
+namespace resa {
+
+// ---------------------------------------------------------------------------
+// Fixed shape limits
+// ---------------------------------------------------------------------------
+constexpr int kBlock = 16;          // tokens per block / page
+constexpr int kMaxGroup = 16;       // query heads per kv head (one m16 MMA tile)
+constexpr int kMaxKvHeads = 8;
+constexpr int kTargetCtas = 4 * 148;  // split-KV sizing: ~4 resident CTAs per SM
+
+// Work units (sequence, kv head) x splits are bounded so the partial-result
+// region of the workspace depends on (batch, Hkv) only.
+inline int decode_max_splits(int batch, int hkv) {
+    int units = batch * hkv;
+    int s = (kTargetCtas + units - 1) / units;
+    return s < 1 ? 1 : (s > 128 ? 128 : s);
+}
+constexpr int kRectRowsPerTile = 64;    // query rows (chunk position x group head) per CTA
+inline int rect_row_tiles(int max_chunk, int group) {
+    int rows = max_chunk * group;
+    return (rows + kRectRowsPerTile - 1) / kRectRowsPerTile;
+}
+inline int rect_max_splits(int batch, int hkv, int row_tiles) {
+    int units = batch * hkv * (row_tiles > 0 ? row_tiles : 1);
+    int s = (2 * 148 + units - 1) / units;
+    return s < 1 ? 1 : (s > 64 ? 64 : s);
+}
+
+// ---------------------------------------------------------------------------
+// Workspace layout (byte offsets).  Every region except the rectification
+// partials depends only on (heads, d, batch, max_pages), so decode and
+// rectification calls of different chunk sizes find the same regions; the
+// rectification partials come last.
+// ---------------------------------------------------------------------------
+constexpr int kMaxRowTiles = 64;  // rectification row tiles per (sequence, kv head)
+
+struct WsLayout {
+    size_t err;          // uint32 error word
+    size_t dec_ticket;   // uint32 [B][Hkv]
+    size_t rect_ticket;  // uint32 [B][Hkv][kMaxRowTiles]
+    size_t scores;       // f32 [B][Hkv][max_pages]
+    size_t sel_idx;      // i32 [B][Hkv][max_pages + 1]
+    size_t sel_cnt;      // i32 [B][Hkv]
+    size_t dec_o;        // f32 [B][Hkv][dec_splits][kMaxGroup][d]
+    size_t dec_lse;      // f32 [B][Hkv][dec_splits][kMaxGroup]
+    size_t rect_o;       // f32 [B][Hkv][row_tiles][rect_splits][kRectRowsPerTile][d]
+    size_t rect_lse;     // f32 [B][Hkv][row_tiles][rect_splits][kRectRowsPerTile]
+    size_t total;
+    int dec_splits;
+    int row_tiles;
+    int rect_splits;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Layout for a call that rectifies chunks of `chunk` tokens (0: no rectification).
+inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int chunk) {
+    WsLayout w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    int g = hkv > 0 ? hq / hkv : 1;
+    w.dec_splits = decode_max_splits(batch, hkv);
+    w.row_tiles = chunk > 0 ? rect_row_tiles(chunk, g) : 0;
+    w.rect_splits = chunk > 0 ? rect_max_splits(batch, hkv, w.row_tiles) : 0;
+    size_t units = (size_t)batch * hkv;
+    w.err = take(256);
+    w.dec_ticket = take(units * 4);
+    w.rect_ticket = take(units * kMaxRowTiles * 4);
+    w.scores = take(units * max_pages * 4);
+    w.sel_idx = take(units * (max_pages + 1) * 4);
+    w.sel_cnt = take(units * 4);
+    w.dec_o = take(units * w.dec_splits * kMaxGroup * d * 4);
+    w.dec_lse = take(units * w.dec_splits * kMaxGroup * 4);
+    size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerTile;
+    w.rect_o = take(rect_rows * d * 4);
+    w.rect_lse = take(rect_rows * 4);
+    w.total = off;
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
+    if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t x) {
+    return __uint_as_float(((uint32_t)x) << 16);
+}
+__device__ __forceinline__ float bf_lo(uint32_t pair) { return __uint_as_float(pair << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t pair) { return __uint_as_float(pair & 0xffff0000u); }
+
+// Keep the earlier bit pattern on equality (matches a sequential scan).
+__device__ __forceinline__ uint16_t bf_min(uint16_t cur, uint16_t x) {
+    return bf16_bits_to_f32(x) < bf16_bits_to_f32(cur) ? x : cur;
+}
+__device__ __forceinline__ uint16_t bf_max(uint16_t cur, uint16_t x) {
+    return bf16_bits_to_f32(x) > bf16_bits_to_f32(cur) ? x : cur;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// mbarrier ------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: each try_wait suspends for a hardware-chosen interval; after
+// kMaxPolls unsuccessful polls the wait gives up and reports false.
+constexpr uint32_t kMaxPolls = 1u << 22;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kMaxPolls; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// TMA: 3-D tiled bulk tensor load into shared memory, completion on an mbarrier.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Warp-level tensor-core helpers (bf16 in, fp32 accumulate) ------------------
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Byte offset of (row, 16-byte chunk) inside a tile written by TMA with
+// CU_TENSOR_MAP_SWIZZLE_128B: rows are 128 bytes, chunk index XOR (row % 8).
+__device__ __forceinline__ uint32_t swz128(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device and process
+// (an idempotent attribute; later calls, e.g. during CUDA-graph capture, only
+// read a flag).
+template <typename Kernel>
+inline cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<int> (&done)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev].store(1, std::memory_order_release);
+    return e;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (defined in the kernel translation units)
+// ---------------------------------------------------------------------------
+struct Shape {
+    int hq, hkv, g, d, bs;
+    float sm_scale;
+    int batch, max_pages, num_pages;
+};
+
+cudaError_t launch_append(const Shape &s, void *k, void *v, void *desc, const int32_t *page_table,
+                          const int32_t *seq_len, const void *k_new, const void *v_new,
+                          uint32_t *err, cudaStream_t st);
+cudaError_t launch_build_descriptors(const Shape &s, const void *k, void *desc,
+                                     const int32_t *page_table, const int32_t *seq_len,
+                                     const int32_t *first_block, uint32_t *err, cudaStream_t st);
+cudaError_t launch_rectify_writeback(const Shape &s, void *k, void *v, void *desc,
+                                     const int32_t *page_table, const int32_t *seq_len, int f,
+                                     const void *k_new, const void *v_new, uint32_t *err,
+                                     cudaStream_t st);
+cudaError_t launch_score(const Shape &s, const void *desc, const int32_t *page_table,
+                         const int32_t *seq_len, const void *q, float *scores, uint32_t *err,
+                         cudaStream_t st);
+cudaError_t launch_select(const Shape &s, const float *scores, const int32_t *seq_len,
+                          const int32_t *topk, int max_topk, int32_t *block_idx,
+                          int32_t *block_cnt, uint32_t *err, cudaStream_t st);
+cudaError_t launch_sparse_decode(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                 const int32_t *page_table, const int32_t *seq_len, const void *q,
+                                 const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
+                                 int splits, float *part_o, float *part_lse, uint32_t *tickets,
+                                 float *out, float *lse, uint32_t *err, cudaStream_t st);
+cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap &kmap,
+                                     const CUtensorMap &vmap, const int32_t *page_table,
+                                     const int32_t *seq_len, int f, const void *q_chunk,
+                                     int row_tiles, int splits, float *part_o, float *part_lse,
+                                     uint32_t *tickets, float *out, float *lse, uint32_t *err,
+                                     cudaStream_t st);
+
+}  // namespace resa

@@ -240,6 +240,33 @@ class OracleCache:
                              _ptr(lse), self.B, self.hq, self.hkv, self.d, self.bs, self.max_pages)
         return out, lse
 
+    def rectify_rows(self, q_chunk, k_new, v_new, seq_len, f: int, rows,
+                     sm_scale: Optional[float] = None):
+        """Rectification evaluated on a sample of chunk rows: the same three
+        steps as rectify() (write-back, descriptor refresh of the touched
+        blocks, causal attention), with the attention of chunk row r taken as
+        dense attention of q_chunk[:, r] over positions 0 .. L-f+r.  Returns
+        {r: (out [B][hq][d], lse [B][hq])}."""
+        kn, vn, sl = bits(k_new), bits(v_new), _i32(seq_len)
+        for b in range(self.B):
+            L = int(sl[b])
+            if f > L:
+                continue  # a chunk longer than the sequence leaves it untouched
+            for r in range(f):
+                pos = L - f + r
+                page = self.page_table[b, pos // self.bs]
+                self.K[page, :, pos % self.bs] = kn[b, r]
+                self.V[page, :, pos % self.bs] = vn[b, r]
+        ok = sl >= f
+        self.build_descriptors(np.where(ok, sl, 0).astype(np.int32),
+                               np.where(ok, (sl - f) // self.bs, 0).astype(np.int32))
+        qc = bits(q_chunk)
+        res = {}
+        for r in rows:
+            res[int(r)] = self.dense_attention(qc[:, r], np.maximum(sl - f + int(r) + 1, 0),
+                                               sm_scale)
+        return res
+
     # Views used by tests ----------------------------------------------------
     def keys(self, b: int, h: int, L: int) -> np.ndarray:
         """Keys of sequence b, kv head h, positions 0 .. L-1 as float32 [L][d]."""

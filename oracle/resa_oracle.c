@@ -289,6 +289,7 @@ void oracle_rectify(const uint16_t *q_chunk, const uint16_t *k_new, const uint16
     int g = hq / hkv;
     for (int b = 0; b < B; ++b) {
         int L = seq_len[b];
+        if (f > L) continue; /* a chunk longer than the sequence leaves it untouched */
         for (int r = 0; r < f; ++r)
             for (int h = 0; h < hkv; ++h)
                 for (int j = 0; j < d; ++j) {
@@ -306,6 +307,7 @@ void oracle_rectify(const uint16_t *q_chunk, const uint16_t *k_new, const uint16
         for (int r = 0; r < f; ++r)
             for (int qh = 0; qh < hq; ++qh) {
                 int L = seq_len[b];
+                if (f > L) continue;
                 int last = L - f + r;
                 int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)(last + 1));
                 for (int t = 0; t <= last; ++t) pos[t] = t;

@@ -1,0 +1,439 @@
+"""CUDA path (through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Bars: descriptors, written K/V and block sets bit-exact (block sets may differ
+only on blocks whose oracle fp32 score is within 1e-6 relative of the k-th
+score); attention outputs within 2e-3 absolute (bf16 K/V, fp32 accumulation);
+log-sum-exp within 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_resa_b200 import inputs
+from block_sparse_long_resa_b200 import resa as R
+from block_sparse_long_resa_b200.cache import LayerCache, workspace
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+OUT_ATOL = 2e-3
+LSE_ATOL = 1e-3
+TIE_REL = 1e-6
+
+
+def oracle_of(p, desc=None):
+    return O.OracleCache(p.k_cache, p.v_cache, p.page_table, p.num_q_heads, p.num_kv_heads,
+                         p.head_dim, p.block_size, desc=desc)
+
+
+def cfg_of(p):
+    return R.make_config(p.num_q_heads, p.num_kv_heads, p.head_dim, p.block_size)
+
+
+def setup_layer(p, dev, max_chunk=64):
+    cfg = cfg_of(p)
+    lc = LayerCache.from_problem(p, dev)
+    ws = workspace(cfg, lc.batch, lc.max_pages, max_chunk, dev)
+    R.resa_build_descriptors(cfg, lc.struct(), None, ws)
+    return cfg, lc, ws
+
+
+def assert_no_device_error(ws):
+    torch.cuda.synchronize()
+    assert R.resa_check_device_status(ws, raise_on_error=False) == 0
+
+
+def bits_of(t):
+    return O.bits(t)
+
+
+def check_block_sets(gidx, gcnt, oidx, ocnt, oscores, topk, L, bs):
+    """Returns True when the sets are identical; asserts differences are near-ties."""
+    same = True
+    B, H = ocnt.shape
+    for b in range(B):
+        M = (int(L[b]) - 1) // bs
+        k = min(int(topk[b]), M)
+        for h in range(H):
+            assert int(gcnt[b, h]) == int(ocnt[b, h]) == k + 1
+            g = gidx[b, h, :k + 1].tolist()
+            o = oidx[b, h, :k + 1].tolist()
+            assert g[-1] == o[-1] == M
+            assert g[:-1] == sorted(set(g[:-1])), "GPU list must be ascending and unique"
+            diff = set(g[:-1]) ^ set(o[:-1])
+            if diff:
+                same = False
+                s = oscores[b, h, :M].astype(np.float64)
+                sk = np.sort(s)[::-1][k - 1]
+                for i in diff:
+                    assert abs(s[i] - sk) <= TIE_REL * abs(sk), (b, h, i, s[i], sk)
+    return same
+
+
+# --------------------------------------------------------------------------- cases
+
+TINY = dict(seed=1, batch=1, num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16,
+            ctx_lens=[2048], topk=[16])
+QWEN32K = dict(seed=2, batch=1, num_q_heads=28, num_kv_heads=4, head_dim=128, block_size=16,
+               ctx_lens=[32768])  # top-k = 10% = 205
+RAGGED = dict(seed=3, batch=5, num_q_heads=28, num_kv_heads=4, head_dim=128, block_size=16,
+              ctx_lens=[1, 15, 16, 300, 5003], topk=[4, 16, 16, 7, 500], paged=True)
+RAGGED64 = dict(seed=4, batch=3, num_q_heads=8, num_kv_heads=1, head_dim=64, block_size=16,
+                ctx_lens=[33, 257, 1111], topk=[100, 3, 60], paged=True)
+
+
+def make(case, device="cpu", **over):
+    kw = dict(case)
+    kw.update(over)
+    seed = kw.pop("seed")
+    B = kw.pop("batch")
+    return inputs.make_decode_problem(seed, B, kw.pop("num_q_heads"), kw.pop("num_kv_heads"),
+                                      kw.pop("head_dim"), kw.pop("block_size"),
+                                      kw.pop("ctx_lens"), device=device, **kw)
+
+
+@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED, RAGGED64], ids=["tiny", "qwen32k",
+                                                                         "ragged", "ragged64"])
+def test_build_descriptors_bit_exact(cuda_device, case):
+    p = make(case)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+
+
+def test_build_descriptors_from_first_block(cuda_device):
+    p = make(RAGGED)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    lc.desc.zero_()
+    first = torch.tensor([0, 0, 1, 7, 300], dtype=torch.int32)
+    R.resa_build_descriptors(cfg, lc.struct(), first.to(cuda_device), ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len, first)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+
+
+@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED, RAGGED64], ids=["tiny", "qwen32k",
+                                                                         "ragged", "ragged64"])
+def test_decode_step_matches_oracle(cuda_device, case):
+    p = make(case)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L.to(cuda_device))
+    max_topk = int(p.topk.max())
+    B, Hq, Hkv, d = p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=cuda_device)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=cuda_device)
+    idx = torch.full((B, Hkv, max_topk + 1), -1, dtype=torch.int32, device=cuda_device)
+    cnt = torch.zeros(B, Hkv, dtype=torch.int32, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_decode_step(cfg, lc.struct(), dev(p.q), dev(p.k_new), dev(p.v_new), dev(p.topk),
+                       max_topk, out, lse, idx, cnt, ws)
+    assert_no_device_error(ws)
+
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    r = o.decode_step(p.q, p.k_new, p.v_new, p.topk, L, max_topk)
+    # append: K, V and descriptors bit-exact
+    np.testing.assert_array_equal(bits_of(lc.k), o.K)
+    np.testing.assert_array_equal(bits_of(lc.v), o.V)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+    gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    same = check_block_sets(gidx, gcnt, r["block_idx"], r["block_cnt"], r["scores"], p.topk, L,
+                            p.block_size)
+    ref_out, ref_lse = (r["out"], r["lse"]) if same else o.sparse_attention(p.q, gidx, gcnt, L)
+    np.testing.assert_allclose(out.cpu().numpy(), ref_out, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+    # the needles are found
+    for b in range(B):
+        M = (int(L[b]) - 1) // p.block_size
+        if M - 1 >= 4 and int(p.topk[b]) >= 16:
+            for h in range(Hkv):
+                sel = set(gidx[b, h, :gcnt[b, h]].tolist())
+                assert set(p.needle_blocks[b, h].tolist()) <= sel
+
+
+@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED], ids=["tiny", "qwen32k", "ragged"])
+def test_select_blocks_scores(cuda_device, case):
+    p = make(case)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L.to(cuda_device))
+    R.resa_append_token(cfg, lc.struct(), p.k_new.to(cuda_device), p.v_new.to(cuda_device), ws)
+    max_topk = int(p.topk.max())
+    B, Hkv = p.batch, p.num_kv_heads
+    idx = torch.full((B, Hkv, max_topk + 1), -1, dtype=torch.int32, device=cuda_device)
+    cnt = torch.zeros(B, Hkv, dtype=torch.int32, device=cuda_device)
+    scores = torch.full((B, Hkv, lc.max_pages), float("nan"), device=cuda_device)
+    R.resa_select_blocks(cfg, lc.struct(), p.q.to(cuda_device), p.topk.to(cuda_device), max_topk,
+                         idx, cnt, scores, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    o.append(p.k_new, p.v_new, L)
+    sc = o.block_scores(o.pooled_query(p.q), L)
+    oidx, ocnt = o.select(sc, p.topk, L, max_topk)
+    gs = scores.cpu().numpy()
+    for b in range(B):
+        M = (int(L[b]) - 1) // p.block_size
+        np.testing.assert_allclose(gs[b, :, :M], sc[b, :, :M], rtol=2e-6, atol=2e-6)
+    check_block_sets(idx.cpu().numpy(), cnt.cpu().numpy(), oidx, ocnt, sc, p.topk, L,
+                     p.block_size)
+
+
+def test_select_exact_ties_and_edges(cuda_device):
+    """All keys equal: every score ties, the lowest indices win."""
+    p = make(RAGGED64, seed=9, ctx_lens=[333, 257, 1999])
+    p.k_cache[:] = 0.5
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    lc.seq_len.copy_((p.ctx_len + 1).to(cuda_device))
+    topk = torch.tensor([5, 0, 10**6], dtype=torch.int32)
+    max_topk = 80
+    idx = torch.full((3, 1, max_topk + 1), -1, dtype=torch.int32, device=cuda_device)
+    cnt = torch.zeros(3, 1, dtype=torch.int32, device=cuda_device)
+    R.resa_select_blocks(cfg, lc.struct(), p.q.to(cuda_device), topk.to(cuda_device), max_topk,
+                         idx, cnt, None, ws)
+    code = R.resa_check_device_status(ws, raise_on_error=False)
+    assert code == R.DEVERR_TOPK       # sequence 2 asks for more than max_topk
+    idx, cnt = idx.cpu(), cnt.cpu()
+    L = (p.ctx_len + 1).tolist()
+    M = [(x - 1) // 16 for x in L]
+    assert idx[0, 0, :cnt[0, 0]].tolist() == [0, 1, 2, 3, 4, M[0]]
+    assert idx[1, 0, :cnt[1, 0]].tolist() == [M[1]]
+    assert idx[2, 0, :cnt[2, 0]].tolist() == list(range(max_topk)) + [M[2]]
+
+
+def test_sparse_decode_given_blocks(cuda_device):
+    """Attention over caller-chosen blocks, including a partial current block
+    and a block id outside the sequence (skipped, error bit set)."""
+    p = make(QWEN32K, ctx_lens=[32768 + 5])
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len.clone()
+    M = (int(L[0]) - 1) // 16
+    rng = np.random.default_rng(5)
+    blocks = np.sort(rng.choice(M, size=300, replace=False)).astype(np.int32)
+    idx = np.full((1, 4, 302), -1, dtype=np.int32)
+    cnt = np.full((1, 4), 301, dtype=np.int32)
+    for h in range(4):
+        idx[0, h, :300] = np.sort(rng.choice(M, size=300, replace=False))
+        idx[0, h, 300] = M
+    out = torch.empty(1, 28, 128, device=cuda_device)
+    lse = torch.empty(1, 28, device=cuda_device)
+    R.resa_sparse_decode(cfg, lc.struct(), p.q.to(cuda_device), torch.from_numpy(idx).to(cuda_device),
+                         torch.from_numpy(cnt).to(cuda_device), 301, out, lse, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    ref, ref_lse = o.sparse_attention(p.q, idx, cnt, L)
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+    # an out-of-range block id is skipped and reported
+    idx[0, 0, 0] = M + 50
+    R.resa_sparse_decode(cfg, lc.struct(), p.q.to(cuda_device), torch.from_numpy(idx).to(cuda_device),
+                         torch.from_numpy(cnt).to(cuda_device), 301, out, lse, ws)
+    code = R.resa_check_device_status(ws, raise_on_error=False)
+    assert code & R.DEVERR_BLOCK
+
+
+def test_all_blocks_equals_dense(cuda_device):
+    p = make(RAGGED)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L.to(cuda_device))
+    B = p.batch
+    max_topk = int((L.max() - 1) // 16)
+    topk = torch.full((B,), 10**6, dtype=torch.int32)
+    out = torch.empty(B, 28, 128, device=cuda_device)
+    idx = torch.empty(B, 4, max_topk + 1, dtype=torch.int32, device=cuda_device)
+    cnt = torch.empty(B, 4, dtype=torch.int32, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_decode_step(cfg, lc.struct(), dev(p.q), dev(p.k_new), dev(p.v_new), dev(topk),
+                       max_topk, out, None, idx, cnt, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.append(p.k_new, p.v_new, L)
+    dense, _ = o.dense_attention(p.q, L)
+    np.testing.assert_allclose(out.cpu().numpy(), dense, rtol=0, atol=OUT_ATOL)
+
+
+@pytest.mark.parametrize("shape,ctx,f", [
+    ((4, 2, 64), [2049], 32),
+    ((28, 4, 128), [4096, 1000], 32),
+    ((28, 4, 128), [777], 13),
+    ((8, 1, 64), [40, 64, 300], 40),
+], ids=["tiny", "qwen-aligned", "qwen-unaligned", "whole-seq"])
+def test_rectify_matches_oracle(cuda_device, shape, ctx, f):
+    hq, hkv, d = shape
+    p = inputs.make_decode_problem(20 + f, len(ctx), hq, hkv, d, 16, ctx, paged=True,
+                                   needles=0, topk=[1] * len(ctx))
+    cfg, lc, ws = setup_layer(p, cuda_device, max_chunk=f)
+    L = p.ctx_len.clone()
+    qc, kc, vc = inputs.make_rectify_chunk(f, len(ctx), f, hq, hkv, d)
+    B = len(ctx)
+    out = torch.empty(B, f, hq, d, device=cuda_device)
+    lse = torch.empty(B, f, hq, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_rectify_attention(cfg, lc.struct(), f, dev(qc), dev(kc), dev(vc), out, lse, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(L)
+    ref, ref_lse = o.rectify(qc, kc, vc, L, f)
+    np.testing.assert_array_equal(bits_of(lc.k), o.K)
+    np.testing.assert_array_equal(bits_of(lc.v), o.V)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+
+
+def test_rectify_chunk_longer_than_sequence_is_reported(cuda_device):
+    p = inputs.make_decode_problem(31, 2, 4, 2, 64, 16, [10, 100], needles=0, topk=[1, 1])
+    cfg, lc, ws = setup_layer(p, cuda_device, max_chunk=32)
+    qc, kc, vc = inputs.make_rectify_chunk(31, 2, 32, 4, 2, 64)
+    out = torch.zeros(2, 32, 4, 64, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_rectify_attention(cfg, lc.struct(), 32, dev(qc), dev(kc), dev(vc), out, None, ws)
+    code = R.resa_check_device_status(ws, raise_on_error=False)
+    assert code & R.DEVERR_CHUNK
+    # the valid sequence was still rectified
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    res = o.rectify_rows(qc, kc, vc, p.ctx_len, 32, [0, 31])
+    for r, (ref, _) in res.items():
+        np.testing.assert_allclose(out[1, r].cpu().numpy(), ref[1], rtol=0, atol=OUT_ATOL)
+
+
+def test_decode_loop_with_rectification(cuda_device):
+    """A few ReSA cycles (f = 8): sparse decode steps appending tokens, then a
+    rectification of the last f tokens; every step checked against the oracle."""
+    p = make(QWEN32K, batch=2, ctx_lens=[3000, 1234], topk=[20, 16], paged=True, seed=44)
+    cfg, lc, ws = setup_layer(p, cuda_device, max_chunk=8)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    f, B = 8, 2
+    L = p.ctx_len.clone()
+    dev = lambda t: t.to(cuda_device)
+    out = torch.empty(B, 28, 128, device=cuda_device)
+    idx = torch.empty(B, 4, 21, dtype=torch.int32, device=cuda_device)
+    cnt = torch.empty(B, 4, dtype=torch.int32, device=cuda_device)
+    for cycle in range(2):
+        for s in range(f - 1):
+            q, kn, vn = inputs.make_step_tokens(44, cycle * f + s, B, 28, 4, 128, p.k_scale)
+            L = L + 1
+            lc.seq_len.copy_(dev(L))
+            R.resa_decode_step(cfg, lc.struct(), dev(q), dev(kn), dev(vn), dev(p.topk), 20, out,
+                               None, idx, cnt, ws)
+            r = o.decode_step(q, kn, vn, p.topk, L, 20)
+            gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+            same = check_block_sets(gidx, gcnt, r["block_idx"], r["block_cnt"], r["scores"],
+                                    p.topk, L, 16)
+            ref = r["out"] if same else o.sparse_attention(q, gidx, gcnt, L)[0]
+            np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+        L = L + 1
+        lc.seq_len.copy_(dev(L))
+        qc, kc, vc = inputs.make_rectify_chunk(100 + cycle, B, f, 28, 4, 128)
+        rout = torch.empty(B, f, 28, 128, device=cuda_device)
+        R.resa_rectify_attention(cfg, lc.struct(), f, dev(qc), dev(kc), dev(vc), rout, None, ws)
+        ref, _ = o.rectify(qc, kc, vc, L, f)
+        np.testing.assert_allclose(rout.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+        np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+    assert_no_device_error(ws)
+
+
+# --------------------------------------------------------------------------- full sizes
+
+def test_full_size_256k_layer(cuda_device):
+    """One layer of the 256K long-context decode workload (28 q / 4 kv heads,
+    d 128, 262144-token cache, top-k 1638 + current block), in the launch
+    configuration the benchmark times; the oracle computes every output."""
+    p = inputs.make_decode_problem(7, 1, 28, 4, 128, 16, [262144], device=cuda_device)
+    cfg = cfg_of(p)
+    lc = LayerCache(k=p.k_cache, v=p.v_cache,
+                    desc=torch.zeros(p.num_pages, 4, 2, 128, dtype=torch.bfloat16,
+                                     device=cuda_device),
+                    page_table=p.page_table, seq_len=p.ctx_len.clone())
+    ws = workspace(cfg, 1, lc.max_pages, 32, cuda_device)
+    R.resa_build_descriptors(cfg, lc.struct(), None, ws)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L)
+    k = int(p.topk[0])
+    assert k == 1638
+    out = torch.empty(1, 28, 128, device=cuda_device)
+    idx = torch.empty(1, 4, k + 1, dtype=torch.int32, device=cuda_device)
+    cnt = torch.empty(1, 4, dtype=torch.int32, device=cuda_device)
+    R.resa_decode_step(cfg, lc.struct(), p.q, p.k_new, p.v_new, p.topk, k, out, None, idx, cnt,
+                       ws)
+    assert_no_device_error(ws)
+    cpu = lambda t: t.cpu()
+    o = O.OracleCache(cpu(p.k_cache), cpu(p.v_cache), cpu(p.page_table), 28, 4, 128, 16)
+    o.build_descriptors(cpu(p.ctx_len))
+    r = o.decode_step(cpu(p.q), cpu(p.k_new), cpu(p.v_new), cpu(p.topk), cpu(L), k)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+    gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    same = check_block_sets(gidx, gcnt, r["block_idx"], r["block_cnt"], r["scores"],
+                            cpu(p.topk), cpu(L), 16)
+    ref = r["out"] if same else o.sparse_attention(cpu(p.q), gidx, gcnt, cpu(L))[0]
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+
+
+def test_full_size_rectification_sampled_rows(cuda_device):
+    """Rectification at the decode-loop workload's size (batch 4, 65536-token
+    cache, f = 32, 28 q / 4 kv heads): every output row computed, sampled rows
+    compared with the oracle."""
+    B, f = 4, 32
+    p = inputs.make_decode_problem(8, B, 28, 4, 128, 16, [65536] * B, device=cuda_device)
+    cfg = cfg_of(p)
+    lc = LayerCache(k=p.k_cache, v=p.v_cache,
+                    desc=torch.zeros(p.num_pages, 4, 2, 128, dtype=torch.bfloat16,
+                                     device=cuda_device),
+                    page_table=p.page_table, seq_len=p.ctx_len.clone())
+    ws = workspace(cfg, B, lc.max_pages, f, cuda_device)
+    R.resa_build_descriptors(cfg, lc.struct(), None, ws)
+    kc0, vc0 = p.k_cache.cpu(), p.v_cache.cpu()
+    qc, kc, vc = inputs.make_rectify_chunk(8, B, f, 28, 4, 128, device=cuda_device)
+    out = torch.empty(B, f, 28, 128, device=cuda_device)
+    R.resa_rectify_attention(cfg, lc.struct(), f, qc, kc, vc, out, None, ws)
+    assert_no_device_error(ws)
+    o = O.OracleCache(kc0, vc0, p.page_table.cpu(), 28, 4, 128, 16)
+    o.build_descriptors(p.ctx_len.cpu())
+    rows = [0, 13, 31]
+    res = o.rectify_rows(qc.cpu(), kc.cpu(), vc.cpu(), p.ctx_len.cpu(), f, rows)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+    for r in rows:
+        np.testing.assert_allclose(out[:, r].cpu().numpy(), res[r][0], rtol=0, atol=OUT_ATOL)
+    assert torch.isfinite(out).all()
+
+
+def test_full_size_continuous_batching(cuda_device):
+    """Continuous-batching workload: 32 sequences with lengths uniform in
+    [8192, 131072], random physical page order, top-k 10% per sequence."""
+    lens = inputs.continuous_batch_lengths(9, 32, 8192, 131072)
+    p = inputs.make_decode_problem(9, 32, 28, 4, 128, 16, lens, paged=True, device=cuda_device,
+                                   reserve_tokens=16)
+    cfg = cfg_of(p)
+    lc = LayerCache(k=p.k_cache, v=p.v_cache,
+                    desc=torch.zeros(p.num_pages, 4, 2, 128, dtype=torch.bfloat16,
+                                     device=cuda_device),
+                    page_table=p.page_table, seq_len=p.ctx_len.clone())
+    ws = workspace(cfg, 32, lc.max_pages, 0, cuda_device)
+    R.resa_build_descriptors(cfg, lc.struct(), None, ws)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L)
+    max_topk = int(p.topk.max())
+    out = torch.empty(32, 28, 128, device=cuda_device)
+    idx = torch.empty(32, 4, max_topk + 1, dtype=torch.int32, device=cuda_device)
+    cnt = torch.empty(32, 4, dtype=torch.int32, device=cuda_device)
+    R.resa_decode_step(cfg, lc.struct(), p.q, p.k_new, p.v_new, p.topk, max_topk, out, None, idx,
+                       cnt, ws)
+    assert_no_device_error(ws)
+    cpu = lambda t: t.cpu()
+    o = O.OracleCache(cpu(p.k_cache), cpu(p.v_cache), cpu(p.page_table), 28, 4, 128, 16)
+    o.build_descriptors(cpu(p.ctx_len))
+    r = o.decode_step(cpu(p.q), cpu(p.k_new), cpu(p.v_new), cpu(p.topk), cpu(L), max_topk)
+    gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    same = check_block_sets(gidx, gcnt, r["block_idx"], r["block_cnt"], r["scores"],
+                            cpu(p.topk), cpu(L), 16)
+    ref = r["out"] if same else o.sparse_attention(cpu(p.q), gidx, gcnt, cpu(L))[0]
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)

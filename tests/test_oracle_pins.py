@@ -376,3 +376,25 @@ def test_decode_step_with_all_blocks_equals_last_rectify_row():
     b_.build_descriptors(L - 1)
     r = b_.decode_step(qc[:, f - 1], kc[:, f - 1], vc[:, f - 1], [10**6] * p.batch, L, 64)
     np.testing.assert_allclose(r["out"], out_r[:, f - 1], rtol=0, atol=1e-12)
+
+
+def test_rectify_rows_equals_rectify_and_skips_short_sequences():
+    p = small_problem(seed=15, d=32, bs=8, ctx=(90, 20), hq=4, hkv=2)
+    f = 24
+    qc, kc, vc = inputs.make_rectify_chunk(15, p.batch, f, 4, 2, 32)
+    a = oracle_of(p)
+    a.build_descriptors(p.ctx_len)
+    out, lse = a.rectify(qc, kc, vc, p.ctx_len, f)
+    b_ = oracle_of(p)
+    b_.build_descriptors(p.ctx_len)
+    res = b_.rectify_rows(qc, kc, vc, p.ctx_len, f, [0, 7, 23])
+    np.testing.assert_array_equal(a.K, b_.K)
+    np.testing.assert_array_equal(a.desc, b_.desc)
+    for r, (o_r, l_r) in res.items():
+        np.testing.assert_allclose(o_r[0], out[0, r], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l_r[0], lse[0, r], rtol=0, atol=1e-12)
+    # sequence 1 (L = 20 < f) is left untouched by both
+    fresh = oracle_of(p)
+    for blk in range(3):
+        page = fresh.page_table[1, blk]
+        np.testing.assert_array_equal(a.K[page], fresh.K[page])
