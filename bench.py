@@ -41,6 +41,9 @@ WORKLOADS = {
                      text="long-context decode: 28 layers x (28 q / 4 kv heads, d 128), batch 1, "
                           "262144-token bf16 cache, block 16, top-k 10% (1638) + current block, "
                           "ReSA cycle f=32 (31 sparse decode steps + 1 dense rectification)"),
+    "layer256k": dict(layers=1, batch=1, hq=28, hkv=4, d=128, ctx=[262144], f=32, paged=False,
+                      text="one layer of the long-context decode workload (28 q / 4 kv, d 128), "
+                           "262144-token cache, top-k 10% + current block, ReSA cycle f=32"),
     "loop64k": dict(layers=1, batch=4, hq=28, hkv=4, d=128, ctx=[65536] * 4, f=32, paged=False,
                     text="ReSA decode loop: 1 layer (28 q / 4 kv, d 128), batch 4, 65536-token "
                          "cache, top-k 10%, 31 sparse decode steps + 1 rectification of 32"),

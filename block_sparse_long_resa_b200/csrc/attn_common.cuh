@@ -14,8 +14,8 @@ namespace resa {
 template <int D>
 struct RowState {
     float m[2];          // running max of the base-2 logits
-    float l[2];          // this lane's share of the running sum of the bf16-rounded weights
-    float lx[2];         // the same sum over the unrounded weights (for the log-sum-exp)
+    float l[2];          // this lane's share of the running sum of the weights
+    float lx[2];         // copy of l kept for the log-sum-exp
     float acc[D / 8][4]; // O accumulators: n-tile j covers channels 8j .. 8j+7
     __device__ __forceinline__ void init() {
         m[0] = m[1] = -INFINITY;
@@ -91,25 +91,24 @@ __device__ __forceinline__ void attend_tile16(RowState<D> &st, const uint32_t (&
         alpha[r] = exp2f(st.m[r] - base[r]);
         st.m[r] = mnew;
     }
-    uint32_t pa[4];
-    float psum[2] = {0.f, 0.f}, pxsum[2] = {0.f, 0.f};
+    // P enters the P.V MMA as bf16 hi + lo parts (two MMAs), so the weights
+    // keep ~16 significant bits: rows that see only a few tokens stay within
+    // the fp32-accumulation error budget.
+    uint32_t pa[4], pl[4];
+    float psum[2] = {0.f, 0.f};
 #pragma unroll
     for (int n = 0; n < 2; ++n) {
         const float p0 = exp2f(s[n][0] - base[0]), p1 = exp2f(s[n][1] - base[0]);
         const float p2 = exp2f(s[n][2] - base[1]), p3 = exp2f(s[n][3] - base[1]);
-        pa[2 * n] = pack_bf16(p0, p1);
-        pa[2 * n + 1] = pack_bf16(p2, p3);
-        // O is normalised by the sum of the same bf16-rounded weights the P.V
-        // MMA uses; the log-sum-exp takes the unrounded weights.
-        psum[0] += bf_lo(pa[2 * n]) + bf_hi(pa[2 * n]);
-        psum[1] += bf_lo(pa[2 * n + 1]) + bf_hi(pa[2 * n + 1]);
-        pxsum[0] += p0 + p1;
-        pxsum[1] += p2 + p3;
+        split_bf16(p0, p1, pa[2 * n], pl[2 * n]);
+        split_bf16(p2, p3, pa[2 * n + 1], pl[2 * n + 1]);
+        psum[0] += p0 + p1;
+        psum[1] += p2 + p3;
     }
     st.l[0] = st.l[0] * alpha[0] + psum[0];
     st.l[1] = st.l[1] * alpha[1] + psum[1];
-    st.lx[0] = st.lx[0] * alpha[0] + pxsum[0];
-    st.lx[1] = st.lx[1] * alpha[1] + pxsum[1];
+    st.lx[0] = st.l[0];
+    st.lx[1] = st.l[1];
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) {
         st.acc[j][0] *= alpha[0];
@@ -129,6 +128,8 @@ __device__ __forceinline__ void attend_tile16(RowState<D> &st, const uint32_t (&
             ldmatrix_x4_trans(r, v_tile + swz128(row, (dim % 64) / 8));
             mma_bf16_16816(st.acc[2 * np], pa, r[0], r[1]);
             mma_bf16_16816(st.acc[2 * np + 1], pa, r[2], r[3]);
+            mma_bf16_16816(st.acc[2 * np], pl, r[0], r[1]);
+            mma_bf16_16816(st.acc[2 * np + 1], pl, r[2], r[3]);
         }
     }
 }

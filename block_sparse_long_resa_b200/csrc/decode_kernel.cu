@@ -1,39 +1,146 @@
-// Group block-sparse split-KV decode (GBSA, ReSA summary §3.4.1 Eq. 2; kernel
-// design §3.4.4 / Algorithm 2, re-done for sm_100a).
+// Group block-sparse split-KV decode (GBSA, ReSA summary §3.4.1 Eq. 2; the
+// split-execution kernel of §3.4.4, redone for sm_100a).
 //
-// Grid (splits, Hkv, batch).  CTA (split s, kv head h, sequence b) takes the
-// s-th contiguous slice of the group's selected block list; each of its four
-// warps takes every fourth block of the slice and keeps its own online-softmax
-// state for the group's g query heads (rows of one m16 MMA tile), so the K/V
-// of a block are fetched once for the whole group.  A warp streams its blocks
-// through a private ring of kStages shared-memory stages: lane 0 issues two
-// 3-D TMA loads per block (K and V, each one (page, head) tile of 16 x D bf16,
-// 128-byte swizzled) that complete on the stage's mbarrier.
+// Grid (splits, Hkv, batch), one 8-warp CTA per SM.  CTA (s, h, b) takes the
+// s-th contiguous slice of the group's selected block list; warp w takes
+// every eighth block of the slice and keeps its own online-softmax state for
+// the group's g query heads, so the K/V of a block are fetched once for the
+// whole group.  Each warp streams its blocks through a private ring of
+// kStages shared-memory stages: lane 0 issues two 3-D TMA loads per block
+// (the (page, head) K and V tiles of 16 x D bf16, 128-byte swizzled) that
+// complete on the stage's mbarrier.  Block ids and pages of the slice are
+// staged in shared memory once, up front.
 //
-// The CTA merges its warps' states, then either writes the final output (one
-// split) or a partial (o, lse) and takes an atomic ticket; the CTA that draws
-// the last ticket of its (sequence, kv head) merges every split's partial and
-// resets the ticket.  No CTA waits on another.
+// The MMAs run with the operands swapped, S^T = K Q^T and O^T = V^T P^T
+// (bf16 m16n8k16, fp32 accumulate), so the g <= 8 heads of a group fill the
+// N = 8 side instead of wasting 9 of 16 M rows; P^T is transposed in
+// registers with movmatrix and enters the P.V MMA as bf16 hi + lo parts.
+//
+// The CTA merges its warps, then writes the final output (one split) or a
+// partial (o, log2-sum-exp) and draws an atomic ticket; the CTA drawing the
+// last ticket of its (sequence, kv head) merges the splits with vectorised,
+// batched loads and resets the ticket.  No CTA waits on another.
 #include "attn_common.cuh"
 
 namespace resa {
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 3;
 
 template <int D>
 struct DecodeSmem {
-    static constexpr int kTileBytes = kBlock * D * 2;               // one K or V tile
+    static constexpr int kTileBytes = kBlock * D * 2;  // one K or V tile
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
     static constexpr int kMergeBytes = kWarps * kMaxGroup * (D + 3) * 4;
     static constexpr int kBytes = (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes) + 1024;
 };
 
-template <int D>
-__global__ void __launch_bounds__(kThreads)
+// Per-warp attention state in the swapped layout: lane holds heads
+// nt*8 + 2*(lane%4) + {0,1} and, of O^T, channels mt*16 + lane/4 (+8).
+template <int D, int NT>
+struct WarpState {
+    float m[NT][2];
+    float l[NT][2];
+    float o[D / 16][NT][4];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            m[n][0] = m[n][1] = -INFINITY;
+            l[n][0] = l[n][1] = 0.f;
+#pragma unroll
+            for (int t = 0; t < D / 16; ++t) o[t][n][0] = o[t][n][1] = o[t][n][2] = o[t][n][3] = 0.f;
+        }
+    }
+};
+
+// One 16-token block: K / V tiles at shared addresses k_tile / v_tile;
+// tokens >= ntok are masked.  qb: B fragments of Q^T (channels x heads).
+template <int D, int NT>
+__device__ __forceinline__ void attend_block_swapped(WarpState<D, NT> &st,
+                                                     const uint32_t (&qb)[D / 16][NT][2],
+                                                     uint32_t k_tile, uint32_t v_tile, int ntok,
+                                                     float scale_log2, int lane) {
+    constexpr int HALVES = D / 64;
+    float s[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+    {  // S^T = K Q^T: A = K tile (tokens x channels), ldmatrix rows = tokens
+        const int tok = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int dsub = (lane >> 4) * 8;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const int dim = ks * 16 + dsub;
+            uint32_t a[4];
+            ldmatrix_x4(a, k_tile + swz128(tok * HALVES + dim / 64, (dim % 64) / 8));
+#pragma unroll
+            for (int n = 0; n < NT; ++n) mma_bf16_16816(s[n], a, qb[ks][n][0], qb[ks][n][1]);
+        }
+    }
+    // Column (= head) softmax.  s[n][e]: token lane/4 + 8*(e>=2), head 2*(lane%4) + (e&1).
+    const int t0 = lane >> 2;
+    uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int tok = t0 + ((e >> 1) << 3);
+            x[e] = tok < ntok ? s[n][e] * scale_log2 : -INFINITY;
+        }
+        float cm[2] = {fmaxf(x[0], x[2]), fmaxf(x[1], x[3])};
+        float alpha[2], base[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            cm[k] = fmaxf(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 4));
+            cm[k] = fmaxf(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 8));
+            cm[k] = fmaxf(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 16));
+            const float mnew = fmaxf(st.m[n][k], cm[k]);
+            base[k] = mnew == -INFINITY ? 0.f : mnew;
+            alpha[k] = exp2f(st.m[n][k] - base[k]);
+            st.m[n][k] = mnew;
+        }
+        const float p0 = exp2f(x[0] - base[0]), p1 = exp2f(x[1] - base[1]);
+        const float p2 = exp2f(x[2] - base[0]), p3 = exp2f(x[3] - base[1]);
+        st.l[n][0] = st.l[n][0] * alpha[0] + p0 + p2;
+        st.l[n][1] = st.l[n][1] * alpha[1] + p1 + p3;
+#pragma unroll
+        for (int t = 0; t < D / 16; ++t) {
+            st.o[t][n][0] *= alpha[0];
+            st.o[t][n][1] *= alpha[1];
+            st.o[t][n][2] *= alpha[0];
+            st.o[t][n][3] *= alpha[1];
+        }
+        // P^T (tokens x heads) as bf16 hi + lo, transposed into B fragments.
+        uint32_t h01, l01, h23, l23;
+        split_bf16(p0, p1, h01, l01);  // tokens 0..7 rows
+        split_bf16(p2, p3, h23, l23);  // tokens 8..15 rows
+        bh[n][0] = movmatrix_trans(h01);
+        bh[n][1] = movmatrix_trans(h23);
+        bl[n][0] = movmatrix_trans(l01);
+        bl[n][1] = movmatrix_trans(l23);
+    }
+    {  // O^T += V^T P^T: A = V^T (channels x tokens) via ldmatrix.trans of V rows
+        const int tok = (lane & 7) + (lane >> 4) * 8;
+        const int dsub = ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            const int dim = mt * 16 + dsub;
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, v_tile + swz128(tok * HALVES + dim / 64, (dim % 64) / 8));
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                mma_bf16_16816(st.o[mt][n], a, bh[n][0], bh[n][1]);
+                mma_bf16_16816(st.o[mt][n], a, bl[n][0], bl[n][1]);
+            }
+        }
+    }
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap,
                          const int32_t *__restrict__ page_table,
@@ -48,7 +155,9 @@ __global__ void __launch_bounds__(kThreads)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     __shared__ uint64_t bars[kWarps][kStages];
+    __shared__ int2 meta[kMaxBlocksPerSplit];  // (page, valid tokens) of the slice's blocks
     __shared__ uint32_t sh_last;
+    __shared__ float sh_lse[kMaxGroup];
 
     const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int S = gridDim.x;
@@ -56,70 +165,77 @@ __global__ void __launch_bounds__(kThreads)
     const int hq = hkv * g;
     const size_t unit = (size_t)b * hkv + h;
 
-    int L = seq_len[b];
+    const int L = seq_len[b];
     int cnt = block_cnt[unit];
-    if (L < 1 || L > max_pages * kBlock) {
+    const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
+    if (!seq_ok) {
         if (threadIdx.x == 0 && split == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
         cnt = 0;
     }
     cnt = max(0, min(cnt, max_topk + 1));
     const int per = (cnt + S - 1) / S;
     const int j0 = min(cnt, split * per), j1 = min(cnt, j0 + per);
+    const int nslice = min(j1 - j0, kMaxBlocksPerSplit);  // the host sizes S so this holds
     const int32_t *list = block_idx + unit * (max_topk + 1);
-    const int nblk_seq = (L + kBlock - 1) / kBlock;
+    const int nblk_seq = seq_ok ? (L + kBlock - 1) / kBlock : 0;
 
     if (threadIdx.x == 0) {
         for (int w = 0; w < kWarps; ++w)
             for (int s = 0; s < kStages; ++s) mbar_init(&bars[w][s], 1);
         fence_mbar_init();
     }
+    for (int i = threadIdx.x; i < nslice; i += kThreads) {
+        const int blk = list[j0 + i];
+        int page = -1, ntok = 0;
+        if (blk >= 0 && blk < nblk_seq) {
+            page = page_table[(size_t)b * max_pages + blk];
+            if (page >= 0 && page < num_pages)
+                ntok = min(kBlock, L - blk * kBlock);
+            else
+                set_error(err, RESA_DEVERR_PAGE);
+        } else {
+            set_error(err, RESA_DEVERR_BLOCK);
+        }
+        meta[i] = make_int2(page, ntok);
+    }
+    // Q^T B fragments: head nt*8 + lane/4 (zero beyond g), channels 2*(lane%4)+{0,1} (+8).
+    uint32_t qb[D / 16][NT][2];
+    {
+        const uint16_t *base = q + ((size_t)b * hq + (size_t)h * g) * D;
+        const int c = 2 * (lane & 3);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int head = n * 8 + (lane >> 2);
+            const uint16_t *row = head < g ? base + (size_t)head * D : nullptr;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                qb[ks][n][0] = row ? *reinterpret_cast<const uint32_t *>(row + ks * 16 + c) : 0u;
+                qb[ks][n][1] = row ? *reinterpret_cast<const uint32_t *>(row + ks * 16 + c + 8) : 0u;
+            }
+        }
+    }
     __syncthreads();
 
-    // This warp's blocks: j0 + warp + kWarps * t, t = 0 .. n_mine-1.
-    const int first = j0 + warp;
-    const int n_mine = first < j1 ? (j1 - first + kWarps - 1) / kWarps : 0;
+    // This warp's blocks: slice entries warp + kWarps * t.
+    const int n_mine = warp < nslice ? (nslice - warp + kWarps - 1) / kWarps : 0;
     uint8_t *ring = smem + (size_t)warp * kStages * SM::kStageBytes;
-
-    // Returns valid tokens of the t-th block (0 when skipped); lane 0 issues
-    // its loads into stage t % kStages (or completes the phase without data).
-    auto block_tokens = [&](int t, int &page_out) -> int {
-        const int blk = list[first + kWarps * t];
-        int page = -1;
-        if (blk >= 0 && blk < nblk_seq) page = page_table[(size_t)b * max_pages + blk];
-        page_out = page;
-        if (page < 0 || page >= num_pages) return 0;
-        return min(kBlock, L - blk * kBlock);
-    };
-    auto issue = [&](int t) {
-        int page;
-        const int nt = block_tokens(t, page);
+    auto issue = [&](int t) {  // lane 0
+        const int2 mt = meta[warp + kWarps * t];
         uint64_t *bar = &bars[warp][t % kStages];
-        if (nt > 0) {
+        if (mt.y > 0) {
             uint8_t *st = ring + (size_t)(t % kStages) * SM::kStageBytes;
-            const int row = (page * hkv + h) * kBlock;
+            const int row = (mt.x * hkv + h) * kBlock;
             mbar_arrive_expect_tx(bar, SM::kStageBytes);
             tma_load_3d(st, &kmap, 0, 0, row, bar);
             tma_load_3d(st + SM::kTileBytes, &vmap, 0, 0, row, bar);
         } else {
-            const int blk = list[first + kWarps * t];
-            set_error(err, (blk >= 0 && blk < nblk_seq) ? RESA_DEVERR_PAGE : RESA_DEVERR_BLOCK);
-            mbar_arrive(bar);
+            mbar_arrive(bar);  // skipped block: complete the phase without data
         }
     };
-
     if (lane == 0)
         for (int t = 0; t < n_mine && t < kStages; ++t) issue(t);
 
-    // Query fragments: rows r < g are the group's query heads.
-    uint32_t qa[D / 16][4];
-    {
-        const int r0 = lane >> 2, r1 = r0 + 8;
-        const uint16_t *base = q + ((size_t)b * hq + (size_t)h * g) * D;
-        load_q_frags<D>(qa, r0 < g ? base + (size_t)r0 * D : nullptr,
-                        r1 < g ? base + (size_t)r1 * D : nullptr, lane);
-    }
-
-    RowState<D> st;
+    WarpState<D, NT> st;
     st.init();
     bool ok = true;
     int t_done = 0;
@@ -129,11 +245,10 @@ __global__ void __launch_bounds__(kThreads)
             ok = false;
             break;
         }
-        int page;
-        const int nt = block_tokens(t, page);
-        if (nt > 0) {
+        const int ntok = meta[warp + kWarps * t].y;
+        if (ntok > 0) {
             const uint32_t ks = smem_u32(ring + (size_t)stage * SM::kStageBytes);
-            attend_tile16<D>(st, qa, ks, ks + SM::kTileBytes, nt, nt, scale_log2, lane);
+            attend_block_swapped<D, NT>(st, qb, ks, ks + SM::kTileBytes, ntok, scale_log2, lane);
         }
         t_done = t + 1;
         fence_proxy_async_smem();
@@ -142,36 +257,41 @@ __global__ void __launch_bounds__(kThreads)
     }
     if (!ok) {
         if (lane == 0) set_error(err, RESA_DEVERR_TIMEOUT);
-        // drain: give every issued load a bounded chance to land before exit
         for (int t = t_done; t < n_mine && t < t_done + kStages; ++t)
             mbar_wait_bounded(&bars[warp][t % kStages], (t / kStages) & 1);
     }
-    finish_rows<D>(st);
-    __syncthreads();  // every warp is done with its ring: reuse it for the merge
-
-    // Merge the warps: per warp m[16], l[16], lx[16], acc[16][D] (unnormalised).
-    float *mw = reinterpret_cast<float *>(smem);
-    float *lw = mw + kWarps * kMaxGroup;
-    float *lxw = lw + kWarps * kMaxGroup;
-    float *ow = lxw + kWarps * kMaxGroup;
-    {
-        const int r0 = lane >> 2, r1 = r0 + 8, cb = 2 * (lane & 3);
-        if ((lane & 3) == 0) {
-            mw[warp * kMaxGroup + r0] = st.m[0];
-            mw[warp * kMaxGroup + r1] = st.m[1];
-            lw[warp * kMaxGroup + r0] = st.l[0];
-            lw[warp * kMaxGroup + r1] = st.l[1];
-            lxw[warp * kMaxGroup + r0] = st.lx[0];
-            lxw[warp * kMaxGroup + r1] = st.lx[1];
-        }
+    // Row sums over the eight lanes that share each head.
 #pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-            float *o0 = ow + ((size_t)warp * kMaxGroup + r0) * D + j * 8 + cb;
-            float *o1 = ow + ((size_t)warp * kMaxGroup + r1) * D + j * 8 + cb;
-            o0[0] = st.acc[j][0];
-            o0[1] = st.acc[j][1];
-            o1[0] = st.acc[j][2];
-            o1[1] = st.acc[j][3];
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            st.l[n][k] += __shfl_xor_sync(0xffffffffu, st.l[n][k], 4);
+            st.l[n][k] += __shfl_xor_sync(0xffffffffu, st.l[n][k], 8);
+            st.l[n][k] += __shfl_xor_sync(0xffffffffu, st.l[n][k], 16);
+        }
+    __syncthreads();  // every ring is drained: reuse it for the merge
+
+    float *mw = reinterpret_cast<float *>(smem);  // [kWarps][16]
+    float *lw = mw + kWarps * kMaxGroup;          // [kWarps][16]
+    float *ow = lw + kWarps * kMaxGroup;          // [kWarps][16][D]
+    {
+        const int hb = 2 * (lane & 3), d0 = lane >> 2;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            if (lane < 4) {
+                mw[warp * kMaxGroup + n * 8 + hb] = st.m[n][0];
+                mw[warp * kMaxGroup + n * 8 + hb + 1] = st.m[n][1];
+                lw[warp * kMaxGroup + n * 8 + hb] = st.l[n][0];
+                lw[warp * kMaxGroup + n * 8 + hb + 1] = st.l[n][1];
+            }
+#pragma unroll
+            for (int t = 0; t < D / 16; ++t) {
+                float *o0 = ow + ((size_t)warp * kMaxGroup + n * 8 + hb) * D + t * 16 + d0;
+                o0[0] = st.o[t][n][0];
+                o0[D] = st.o[t][n][1];
+                o0[8] = st.o[t][n][2];
+                o0[D + 8] = st.o[t][n][3];
+            }
         }
     }
     __syncthreads();
@@ -181,17 +301,18 @@ __global__ void __launch_bounds__(kThreads)
     for (int e = threadIdx.x; e < g * D; e += kThreads) {
         const int r = e / D, c = e % D;
         float mstar = -INFINITY;
+#pragma unroll
         for (int w = 0; w < kWarps; ++w) mstar = fmaxf(mstar, mw[w * kMaxGroup + r]);
-        float lsum = 0.f, lxsum = 0.f, o = 0.f;
+        float lsum = 0.f, o = 0.f;
         if (mstar != -INFINITY) {
+#pragma unroll
             for (int w = 0; w < kWarps; ++w) {
                 const float sc = exp2f(mw[w * kMaxGroup + r] - mstar);
                 lsum += lw[w * kMaxGroup + r] * sc;
-                lxsum += lxw[w * kMaxGroup + r] * sc;
                 o += ow[((size_t)w * kMaxGroup + r) * D + c] * sc;
             }
         }
-        const float lse2 = lsum > 0.f ? mstar + log2f(lxsum) : -INFINITY;
+        const float lse2 = lsum > 0.f ? mstar + log2f(lsum) : -INFINITY;
         const float on = lsum > 0.f ? o / lsum : 0.f;
         if (S == 1) {
             out[((size_t)b * hq + (size_t)h * g + r) * D + c] = on;
@@ -203,7 +324,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     if (S == 1) return;
 
-    // Split combine: the CTA that draws the last ticket merges all splits.
+    // Split combine by the CTA that draws the last ticket.
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -213,41 +334,64 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
     if (!sh_last) return;
     __threadfence();
-    const float *uo = part_o + unit * S * kMaxGroup * D;
+    float *wts = reinterpret_cast<float *>(smem);  // [S][16] merge weights
     const float *ul = part_lse + unit * S * kMaxGroup;
-    for (int e = threadIdx.x; e < g * D; e += kThreads) {
-        const int r = e / D, c = e % D;
+    const float *uo = part_o + unit * S * kMaxGroup * D;
+    for (int i = threadIdx.x; i < S * g; i += kThreads) {
+        const int s = i / g, r = i % g;
+        wts[s * kMaxGroup + r] = __ldcg(&ul[s * kMaxGroup + r]);
+    }
+    __syncthreads();
+    for (int r = warp; r < g; r += kWarps) {
         float mstar = -INFINITY;
-        for (int s = 0; s < S; ++s) mstar = fmaxf(mstar, __ldcg(&ul[s * kMaxGroup + r]));
-        float wsum = 0.f, o = 0.f;
-        if (mstar != -INFINITY) {
-            for (int s = 0; s < S; ++s) {
-                const float w = exp2f(__ldcg(&ul[s * kMaxGroup + r]) - mstar);
-                wsum += w;
-                o += w * __ldcg(&uo[((size_t)s * kMaxGroup + r) * D + c]);
-            }
+        for (int s = lane; s < S; s += 32) mstar = fmaxf(mstar, wts[s * kMaxGroup + r]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
+        float sum = 0.f;
+        if (mstar != -INFINITY)
+            for (int s = lane; s < S; s += 32) sum += exp2f(wts[s * kMaxGroup + r] - mstar);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        __syncwarp();
+        for (int s = lane; s < S; s += 32)
+            wts[s * kMaxGroup + r] = sum > 0.f ? exp2f(wts[s * kMaxGroup + r] - mstar) / sum : 0.f;
+        if (lane == 0) sh_lse[r] = sum > 0.f ? mstar + log2f(sum) : -INFINITY;
+    }
+    __syncthreads();
+    constexpr int C4 = D / 4;
+    for (int item = threadIdx.x; item < g * C4; item += kThreads) {
+        const int r = item / C4, c4 = item % C4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 *src = reinterpret_cast<const float4 *>(uo + (size_t)r * D) + c4;
+#pragma unroll 8
+        for (int s = 0; s < S; ++s) {
+            const float w = wts[s * kMaxGroup + r];
+            const float4 v = __ldcg(src + (size_t)s * kMaxGroup * C4);
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
         }
-        out[((size_t)b * hq + (size_t)h * g + r) * D + c] = wsum > 0.f ? o / wsum : 0.f;
-        if (lse_out && c == 0)
-            lse_out[(size_t)b * hq + (size_t)h * g + r] =
-                wsum > 0.f ? (mstar + log2f(wsum)) * kLn2 : -INFINITY;
+        const size_t orow = (size_t)b * hq + (size_t)h * g + r;
+        reinterpret_cast<float4 *>(out + orow * D)[c4] = acc;
+        if (lse_out && c4 == 0) lse_out[orow] = sh_lse[r] * kLn2;
     }
     if (threadIdx.x == 0) tickets[unit] = 0;
 }
 
-template <int D>
-cudaError_t launch_d(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
-                     const int32_t *page_table, const int32_t *seq_len, const void *q,
-                     const int32_t *block_idx, const int32_t *block_cnt, int max_topk, int splits,
-                     float *part_o, float *part_lse, uint32_t *tickets, float *out, float *lse,
-                     uint32_t *err, cudaStream_t st) {
+template <int D, int NT>
+cudaError_t launch_dn(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                      const int32_t *page_table, const int32_t *seq_len, const void *q,
+                      const int32_t *block_idx, const int32_t *block_cnt, int max_topk, int splits,
+                      float *part_o, float *part_lse, uint32_t *tickets, float *out, float *lse,
+                      uint32_t *err, cudaStream_t st) {
     constexpr int smem = DecodeSmem<D>::kBytes;
     static std::atomic<int> done[64];
-    cudaError_t e = ensure_smem(sparse_decode_kernel<D>, smem, done);
+    cudaError_t e = ensure_smem(sparse_decode_kernel<D, NT>, smem, done);
     if (e != cudaSuccess) return e;
     const float scale_log2 = s.sm_scale * 1.4426950408889634f;
     dim3 grid(splits, s.hkv, s.batch);
-    sparse_decode_kernel<D><<<grid, kThreads, smem, st>>>(
+    sparse_decode_kernel<D, NT><<<grid, kThreads, smem, st>>>(
         kmap, vmap, page_table, seq_len, (const uint16_t *)q, block_idx, block_cnt, max_topk,
         s.hkv, s.g, s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out, lse,
         err);
@@ -261,12 +405,14 @@ cudaError_t launch_sparse_decode(const Shape &s, const CUtensorMap &kmap, const 
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
                                  float *out, float *lse, uint32_t *err, cudaStream_t st) {
+#define RESA_DECODE_ARGS                                                                     \
+    s, kmap, vmap, page_table, seq_len, q, block_idx, block_cnt, max_topk, splits, part_o, \
+        part_lse, tickets, out, lse, err, st
     if (s.d == 128)
-        return launch_d<128>(s, kmap, vmap, page_table, seq_len, q, block_idx, block_cnt,
-                             max_topk, splits, part_o, part_lse, tickets, out, lse, err, st);
+        return s.g <= 8 ? launch_dn<128, 1>(RESA_DECODE_ARGS) : launch_dn<128, 2>(RESA_DECODE_ARGS);
     if (s.d == 64)
-        return launch_d<64>(s, kmap, vmap, page_table, seq_len, q, block_idx, block_cnt, max_topk,
-                            splits, part_o, part_lse, tickets, out, lse, err, st);
+        return s.g <= 8 ? launch_dn<64, 1>(RESA_DECODE_ARGS) : launch_dn<64, 2>(RESA_DECODE_ARGS);
+#undef RESA_DECODE_ARGS
     return cudaErrorInvalidValue;
 }
 

@@ -107,15 +107,6 @@ WsLayout layout_of(const Shape &s, int chunk) {
     return ws_layout(s.hq, s.hkv, s.d, s.batch, s.max_pages, chunk);
 }
 
-int decode_splits(const Shape &s, const WsLayout &w, int max_topk) {
-    // ~8 blocks per CTA at least, at most what the workspace holds.
-    const int by_work = (max_topk + 1 + 7) / 8;
-    int sp = w.dec_splits < by_work ? w.dec_splits : by_work;
-    const int units = s.batch * s.hkv;
-    const int by_sm = (2 * 148 + units - 1) / units;
-    sp = sp < by_sm ? sp : by_sm;
-    return sp < 1 ? 1 : sp;
-}
 
 resa_status_t select_impl(const Shape &s, const resa_cache_t *c, const WsLayout &w, void *ws,
                           const void *q, const int32_t *topk, int max_topk, int32_t *idx,
@@ -134,7 +125,8 @@ resa_status_t decode_impl(const Shape &s, const resa_cache_t *c, const WsLayout 
     if (!make_kv_map(&kmap, c->k, s.num_pages, s.hkv, s.d) ||
         !make_kv_map(&vmap, c->v, s.num_pages, s.hkv, s.d))
         return RESA_ERR_CUDA;
-    const int splits = decode_splits(s, w, max_topk);
+    const int splits = decode_splits_for(s.batch * s.hkv, max_topk + 1);
+    if (splits > w.dec_splits) return RESA_ERR_RANGE;  // max_topk far above max_pages
     return cuda_status(launch_sparse_decode(
         s, kmap, vmap, c->page_table, c->seq_len, q, idx, cnt, max_topk, splits,
         at<float>(ws, w.dec_o), at<float>(ws, w.dec_lse), at<uint32_t>(ws, w.dec_ticket), out, lse,

@@ -18,14 +18,26 @@ namespace resa {
 constexpr int kBlock = 16;          // tokens per block / page
 constexpr int kMaxGroup = 16;       // query heads per kv head (one m16 MMA tile)
 constexpr int kMaxKvHeads = 8;
-constexpr int kTargetCtas = 4 * 148;  // split-KV sizing: ~4 resident CTAs per SM
+constexpr int kNumSms = 148;
+constexpr int kMaxBlocksPerSplit = 512;  // blocks one decode CTA stages in shared memory
+constexpr int kMinBlocksPerSplit = 16;   // two per warp at least
 
-// Work units (sequence, kv head) x splits are bounded so the partial-result
-// region of the workspace depends on (batch, Hkv) only.
-inline int decode_max_splits(int batch, int hkv) {
-    int units = batch * hkv;
-    int s = (kTargetCtas + units - 1) / units;
-    return s < 1 ? 1 : (s > 128 ? 128 : s);
+// Decode splits per (sequence, kv head): about one CTA per SM over all units,
+// at least kMinBlocksPerSplit blocks each, at most kMaxBlocksPerSplit.
+inline int decode_splits_for(int units, int max_blocks) {
+    const int need = (max_blocks + kMaxBlocksPerSplit - 1) / kMaxBlocksPerSplit;
+    const int want = (kNumSms + units - 1) / units;
+    const int work = (max_blocks + kMinBlocksPerSplit - 1) / kMinBlocksPerSplit;
+    int s = want < work ? want : work;
+    s = s > need ? s : need;
+    return s < 1 ? 1 : s;
+}
+// Partial-result capacity of the workspace: enough for any top-k up to max_pages.
+inline int decode_max_splits(int batch, int hkv, int max_pages) {
+    const int units = batch * hkv;
+    const int need = (max_pages + 1 + kMaxBlocksPerSplit - 1) / kMaxBlocksPerSplit;
+    const int want = (kNumSms + units - 1) / units;
+    return want > need ? want : need;
 }
 constexpr int kRectRowsPerTile = 64;    // query rows (chunk position x group head) per CTA
 inline int rect_row_tiles(int max_chunk, int group) {
@@ -75,7 +87,7 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
         return o;
     };
     int g = hkv > 0 ? hq / hkv : 1;
-    w.dec_splits = decode_max_splits(batch, hkv);
+    w.dec_splits = decode_max_splits(batch, hkv, max_pages);
     w.row_tiles = chunk > 0 ? rect_row_tiles(chunk, g) : 0;
     w.rect_splits = chunk > 0 ? rect_max_splits(batch, hkv, w.row_tiles) : 0;
     size_t units = (size_t)batch * hkv;
@@ -190,6 +202,19 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+// Split two fp32 weights into bf16 hi + lo parts (hi + lo carries ~16
+// significant bits), packed as bf16x2 pairs for the MMA operand.
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(a, b);
+    lo = pack_bf16(a - bf_lo(hi), b - bf_hi(hi));
+}
+// Transpose an 8x8 b16 matrix held one row-pair per lane (row lane/4,
+// columns 2*(lane%4)+{0,1}) across the warp.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
 }
 
 // Byte offset of (row, 16-byte chunk) inside a tile written by TMA with

@@ -59,8 +59,14 @@ __global__ void __launch_bounds__(kScoreThreads)
     // Group pooling: mean of the g query heads, fp32, head order, then / g.
     for (int e = threadIdx.x; e < HKV * D; e += kScoreThreads) {
         const int h = e / D, j = e % D;
+        const uint16_t *col = q + ((size_t)b * hq + h * g) * D + j;
+        uint16_t v[kMaxGroup];
+#pragma unroll
+        for (int r = 0; r < kMaxGroup; ++r) v[r] = r < g ? col[(size_t)r * D] : (uint16_t)0;
         float s = 0.f;
-        for (int r = 0; r < g; ++r) s += bf16_bits_to_f32(q[((size_t)b * hq + h * g + r) * D + j]);
+#pragma unroll
+        for (int r = 0; r < kMaxGroup; ++r)
+            if (r < g) s += bf16_bits_to_f32(v[r]);
         qbar_s[h][j] = s / (float)g;
     }
     __syncthreads();
@@ -179,8 +185,22 @@ __global__ void __launch_bounds__(kSelectThreads)
     }
     const float *src = scores + ((size_t)b * hkv + h) * max_pages;
     const bool in_smem = M <= key_cap;
-    if (in_smem)
-        for (int i = tid; i < M; i += kSelectThreads) keys_s[i] = order_key(src[i]);
+    if (in_smem) {
+        constexpr int U = 8;  // loads in flight per thread
+        for (int i0 = tid; i0 < M; i0 += U * kSelectThreads) {
+            float v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * kSelectThreads;
+                v[u] = i < M ? src[i] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * kSelectThreads;
+                if (i < M) keys_s[i] = order_key(v[u]);
+            }
+        }
+    }
     __syncthreads();
     auto key_at = [&](int i) -> uint32_t { return in_smem ? keys_s[i] : order_key(src[i]); };
 
