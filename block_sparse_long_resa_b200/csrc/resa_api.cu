@@ -299,7 +299,8 @@ int32_t resa_kernels_per_call(const char *entry_point) {
         int n;
     } table[] = {{"resa_build_descriptors", 1}, {"resa_append_token", 1},
                  {"resa_select_blocks", 2},     {"resa_sparse_decode", 1},
-                 {"resa_rectify_attention", 2}, {"resa_decode_step", 4}};
+                 {"resa_rectify_attention", 2}, {"resa_decode_step", 4},
+                 {"resa_sparse_decode_noalloc", 1}};
     for (auto &e : table)
         if (strcmp(e.name, entry_point) == 0) return e.n;
     return -1;

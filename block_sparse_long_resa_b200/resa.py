@@ -61,6 +61,7 @@ _SIGS = {
                                ctypes.c_int),
     "resa_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
                          ctypes.c_int),
+    "resa_sparse_decode_noalloc": ([_P, _P, _P, _P, _P, _I, _P, _P, _P, _P], ctypes.c_int),
     "resa_kernels_per_call": ([ctypes.c_char_p], ctypes.c_int32),
     "resa_status_string": ([ctypes.c_int], ctypes.c_char_p),
 }
@@ -185,6 +186,16 @@ def resa_decode_step(cfg, cache, q, k_new, v_new, topk, max_topk: int, out, lse,
                                   _ptr(block_idx), _ptr(block_cnt), _ptr(ws), ws.numel(),
                                   _stream(stream)),
            "resa_decode_step")
+
+
+def resa_sparse_decode_noalloc(cfg, cache, q, block_idx, block_cnt, max_topk: int, out, lse,
+                               dev_error=None, stream=None):
+    """resa_sparse_decode without a workspace, for callers that cannot allocate
+    device memory (scratch lives in a fixed device array inside the library)."""
+    _check(lib().resa_sparse_decode_noalloc(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q),
+                                            _ptr(block_idx), _ptr(block_cnt), max_topk, _ptr(out),
+                                            _ptr(lse), _ptr(dev_error), _stream(stream)),
+           "resa_sparse_decode_noalloc")
 
 
 def resa_kernels_per_call(entry_point: str) -> int:

@@ -180,9 +180,40 @@ RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cac
                                int32_t *block_idx_opt, int32_t *block_cnt_opt, void *ws,
                                size_t ws_bytes, cudaStream_t stream);
 
+/* The group block-sparse decode of resa_sparse_decode for callers that
+ * cannot allocate device memory.  The pages describe no such variant: it
+ * exists for hosts that give this library only input and output pointers,
+ * e.g. a serving engine that reserves all of HBM for its own KV-cache pool
+ * at start-up, or a plugin interface that forbids device allocations after
+ * initialisation, and so cannot provide a workspace.
+ *   - Takes the arguments of resa_sparse_decode minus the workspace; the
+ *     decode scratch (split partials, split tickets, error word) lives in a
+ *     fixed 8 MiB device array inside the library, held by every GPU that
+ *     loads it until the process exits.  Nothing is allocated or freed.
+ *   - Limit: batch * Hkv <= 4096 and batch * Hkv * splits * 16 * (d + 1) * 4
+ *     bytes of partials must fit the array (about 8 MiB); larger calls return
+ *     RESA_ERR_SHAPE.  Splits are chosen as in resa_sparse_decode.
+ *   - The first call on each device looks up the array's device address
+ *     (a runtime query, done once per device with that device current); make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents; the call clears the parts that must start at zero.
+ *     Calls that overlap on the GPU (different streams, or host threads
+ *     without ordering) race on the array: serialise them.
+ *   - dev_error_opt (nullable, device uint32, zeroed by the caller) receives
+ *     the device error bits that resa_check_device_status reports for the
+ *     workspace path. */
+RESA_API resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
+                                                  const resa_cache_t *cache, const void *q,
+                                                  const int32_t *block_idx,
+                                                  const int32_t *block_cnt, int32_t max_topk,
+                                                  float *out, float *lse_opt,
+                                                  uint32_t *dev_error_opt, cudaStream_t stream);
+
 /* Number of kernels each entry point launches per call (for launch
  * accounting): 1 for append and build, 2 for select, 1 for sparse decode,
- * 2 for rectify, 4 for a decode step.  Unknown names return -1. */
+ * 2 for rectify, 4 for a decode step, 1 for the no-allocation decode.
+ * Unknown names return -1. */
 RESA_API int32_t resa_kernels_per_call(const char *entry_point);
 
 /* Human-readable status name. */
