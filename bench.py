@@ -587,11 +587,15 @@ def kernel_breakdown(w, stream, device, reps):
     row = c * w.f + w.f - 2          # last decode step of the last cycle
     rrow = c * w.f + w.f - 1
 
+    rounds = max(1, -(-28 // w.layers))   # >= 28 launches per graph: replay overhead amortised
+
     def timed(enqueue, calls):
+        calls *= rounds
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
-                enqueue()
+                for _ in range(rounds):
+                    enqueue()
             g.replay()
             torch.cuda.synchronize(device)
             e0 = torch.cuda.Event(enable_timing=True)

@@ -165,40 +165,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hq = hkv * g;
     const size_t unit = (size_t)b * hkv + h;
 
+    pdl_launch_next();
     const int L = seq_len[b];
-    int cnt = block_cnt[unit];
-    const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
-    if (!seq_ok) {
-        if (threadIdx.x == 0 && split == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
-        cnt = 0;
-    }
-    cnt = max(0, min(cnt, max_topk + 1));
-    const int per = (cnt + S - 1) / S;
-    const int j0 = min(cnt, split * per), j1 = min(cnt, j0 + per);
-    const int nslice = min(j1 - j0, kMaxBlocksPerSplit);  // the host sizes S so this holds
-    const int32_t *list = block_idx + unit * (max_topk + 1);
-    const int nblk_seq = seq_ok ? (L + kBlock - 1) / kBlock : 0;
-
     if (threadIdx.x == 0) {
         for (int w = 0; w < kWarps; ++w)
             for (int s = 0; s < kStages; ++s) mbar_init(&bars[w][s], 1);
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < nslice; i += kThreads) {
-        const int blk = list[j0 + i];
-        int page = -1, ntok = 0;
-        if (blk >= 0 && blk < nblk_seq) {
-            page = page_table[(size_t)b * max_pages + blk];
-            if (page >= 0 && page < num_pages)
-                ntok = min(kBlock, L - blk * kBlock);
-            else
-                set_error(err, RESA_DEVERR_PAGE);
-        } else {
-            set_error(err, RESA_DEVERR_BLOCK);
-        }
-        meta[i] = make_int2(page, ntok);
-    }
     // Q^T B fragments: head nt*8 + lane/4 (zero beyond g), channels 2*(lane%4)+{0,1} (+8).
+    // q is an input of the step, so it is read before waiting for the selection.
     uint32_t qb[D / 16][NT][2];
     {
         const uint16_t *base = q + ((size_t)b * hq + (size_t)h * g) * D;
@@ -213,6 +188,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 qb[ks][n][1] = row ? *reinterpret_cast<const uint32_t *>(row + ks * 16 + c + 8) : 0u;
             }
         }
+    }
+    pdl_wait();  // block lists / counts come from the preceding selection
+    int cnt = block_cnt[unit];
+    const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
+    if (!seq_ok) {
+        if (threadIdx.x == 0 && split == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
+        cnt = 0;
+    }
+    cnt = max(0, min(cnt, max_topk + 1));
+    const int per = (cnt + S - 1) / S;
+    const int j0 = min(cnt, split * per), j1 = min(cnt, j0 + per);
+    const int nslice = min(j1 - j0, kMaxBlocksPerSplit);  // the host sizes S so this holds
+    const int32_t *list = block_idx + unit * (max_topk + 1);
+    const int nblk_seq = seq_ok ? (L + kBlock - 1) / kBlock : 0;
+
+    for (int i = threadIdx.x; i < nslice; i += kThreads) {
+        const int blk = list[j0 + i];
+        int page = -1, ntok = 0;
+        if (blk >= 0 && blk < nblk_seq) {
+            page = page_table[(size_t)b * max_pages + blk];
+            if (page >= 0 && page < num_pages)
+                ntok = min(kBlock, L - blk * kBlock);
+            else
+                set_error(err, RESA_DEVERR_PAGE);
+        } else {
+            set_error(err, RESA_DEVERR_BLOCK);
+        }
+        meta[i] = make_int2(page, ntok);
     }
     __syncthreads();
 
@@ -391,11 +394,10 @@ cudaError_t launch_dn(const Shape &s, const CUtensorMap &kmap, const CUtensorMap
     if (e != cudaSuccess) return e;
     const float scale_log2 = s.sm_scale * 1.4426950408889634f;
     dim3 grid(splits, s.hkv, s.batch);
-    sparse_decode_kernel<D, NT><<<grid, kThreads, smem, st>>>(
-        kmap, vmap, page_table, seq_len, (const uint16_t *)q, block_idx, block_cnt, max_topk,
-        s.hkv, s.g, s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out, lse,
-        err);
-    return cudaGetLastError();
+    return launch_pdl(sparse_decode_kernel<D, NT>, grid, dim3(kThreads), smem, st, kmap, vmap,
+                      page_table, seq_len, (const uint16_t *)q, block_idx, block_cnt, max_topk,
+                      s.hkv, s.g, s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets,
+                      out, lse, err);
 }
 
 }  // namespace

@@ -1,0 +1,487 @@
+// Dense rectification chunk attention on the 5th-generation tensor cores
+// (ReSA summary §3.4.2; Algorithm 1, rectification check): the f chunk
+// queries of every group head attend causally to the whole cache, after the
+// chunk's fresh K/V were written back.
+//
+// Rows of one (sequence, kv head) are rho = r * g + j (chunk position r, group
+// head j; position L - f + r).  Grid (row groups of 256, splits, batch * Hkv):
+// a CTA owns 256 rows (two M = 128 MMA tiles) and one contiguous range of KV
+// blocks, streamed as tiles of 64 keys (four blocks).
+//
+// Warp roles (384 threads, one CTA per SM):
+//   warp 0      TMA producer: per block and channel half, 2-D tensor loads of
+//               K and V (16 x 64, 128-byte swizzled) into a two-stage ring;
+//   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into a
+//               double-buffered TMEM tile (kind::f16, bf16 inputs), then
+//               O += P V (kind::f16, fp16 inputs), commits on mbarriers;
+//   warps 2-3   convert the V tile bf16 -> fp16 in place (exact for
+//               |v| < 65504), zero blocks that were not loaded;
+//   warps 4-11  softmax, one thread per query row (TMEM lane): tcgen05.ld of
+//               the S row, causal mask, base-2 online softmax with lazy O
+//               rescaling (only when the row maximum grows by more than 8),
+//               P written to shared memory as fp16 in the canonical K-major
+//               swizzled layout.
+// P is fp16 (11-bit mantissa), so the P.V product keeps the weights' precision
+// without a second MMA.  Partial (o, lse) per split are merged by the CTA that
+// draws the last ticket of its (unit, row group).  Waits are bounded.
+#include "tc_common.cuh"
+
+namespace resa {
+namespace {
+
+constexpr int kRows = kRectRowsPerCta;  // 256
+constexpr int kKeys = 64;               // keys per KV tile
+constexpr int kBlocksPerTile = kKeys / kBlock;
+constexpr int kStages = 2;
+constexpr int kNumConv = 2;             // converter warps
+constexpr int kWarpSm0 = 4;             // first softmax warp
+constexpr int kNumSm = 8;               // softmax warps
+constexpr int kThreads = 32 * (kWarpSm0 + kNumSm);
+constexpr int kSmThreads = 32 * kNumSm;
+constexpr int kConvThreads = 32 * kNumConv;
+constexpr float kRescaleSlack = 8.0f;   // log2 units of growth tolerated before rescaling O
+
+template <int D>
+struct TcLayout {
+    static constexpr int kHalves = D / 64;
+    static constexpr int kQTile = 128 * D * 2;     // one M tile of Q, [half][128 rows][128 B]
+    static constexpr int kQHalf = 128 * 128;
+    static constexpr int kKV = kKeys * D * 2;      // K or V tile, [half][64 keys][128 B]
+    static constexpr int kKVHalf = kKeys * 128;
+    static constexpr int kP = 128 * kKeys * 2;     // P of one M tile, [128 rows][128 B]
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = kQOff + 2 * kQTile;
+    static constexpr int kPOff = kKVOff + kStages * 2 * kKV;
+    static constexpr int kBytes = kPOff + 2 * 2 * kP + 1024;
+    // TMEM columns: O[mt] at mt*D, S[buf][mt] at 2*D + (2*buf + mt)*64.
+    static constexpr uint32_t kTmemCols = 512;
+};
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
+    const __half2 h = __floats2half2_rn(bf_lo(x), bf_hi(x));
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    rectify_tc_kernel(const __grid_constant__ CUtensorMap k0map,
+                      const __grid_constant__ CUtensorMap k1map,
+                      const __grid_constant__ CUtensorMap v0map,
+                      const __grid_constant__ CUtensorMap v1map,
+                      const int32_t *__restrict__ page_table, const int32_t *__restrict__ seq_len,
+                      int f, const uint16_t *__restrict__ q_chunk, int hkv, int g, int max_pages,
+                      int num_pages, float scale_log2, float *__restrict__ part_o,
+                      float *__restrict__ part_lse, uint32_t *__restrict__ tickets,
+                      float *__restrict__ out, float *__restrict__ lse_out, uint32_t *err) {
+    using LY = TcLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    __shared__ uint64_t q_ready, kv_full[kStages], v_ready[kStages], s_full[2], p_full[2],
+        pv_done[2];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ uint32_t stage_vmask[kStages];
+    __shared__ uint32_t sh_last;
+
+    const int group = blockIdx.x, split = blockIdx.y, unit = blockIdx.z;
+    const int G = gridDim.x, S = gridDim.y;
+    const int b = unit / hkv, h = unit % hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hq = hkv * g;
+    const int R = f * g;
+
+    const int L = seq_len[b];
+    const bool seq_ok = L >= 1 && L <= max_pages * kBlock && f <= L;
+    if (!seq_ok && threadIdx.x == 0 && group == 0 && split == 0)
+        set_error(err, (L < 1 || L > max_pages * kBlock) ? RESA_DEVERR_SEQ_LEN : RESA_DEVERR_CHUNK);
+    const int start = L - f;
+    const int row0 = group * kRows;
+    const int last_row = min(R, row0 + kRows) - 1;
+    const int lim_max = (seq_ok && row0 < R) ? start + last_row / g + 1 : 0;
+    const int nblk = (lim_max + kBlock - 1) / kBlock;
+    int per = (nblk + S - 1) / S;
+    per = (per + kBlocksPerTile - 1) / kBlocksPerTile * kBlocksPerTile;
+    const int blk0 = min(nblk, split * per), blk1 = min(nblk, blk0 + per);
+    const int ntiles = (blk1 - blk0 + kBlocksPerTile - 1) / kBlocksPerTile;
+
+    uint8_t *q_s = smem + LY::kQOff;
+    uint8_t *kv_s = smem + LY::kKVOff;
+    uint8_t *p_s = smem + LY::kPOff;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&q_ready, kSmThreads);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&v_ready[s], kConvThreads);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], kSmThreads);
+            mbar_init(&pv_done[s], 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) tc::tmem_alloc(&tmem_base_s, LY::kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base_s;
+
+    if (warp == 0) {  // ------------------------------------------------ TMA producer
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int s = i % kStages;
+            if (i >= kStages) ok = mbar_wait_bounded(&pv_done[s], ((i - kStages) / 2) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            const int blk = blk0 + i * kBlocksPerTile + lane;
+            int page = -1;
+            if (lane < kBlocksPerTile && blk < blk1) {
+                page = page_table[(size_t)b * max_pages + blk];
+                if (page < 0 || page >= num_pages) {
+                    set_error(err, RESA_DEVERR_PAGE);
+                    page = -1;
+                }
+            }
+            const uint32_t vmask = __ballot_sync(0xffffffffu, page >= 0);
+            const uint32_t bytes = (uint32_t)__popc(vmask) * 2u * LY::kHalves * kBlock * 128u;
+            if (lane == 0) {
+                stage_vmask[s] = vmask;
+                if (bytes == 0)
+                    mbar_arrive(&kv_full[s]);
+                else
+                    mbar_arrive_expect_tx(&kv_full[s], bytes);
+            }
+            __syncwarp();
+            if (page >= 0) {
+                const int y = (page * hkv + h) * kBlock;
+                uint8_t *kt = kv_s + (size_t)s * 2 * LY::kKV;
+                uint8_t *vt = kt + LY::kKV;
+                const int off = lane * kBlock * 128;  // this block's 16 rows in each half
+                tc::tma_load_2d(kt + off, &k0map, 0, y, &kv_full[s]);
+                tc::tma_load_2d(vt + off, &v0map, 0, y, &kv_full[s]);
+                if (LY::kHalves == 2) {
+                    tc::tma_load_2d(kt + LY::kKVHalf + off, &k1map, 0, y, &kv_full[s]);
+                    tc::tma_load_2d(vt + LY::kKVHalf + off, &v1map, 0, y, &kv_full[s]);
+                }
+            }
+        }
+        if (!ok && lane == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+    } else if (warp == 1) {  // ----------------------------------------- MMA issuer
+        constexpr uint32_t idesc_qk = tc::idesc_f16(1, 1, 0, 0, 128, kKeys);
+        constexpr uint32_t idesc_pv = tc::idesc_f16(0, 0, 0, 1, 128, D);
+        bool ok = mbar_wait_bounded(&q_ready, 0);
+        auto issue_qk = [&](int i) {
+            const int s = i % kStages, buf = i & 1;
+            const uint32_t kt = smem_u32(kv_s + (size_t)s * 2 * LY::kKV);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const uint32_t qt = smem_u32(q_s + mt * LY::kQTile);
+                const uint32_t d_tmem = tmem + 2 * D + (2 * buf + mt) * kKeys;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int half = ks / 4, kin = ks % 4;
+                    const uint64_t a = tc::smem_desc(qt + half * LY::kQHalf + kin * 32, 16, 1024);
+                    const uint64_t bd = tc::smem_desc(kt + half * LY::kKVHalf + kin * 32, 16, 1024);
+                    tc::mma_f16_ss(d_tmem, a, bd, idesc_qk, ks > 0 ? 1u : 0u);
+                }
+            }
+            tc::commit(&s_full[buf]);
+        };
+        if (lane == 0 && ok && ntiles > 0) {
+            ok = mbar_wait_bounded(&kv_full[0], 0);
+            tc::fence_after_sync();
+            if (ok) issue_qk(0);
+            for (int i = 0; i < ntiles && ok; ++i) {
+                const int s = i % kStages, buf = i & 1;
+                if (i + 1 < ntiles) {
+                    ok = mbar_wait_bounded(&kv_full[(i + 1) % kStages], ((i + 1) / kStages) & 1);
+                    tc::fence_after_sync();
+                    if (!ok) break;
+                    issue_qk(i + 1);  // S[(i+1)&1] was released by the softmax of tile i-1
+                }
+                ok = mbar_wait_bounded(&p_full[buf], (i / 2) & 1) &&
+                     mbar_wait_bounded(&v_ready[s], (i / kStages) & 1);
+                tc::fence_after_sync();
+                if (!ok) break;
+                const uint32_t vt = smem_u32(kv_s + (size_t)s * 2 * LY::kKV + LY::kKV);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    const uint32_t pt = smem_u32(p_s + (size_t)(2 * buf + mt) * LY::kP);
+#pragma unroll
+                    for (int kk = 0; kk < kKeys / 16; ++kk) {
+                        const uint64_t a = tc::smem_desc(pt + kk * 32, 16, 1024);
+                        const uint64_t bd = tc::smem_desc(vt + kk * 16 * 128, LY::kKVHalf, 1024);
+                        tc::mma_f16_ss(tmem + mt * D, a, bd, idesc_pv,
+                                       (i > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                tc::commit(&pv_done[buf]);
+            }
+            if (!ok) set_error(err, RESA_DEVERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp < kWarpSm0) {  // ---------------------------------- V converters
+        const int ct = threadIdx.x - 64;
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int s = i % kStages;
+            ok = mbar_wait_bounded(&kv_full[s], (i / kStages) & 1);
+            if (!ok) break;
+            const uint32_t vmask = stage_vmask[s];
+            uint4 *vt = reinterpret_cast<uint4 *>(kv_s + (size_t)s * 2 * LY::kKV + LY::kKV);
+            constexpr int kChunks = LY::kKV / 16;           // 16-byte chunks of the tile
+            constexpr int kChunksPerBlock = kBlock * 128 / 16;  // per half
+            for (int c = ct; c < kChunks; c += kConvThreads) {
+                const int blk_in_tile = (c % (LY::kKVHalf / 16)) / kChunksPerBlock;
+                uint4 x = vt[c];
+                if ((vmask >> blk_in_tile) & 1u) {
+                    x.x = bf16x2_to_f16x2(x.x);
+                    x.y = bf16x2_to_f16x2(x.y);
+                    x.z = bf16x2_to_f16x2(x.z);
+                    x.w = bf16x2_to_f16x2(x.w);
+                } else {
+                    x = make_uint4(0u, 0u, 0u, 0u);
+                }
+                vt[c] = x;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&v_ready[s]);
+        }
+        if (!ok && ct == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+    } else {  // -------------------------------------------------------- softmax
+        const int st = threadIdx.x - 32 * kWarpSm0;  // 0..255
+        const int mt = st >> 7, r = st & 127;
+        const int rho = row0 + mt * 128 + r;
+        const bool row_ok = seq_ok && rho < R;
+        const int lim = row_ok ? start + rho / g + 1 : 0;
+        const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
+        // Q row into the K-major swizzled tile (zeros for padding rows).
+        {
+            const uint4 *src = row_ok ? reinterpret_cast<const uint4 *>(
+                                            q_chunk + (((size_t)b * f + rho / g) * hq +
+                                                       (size_t)h * g + rho % g) * D)
+                                      : nullptr;
+            uint8_t *qt = q_s + mt * LY::kQTile;
+#pragma unroll
+            for (int hf = 0; hf < LY::kHalves; ++hf)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = src ? src[hf * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4 *>(qt + hf * LY::kQHalf + swz128(r, c)) = v;
+                }
+            fence_proxy_async_smem();
+            mbar_arrive(&q_ready);
+        }
+        float m_use = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int i = 0; i < ntiles; ++i) {
+            const int buf = i & 1;
+            ok = mbar_wait_bounded(&s_full[buf], (i / 2) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc::fence_after_sync();
+            uint32_t sv[2][32];
+            const uint32_t scol = tmem + lane_base + 2 * D + (2 * buf + mt) * kKeys;
+            tc::tmem_ld32(scol, sv[0]);
+            tc::tmem_ld32(scol + 32, sv[1]);
+            tc::tmem_wait_ld();
+            const int t0 = (blk0 + i * kBlocksPerTile) * kBlock;
+            const uint32_t vmask = stage_vmask[i % kStages];
+            const int tend = blk1 * kBlock;
+            float x[64];
+            float mtile = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const int t = t0 + j;
+                const bool valid = t < lim && t < tend && ((vmask >> (j / kBlock)) & 1u);
+                x[j] = valid ? __uint_as_float(sv[j >> 5][j & 31]) * scale_log2 : -INFINITY;
+                mtile = fmaxf(mtile, x[j]);
+            }
+            const bool need = mtile > m_use + kRescaleSlack;
+            if (__any_sync(0xffffffffu, need)) {
+                const float m_new = fmaxf(m_use, mtile);
+                const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_new);
+                l *= alpha;
+                if (i > 0) {  // O holds earlier tiles: wait for the last P.V, scale it
+                    ok = mbar_wait_bounded(&pv_done[(i - 1) & 1], ((i - 1) / 2) & 1);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int c4 = 0; c4 < D / 32; ++c4) {
+                        uint32_t ov[32];
+                        const uint32_t ocol = tmem + lane_base + mt * D + c4 * 32;
+                        tc::tmem_ld32(ocol, ov);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+                        tc::tmem_st32(ocol, ov);
+                    }
+                    tc::tmem_wait_st();
+                }
+                m_use = m_new;
+            }
+            // P buffer `buf` is free once the P.V of tile i-2 completed.
+            if (i >= 2) {
+                ok = mbar_wait_bounded(&pv_done[buf], ((i - 2) / 2) & 1);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            uint8_t *prow = p_s + (size_t)(2 * buf + mt) * LY::kP;
+            float psum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = m_use == -INFINITY ? 0.f : exp2f(x[c * 8 + 2 * e] - m_use);
+                    const float p1 = m_use == -INFINITY ? 0.f : exp2f(x[c * 8 + 2 * e + 1] - m_use);
+                    const __half2 hp = __floats2half2_rn(p0, p1);
+                    w[e] = *reinterpret_cast<const uint32_t *>(&hp);
+                    const float2 back = __half22float2(hp);
+                    psum += back.x + back.y;  // the sum of the weights the MMA sees
+                }
+                *reinterpret_cast<uint4 *>(prow + swz128(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            l += psum;
+            fence_proxy_async_smem();
+            tc::fence_before_sync();
+            mbar_arrive(&p_full[buf]);
+        }
+        if (!ok && lane == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+        // Final O row (all P.V done), normalised; partial or final output.
+        float lse2 = -INFINITY;
+        float inv = 0.f;
+        bool have = false;
+        if (ok && ntiles > 0) {
+            ok = mbar_wait_bounded(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) / 2) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            tc::fence_after_sync();
+            have = ok;
+        }
+        if (l > 0.f) {
+            lse2 = m_use + log2f(l);
+            inv = 1.f / l;
+        }
+        const float kLn2 = 0.6931471805599453f;
+        const int r_pos = rho / g, jh = rho % g;
+        const size_t orow = ((size_t)b * f + r_pos) * hq + (size_t)h * g + jh;
+        const size_t slot = ((size_t)unit * G + group) * S + split;
+        float *dst = S == 1 ? out + orow * D : part_o + (slot * kRows + mt * 128 + r) * D;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t ov[32];
+            if (have) {
+                tc::tmem_ld32(tmem + lane_base + mt * D + c4 * 32, ov);
+                tc::tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ov[j] = 0u;
+            }
+            if (rho < R) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    float4 v = make_float4(__uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv,
+                                           __uint_as_float(ov[j + 2]) * inv,
+                                           __uint_as_float(ov[j + 3]) * inv);
+                    if (!have || l <= 0.f) v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4 *>(dst + c4 * 32 + j) = v;
+                }
+            }
+        }
+        if (rho < R) {
+            if (S == 1) {
+                if (lse_out) lse_out[orow] = have ? lse2 * kLn2 : -INFINITY;
+            } else {
+                part_lse[slot * kRows + mt * 128 + r] = have ? lse2 : -INFINITY;
+            }
+        }
+    }
+
+    // Release TMEM once every TMEM access of the CTA is done.
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, LY::kTmemCols);
+    if (S == 1) return;
+
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t ticket = atomicAdd(&tickets[(size_t)unit * kMaxRowTiles + group], 1u);
+        sh_last = ticket == (uint32_t)(S - 1);
+    }
+    __syncthreads();
+    if (!sh_last) return;
+    __threadfence();
+    const size_t slot0 = ((size_t)unit * G + group) * S;
+    const int nrows = min(kRows, R - row0);
+    constexpr int C4 = D / 4;
+    for (int e = threadIdx.x; e < nrows * C4; e += kThreads) {
+        const int rl = e / C4, c4 = e % C4;
+        float mstar = -INFINITY;
+        for (int s = 0; s < S; ++s) mstar = fmaxf(mstar, __ldcg(&part_lse[(slot0 + s) * kRows + rl]));
+        float wsum = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (mstar != -INFINITY) {
+#pragma unroll 4
+            for (int s = 0; s < S; ++s) {
+                const float w = exp2f(__ldcg(&part_lse[(slot0 + s) * kRows + rl]) - mstar);
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                                            part_o + ((slot0 + s) * kRows + rl) * D) + c4);
+                wsum += w;
+                acc.x += w * v.x;
+                acc.y += w * v.y;
+                acc.z += w * v.z;
+                acc.w += w * v.w;
+            }
+        }
+        const float iw = wsum > 0.f ? 1.f / wsum : 0.f;
+        const int rho = row0 + rl;
+        const size_t orow = ((size_t)b * f + rho / g) * hq + (size_t)h * g + rho % g;
+        reinterpret_cast<float4 *>(out + orow * D)[c4] =
+            make_float4(acc.x * iw, acc.y * iw, acc.z * iw, acc.w * iw);
+        if (lse_out && c4 == 0)
+            lse_out[orow] = wsum > 0.f ? (mstar + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+    }
+    if (threadIdx.x == 0) tickets[(size_t)unit * kMaxRowTiles + group] = 0;
+}
+
+template <int D>
+cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *page_table,
+                      const int32_t *seq_len, int f, const void *q_chunk, int groups, int splits,
+                      float *part_o, float *part_lse, uint32_t *tickets, float *out, float *lse,
+                      uint32_t *err, cudaStream_t st) {
+    constexpr int smem = TcLayout<D>::kBytes;
+    static std::atomic<int> done[64];
+    cudaError_t e = ensure_smem(rectify_tc_kernel<D>, smem, done);
+    if (e != cudaSuccess) return e;
+    const float scale_log2 = s.sm_scale * 1.4426950408889634f;
+    dim3 grid(groups, splits, s.batch * s.hkv);
+    rectify_tc_kernel<D><<<grid, kThreads, smem, st>>>(
+        maps[0], maps[1], maps[2], maps[3], page_table, seq_len, f, (const uint16_t *)q_chunk,
+        s.hkv, s.g, s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out, lse,
+        err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap *maps,
+                                     const int32_t *page_table, const int32_t *seq_len, int f,
+                                     const void *q_chunk, int groups, int splits, float *part_o,
+                                     float *part_lse, uint32_t *tickets, float *out, float *lse,
+                                     uint32_t *err, cudaStream_t st) {
+    if (groups > kMaxRowTiles) return cudaErrorInvalidValue;
+    if (s.d == 128)
+        return launch_tc<128>(s, maps, page_table, seq_len, f, q_chunk, groups, splits, part_o,
+                              part_lse, tickets, out, lse, err, st);
+    if (s.d == 64)
+        return launch_tc<64>(s, maps, page_table, seq_len, f, q_chunk, groups, splits, part_o,
+                             part_lse, tickets, out, lse, err, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace resa

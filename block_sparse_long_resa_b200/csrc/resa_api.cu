@@ -42,6 +42,23 @@ bool make_kv_map(CUtensorMap *map, void *base, int num_pages, int hkv, int d) {
     return r == CUDA_SUCCESS;
 }
 
+// One channel half (64 columns) of a K or V cache as a 2-D tensor: rows are
+// tokens of every (page, head) block (row stride d*2 bytes); one box is the
+// 16 rows x 64 channels of one block, 128-byte swizzled.
+bool make_kv_half_map(CUtensorMap *map, void *base, int half, int num_pages, int hkv, int d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    void *b = static_cast<uint8_t *>(base) + (size_t)half * 128;
+    const cuuint64_t dims[2] = {64, (cuuint64_t)num_pages * hkv * kBlock};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kBlock};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 resa_status_t check_config(const resa_config_t *cfg, Shape *s) {
@@ -108,13 +125,20 @@ WsLayout layout_of(const Shape &s, int chunk) {
 }
 
 
+// Score (optionally appending the decode token in the same launch), then select.
 resa_status_t select_impl(const Shape &s, const resa_cache_t *c, const WsLayout &w, void *ws,
                           const void *q, const int32_t *topk, int max_topk, int32_t *idx,
-                          int32_t *cnt, float *scores, cudaStream_t st) {
+                          int32_t *cnt, float *scores, const void *k_new, const void *v_new,
+                          cudaStream_t st) {
     uint32_t *err = at<uint32_t>(ws, w.err);
-    RESA_TRY(cuda_status(launch_score(s, c->desc, c->page_table, c->seq_len, q, scores, err, st)));
-    RESA_TRY(cuda_status(
-        launch_select(s, scores, c->seq_len, topk, max_topk, idx, cnt, err, st)));
+    uint32_t *hist = at<uint32_t>(ws, w.hist);
+    uint32_t *range = at<uint32_t>(ws, w.hist_range);
+    const bool append = k_new != nullptr;
+    RESA_TRY(cuda_status(launch_score(s, c->desc, c->page_table, c->seq_len, q, scores, hist,
+                                      range, append ? c->k : nullptr, append ? c->v : nullptr,
+                                      k_new, v_new, err, st)));
+    RESA_TRY(cuda_status(launch_select(s, scores, hist, range, c->seq_len, topk, max_topk, idx,
+                                       cnt, err, st)));
     return RESA_OK;
 }
 
@@ -147,7 +171,7 @@ size_t resa_workspace_size(const resa_config_t *cfg, int32_t batch, int32_t max_
         return 0;
     size_t best = ws_layout(s.hq, s.hkv, s.d, batch, max_pages, 0).total;
     for (int f = 1; f <= max_chunk; ++f) {
-        if (rect_row_tiles(f, s.g) > kMaxRowTiles) break;
+        if (rect_row_groups(f, s.g) > kMaxRowTiles) break;
         const size_t t = ws_layout(s.hq, s.hkv, s.d, batch, max_pages, f).total;
         best = t > best ? t : best;
     }
@@ -219,7 +243,8 @@ resa_status_t resa_select_blocks(const resa_config_t *cfg, const resa_cache_t *c
     const WsLayout w = layout_of(s, 0);
     RESA_TRY(check_ws(ws, ws_bytes, w));
     float *scores = scores_opt ? scores_opt : at<float>(ws, w.scores);
-    return select_impl(s, cache, w, ws, q, topk, max_topk, block_idx, block_cnt, scores, stream);
+    return select_impl(s, cache, w, ws, q, topk, max_topk, block_idx, block_cnt, scores, nullptr,
+                       nullptr, stream);
 }
 
 resa_status_t resa_sparse_decode(const resa_config_t *cfg, const resa_cache_t *cache,
@@ -246,7 +271,7 @@ resa_status_t resa_rectify_attention(const resa_config_t *cfg, const resa_cache_
     RESA_TRY(check_cache(cache, &s, true, true));
     if (!q_chunk || !k_new || !v_new || !out) return RESA_ERR_NULL;
     if (f < 1) return RESA_ERR_RANGE;
-    if (rect_row_tiles(f, s.g) > kMaxRowTiles) return RESA_ERR_UNSUPPORTED;
+    if (rect_row_groups(f, s.g) > kMaxRowTiles) return RESA_ERR_UNSUPPORTED;
     if (!aligned16(q_chunk) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out))
         return RESA_ERR_UNSUPPORTED;
     const WsLayout w = layout_of(s, f);
@@ -255,12 +280,16 @@ resa_status_t resa_rectify_attention(const resa_config_t *cfg, const resa_cache_
     RESA_TRY(cuda_status(launch_rectify_writeback(s, cache->k, cache->v, cache->desc,
                                                   cache->page_table, cache->seq_len, f, k_new,
                                                   v_new, err, stream)));
-    CUtensorMap kmap, vmap;
-    if (!make_kv_map(&kmap, cache->k, s.num_pages, s.hkv, s.d) ||
-        !make_kv_map(&vmap, cache->v, s.num_pages, s.hkv, s.d))
-        return RESA_ERR_CUDA;
+    CUtensorMap maps[4];
+    const int halves = s.d / 64;
+    for (int hf = 0; hf < 2; ++hf) {
+        const int use = hf < halves ? hf : 0;  // d = 64: one half, second map unused
+        if (!make_kv_half_map(&maps[hf], cache->k, use, s.num_pages, s.hkv, s.d) ||
+            !make_kv_half_map(&maps[2 + hf], cache->v, use, s.num_pages, s.hkv, s.d))
+            return RESA_ERR_CUDA;
+    }
     return cuda_status(launch_rectify_attention(
-        s, kmap, vmap, cache->page_table, cache->seq_len, f, q_chunk, w.row_tiles, w.rect_splits,
+        s, maps, cache->page_table, cache->seq_len, f, q_chunk, w.row_tiles, w.rect_splits,
         at<float>(ws, w.rect_o), at<float>(ws, w.rect_lse), at<uint32_t>(ws, w.rect_ticket), out,
         lse_opt, err, stream));
 }
@@ -284,11 +313,10 @@ resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cac
     RESA_TRY(check_ws(ws, ws_bytes, w));
     int32_t *idx = block_idx_opt && block_cnt_opt ? block_idx_opt : at<int32_t>(ws, w.sel_idx);
     int32_t *cnt = block_idx_opt && block_cnt_opt ? block_cnt_opt : at<int32_t>(ws, w.sel_cnt);
-    RESA_TRY(cuda_status(launch_append(s, cache->k, cache->v, cache->desc, cache->page_table,
-                                       cache->seq_len, k_new, v_new, at<uint32_t>(ws, w.err),
-                                       stream)));
+    // append + scores in one launch (the append touches only the current
+    // block, which is never scored), then select, then attend
     RESA_TRY(select_impl(s, cache, w, ws, q, topk, max_topk, idx, cnt, at<float>(ws, w.scores),
-                         stream));
+                         k_new, v_new, stream));
     return decode_impl(s, cache, w, ws, q, idx, cnt, max_topk, out, lse_opt, stream);
 }
 
@@ -299,7 +327,7 @@ int32_t resa_kernels_per_call(const char *entry_point) {
         int n;
     } table[] = {{"resa_build_descriptors", 1}, {"resa_append_token", 1},
                  {"resa_select_blocks", 2},     {"resa_sparse_decode", 1},
-                 {"resa_rectify_attention", 2}, {"resa_decode_step", 4},
+                 {"resa_rectify_attention", 2}, {"resa_decode_step", 3},
                  {"resa_sparse_decode_noalloc", 1}};
     for (auto &e : table)
         if (strcmp(e.name, entry_point) == 0) return e.n;

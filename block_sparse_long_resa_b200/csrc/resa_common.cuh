@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "../../include/resa.h"
 
@@ -39,14 +40,15 @@ inline int decode_max_splits(int batch, int hkv, int max_pages) {
     const int want = (kNumSms + units - 1) / units;
     return want > need ? want : need;
 }
-constexpr int kRectRowsPerTile = 64;    // query rows (chunk position x group head) per CTA
-inline int rect_row_tiles(int max_chunk, int group) {
-    int rows = max_chunk * group;
-    return (rows + kRectRowsPerTile - 1) / kRectRowsPerTile;
+constexpr int kRectRowsPerCta = 256;  // query rows (chunk position x group head) per CTA
+inline int rect_row_groups(int chunk, int group) {
+    const int rows = chunk * group;
+    return (rows + kRectRowsPerCta - 1) / kRectRowsPerCta;
 }
-inline int rect_max_splits(int batch, int hkv, int row_tiles) {
-    int units = batch * hkv * (row_tiles > 0 ? row_tiles : 1);
-    int s = (2 * 148 + units - 1) / units;
+// One CTA per SM over all (unit, row group) pairs.
+inline int rect_splits_for(int batch, int hkv, int groups) {
+    const int units = batch * hkv * (groups > 0 ? groups : 1);
+    const int s = kNumSms / units;
     return s < 1 ? 1 : (s > 64 ? 64 : s);
 }
 
@@ -56,22 +58,24 @@ inline int rect_max_splits(int batch, int hkv, int row_tiles) {
 // rectification calls of different chunk sizes find the same regions; the
 // rectification partials come last.
 // ---------------------------------------------------------------------------
-constexpr int kMaxRowTiles = 64;  // rectification row tiles per (sequence, kv head)
+constexpr int kMaxRowTiles = 64;  // rectification row groups per (sequence, kv head)
 
 struct WsLayout {
     size_t err;          // uint32 error word
     size_t dec_ticket;   // uint32 [B][Hkv]
     size_t rect_ticket;  // uint32 [B][Hkv][kMaxRowTiles]
+    size_t hist;         // uint32 [B][Hkv][65536] score-key histogram (kept zero between calls)
+    size_t hist_range;   // uint32 [B][Hkv][2] touched-bin range (kept zero between calls)
     size_t scores;       // f32 [B][Hkv][max_pages]
     size_t sel_idx;      // i32 [B][Hkv][max_pages + 1]
     size_t sel_cnt;      // i32 [B][Hkv]
     size_t dec_o;        // f32 [B][Hkv][dec_splits][kMaxGroup][d]
     size_t dec_lse;      // f32 [B][Hkv][dec_splits][kMaxGroup]
-    size_t rect_o;       // f32 [B][Hkv][row_tiles][rect_splits][kRectRowsPerTile][d]
-    size_t rect_lse;     // f32 [B][Hkv][row_tiles][rect_splits][kRectRowsPerTile]
+    size_t rect_o;       // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta][d]
+    size_t rect_lse;     // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta]
     size_t total;
     int dec_splits;
-    int row_tiles;
+    int row_tiles;   // rectification row groups of kRectRowsPerCta
     int rect_splits;
 };
 
@@ -88,18 +92,20 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     };
     int g = hkv > 0 ? hq / hkv : 1;
     w.dec_splits = decode_max_splits(batch, hkv, max_pages);
-    w.row_tiles = chunk > 0 ? rect_row_tiles(chunk, g) : 0;
-    w.rect_splits = chunk > 0 ? rect_max_splits(batch, hkv, w.row_tiles) : 0;
+    w.row_tiles = chunk > 0 ? rect_row_groups(chunk, g) : 0;
+    w.rect_splits = chunk > 0 ? rect_splits_for(batch, hkv, w.row_tiles) : 0;
     size_t units = (size_t)batch * hkv;
     w.err = take(256);
     w.dec_ticket = take(units * 4);
     w.rect_ticket = take(units * kMaxRowTiles * 4);
+    w.hist = take(units * 65536 * 4);
+    w.hist_range = take(units * 2 * 4);
     w.scores = take(units * max_pages * 4);
     w.sel_idx = take(units * (max_pages + 1) * 4);
     w.sel_cnt = take(units * 4);
     w.dec_o = take(units * w.dec_splits * kMaxGroup * d * 4);
     w.dec_lse = take(units * w.dec_splits * kMaxGroup * 4);
-    size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerTile;
+    size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerCta;
     w.rect_o = take(rect_rows * d * 4);
     w.rect_lse = take(rect_rows * 4);
     w.total = off;
@@ -180,6 +186,23 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// TMA: contiguous bulk copy global -> shared (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes,
+                                          uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding grid's completion and
+// memory; allow the next grid to be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_next() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Warp-level tensor-core helpers (bf16 in, fp32 accumulate) ------------------
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -237,6 +260,25 @@ inline cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<int> (&done
     return e;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel in the stream drains; it must execute pdl_wait() before
+// touching anything an earlier kernel writes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // Host-side launchers (defined in the kernel translation units)
 // ---------------------------------------------------------------------------
@@ -256,22 +298,26 @@ cudaError_t launch_rectify_writeback(const Shape &s, void *k, void *v, void *des
                                      const int32_t *page_table, const int32_t *seq_len, int f,
                                      const void *k_new, const void *v_new, uint32_t *err,
                                      cudaStream_t st);
-cudaError_t launch_score(const Shape &s, const void *desc, const int32_t *page_table,
-                         const int32_t *seq_len, const void *q, float *scores, uint32_t *err,
-                         cudaStream_t st);
-cudaError_t launch_select(const Shape &s, const float *scores, const int32_t *seq_len,
-                          const int32_t *topk, int max_topk, int32_t *block_idx,
-                          int32_t *block_cnt, uint32_t *err, cudaStream_t st);
+// Scores every complete block; with K != nullptr it also appends the decode
+// token (k_new / v_new) in the same launch.
+cudaError_t launch_score(const Shape &s, void *desc, const int32_t *page_table,
+                         const int32_t *seq_len, const void *q, float *scores, uint32_t *hist,
+                         uint32_t *hist_range, void *K, void *V, const void *k_new,
+                         const void *v_new, uint32_t *err, cudaStream_t st);
+cudaError_t launch_select(const Shape &s, const float *scores, uint32_t *hist,
+                          uint32_t *hist_range, const int32_t *seq_len, const int32_t *topk,
+                          int max_topk, int32_t *block_idx, int32_t *block_cnt, uint32_t *err,
+                          cudaStream_t st);
 cudaError_t launch_sparse_decode(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
                                  const int32_t *page_table, const int32_t *seq_len, const void *q,
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
                                  float *out, float *lse, uint32_t *err, cudaStream_t st);
-cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap &kmap,
-                                     const CUtensorMap &vmap, const int32_t *page_table,
-                                     const int32_t *seq_len, int f, const void *q_chunk,
-                                     int row_tiles, int splits, float *part_o, float *part_lse,
-                                     uint32_t *tickets, float *out, float *lse, uint32_t *err,
-                                     cudaStream_t st);
+// maps: K half 0, K half 1, V half 0, V half 1 (2-D, 16 x 64 boxes, 128-byte swizzle).
+cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap *maps,
+                                     const int32_t *page_table, const int32_t *seq_len, int f,
+                                     const void *q_chunk, int groups, int splits, float *part_o,
+                                     float *part_lse, uint32_t *tickets, float *out, float *lse,
+                                     uint32_t *err, cudaStream_t st);
 
 }  // namespace resa

@@ -170,8 +170,9 @@ RESA_API resa_status_t resa_rectify_attention(const resa_config_t *cfg, const re
                                      size_t ws_bytes, cudaStream_t stream);
 
 /* One sparse decode step of one layer (Algorithm 1 inner body): append the
- * decode token (resa_append_token), select blocks (resa_select_blocks) and
- * attend (resa_sparse_decode).  seq_len must already count the decode token.
+ * decode token (as resa_append_token, fused into the scoring launch), select
+ * blocks (resa_select_blocks) and attend (resa_sparse_decode).  seq_len must
+ * already count the decode token.
  * block_idx_opt / block_cnt_opt (nullable) receive the selection; when NULL
  * it lives in the workspace. */
 RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cache,
@@ -212,8 +213,8 @@ RESA_API resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
 
 /* Number of kernels each entry point launches per call (for launch
  * accounting): 1 for append and build, 2 for select, 1 for sparse decode,
- * 2 for rectify, 4 for a decode step, 1 for the no-allocation decode.
- * Unknown names return -1. */
+ * 2 for rectify, 3 for a decode step (append fused with scoring), 1 for the
+ * no-allocation decode.  Unknown names return -1. */
 RESA_API int32_t resa_kernels_per_call(const char *entry_point);
 
 /* Human-readable status name. */
