@@ -563,6 +563,7 @@ def run_resa(args):
                           "peak": hbm_peak, "unit": "GB/s", "frac": step_gbs / hbm_peak},
         "rectify": rect,
         "kernel_breakdown_us": bd,
+        "sparse_vs_dense_step_speedup": bd["dense_decode_step_us"] / bd["decode_step_us"],
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": K * w.launches_per_cycle(),
@@ -624,6 +625,17 @@ def kernel_breakdown(w, stream, device, reps):
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
         w.topk_ptr(row), w.max_topk, w.out[l], None, w.idx[l], w.cnt[l], w.ws)
         for l in range(n)], n)
+    # dense decode for comparison: the same step with top-k = every block (Eq. 1 path)
+    Ls = w.sched.decode_L(c, w.f - 2)
+    all_k = max((L - 1) // 16 for L in Ls)
+    topk_all = torch.full((w.sched.Bpad,), all_k, dtype=torch.int32, device=device)
+    dense_idx = [torch.empty(w.B, w.hkv, all_k + 1, dtype=torch.int32, device=device)
+                 for _ in range(n)]
+    res["dense_decode_step_us"] = timed(lambda: [R.resa_decode_step(
+        w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
+        topk_all, all_k, w.out[l], None, dense_idx[l], scratch_cnt[l], w.ws)
+        for l in range(n)], n)
+    del dense_idx
     res["rectify_us"] = timed(lambda: [R.resa_rectify_attention(
         w.cfg, w.cache(l, rrow), w.f, w.qc[c, l], w.kc[c, l], w.vc[c, l], w.rout[l], None, w.ws)
         for l in range(n)], n)

@@ -35,6 +35,8 @@ struct DecodeSmem {
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
     static constexpr int kMergeBytes = kWarps * kMaxGroup * (D + 3) * 4;
+    // split merge: weights [S][16] floats + [threads / (D/4)][16][D/4] float4 partial sums
+    static constexpr int kSplitMergeBytes = (kThreads / (D / 4)) * kMaxGroup * D * 4;
     static constexpr int kBytes = (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes) + 1024;
 };
 
@@ -361,19 +363,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) sh_lse[r] = sum > 0.f ? mstar + log2f(sum) : -INFINITY;
     }
     __syncthreads();
+    // (The ring region holds wts then red: S*64 + kSplitMergeBytes <= ring bytes
+    // for every split count the workspace allows.)
+    // Thread (split group sg, float4 column c4) accumulates every row over
+    // splits sg, sg + 8, ...: all its loads are independent and in flight
+    // together; the eight split groups are then summed through shared memory.
     constexpr int C4 = D / 4;
+    constexpr int SG = kThreads / C4;  // split groups
+    float4 *red = reinterpret_cast<float4 *>(wts + S * kMaxGroup);  // [SG][16][C4]
+    {
+        const int c4 = threadIdx.x % C4, sg = threadIdx.x / C4;
+        float4 acc[kMaxGroup];
+#pragma unroll
+        for (int r = 0; r < kMaxGroup; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = sg; sp < S; sp += SG) {
+            const float4 *src = reinterpret_cast<const float4 *>(uo + (size_t)sp * kMaxGroup * D) + c4;
+#pragma unroll
+            for (int r = 0; r < kMaxGroup; ++r) {
+                if (r < g) {
+                    const float w = wts[sp * kMaxGroup + r];
+                    const float4 v = __ldcg(src + (size_t)r * C4);
+                    acc[r].x += w * v.x;
+                    acc[r].y += w * v.y;
+                    acc[r].z += w * v.z;
+                    acc[r].w += w * v.w;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kMaxGroup; ++r)
+            if (r < g) red[((size_t)sg * kMaxGroup + r) * C4 + c4] = acc[r];
+    }
+    __syncthreads();
     for (int item = threadIdx.x; item < g * C4; item += kThreads) {
         const int r = item / C4, c4 = item % C4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 *src = reinterpret_cast<const float4 *>(uo + (size_t)r * D) + c4;
-#pragma unroll 8
-        for (int s = 0; s < S; ++s) {
-            const float w = wts[s * kMaxGroup + r];
-            const float4 v = __ldcg(src + (size_t)s * kMaxGroup * C4);
-            acc.x += w * v.x;
-            acc.y += w * v.y;
-            acc.z += w * v.z;
-            acc.w += w * v.w;
+#pragma unroll
+        for (int sg = 0; sg < SG; ++sg) {
+            const float4 v = red[((size_t)sg * kMaxGroup + r) * C4 + c4];
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
         }
         const size_t orow = (size_t)b * hq + (size_t)h * g + r;
         reinterpret_cast<float4 *>(out + orow * D)[c4] = acc;

@@ -166,26 +166,32 @@ __global__ void rectify_writeback_kernel(uint4 *__restrict__ K, uint4 *__restric
         return;
     }
     const int nt = min(kBlock, L - blk * kBlock);
-    Bf16x8 mn, mx;
-    for (int t = 0; t < nt; ++t) {
+    // All token loads of the block first (fresh chunk values or the cached
+    // keys), then the writes and the position-order min/max fold.
+    uint4 kx[kBlock], vx[kBlock];
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t) {
         const int pos = blk * kBlock + t;
-        uint4 kx;
-        const size_t o = kv_off(page, h, t, c, hkv, d);
-        if (pos >= start) {
-            const size_t src = ((((size_t)b * f + (pos - start)) * hkv + h) * d) / 8 + c;
-            kx = k_new[src];
-            K[o] = kx;
-            V[o] = v_new[src];
-        } else {
-            kx = K[o];
+        if (t < nt) {
+            if (pos >= start) {
+                const size_t src = ((((size_t)b * f + (pos - start)) * hkv + h) * d) / 8 + c;
+                kx[t] = k_new[src];
+                vx[t] = v_new[src];
+            } else {
+                kx[t] = K[kv_off(page, h, t, c, hkv, d)];
+            }
         }
-        const Bf16x8 x = unpack(kx);
-        if (t == 0) {
-            mn = x;
-            mx = x;
-        } else {
-            fold(mn, mx, x);
+    }
+    Bf16x8 mn = unpack(kx[0]), mx = mn;
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t) {
+        const int pos = blk * kBlock + t;
+        if (t < nt && pos >= start) {
+            const size_t o = kv_off(page, h, t, c, hkv, d);
+            K[o] = kx[t];
+            V[o] = vx[t];
         }
+        if (t > 0 && t < nt) fold(mn, mx, unpack(kx[t]));
     }
     desc[desc_off(page, h, 0, c, hkv, d)] = pack(mn);
     desc[desc_off(page, h, 1, c, hkv, d)] = pack(mx);

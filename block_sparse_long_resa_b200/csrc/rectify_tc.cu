@@ -17,13 +17,16 @@
 //   warps 2-3   convert the V tile bf16 -> fp16 in place (exact for
 //               |v| < 65504), zero blocks that were not loaded;
 //   warps 4-11  softmax, one thread per query row (TMEM lane): tcgen05.ld of
-//               the S row, causal mask, base-2 online softmax with lazy O
-//               rescaling (only when the row maximum grows by more than 8),
-//               P written to shared memory as fp16 in the canonical K-major
-//               swizzled layout.
+//               the S row, causal mask (skipped for interior tiles), base-2
+//               online softmax with lazy O rescaling (only when the row
+//               maximum grows by more than 8), P written to shared memory as
+//               fp16 in the canonical K-major swizzled layout.
+// Three K/V stages are in flight (released per stage by the P.V commit); the
+// P tile is single-buffered, written once the previous P.V has completed.
 // P is fp16 (11-bit mantissa), so the P.V product keeps the weights' precision
-// without a second MMA.  Partial (o, lse) per split are merged by the CTA that
-// draws the last ticket of its (unit, row group).  Waits are bounded.
+// without a second MMA.  With several splits the grid is launched
+// cooperatively; after a bounded grid barrier every CTA merges an equal share
+// of all rows' partial (o, lse).  Waits are bounded.
 #include "tc_common.cuh"
 
 namespace resa {
@@ -32,7 +35,7 @@ namespace {
 constexpr int kRows = kRectRowsPerCta;  // 256
 constexpr int kKeys = 64;               // keys per KV tile
 constexpr int kBlocksPerTile = kKeys / kBlock;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kNumConv = 2;             // converter warps
 constexpr int kWarpSm0 = 4;             // first softmax warp
 constexpr int kNumSm = 8;               // softmax warps
@@ -52,10 +55,20 @@ struct TcLayout {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = kQOff + 2 * kQTile;
     static constexpr int kPOff = kKVOff + kStages * 2 * kKV;
-    static constexpr int kBytes = kPOff + 2 * 2 * kP + 1024;
+    static constexpr int kBytes = kPOff + 2 * kP + 1024;  // one P buffer per M tile
     // TMEM columns: O[mt] at mt*D, S[buf][mt] at 2*D + (2*buf + mt)*64.
     static constexpr uint32_t kTmemCols = 512;
 };
+
+__device__ __forceinline__ float ex2(float x) {  // hardware base-2 exponential
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
     const __half2 h = __floats2half2_rn(bf_lo(x), bf_hi(x));
@@ -77,11 +90,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    __shared__ uint64_t q_ready, kv_full[kStages], v_ready[kStages], s_full[2], p_full[2],
-        pv_done[2];
+    __shared__ uint64_t q_ready, kv_full[kStages], v_ready[kStages], kv_empty[kStages], s_full[2],
+        p_full, pv_done;
     __shared__ uint32_t tmem_base_s;
     __shared__ uint32_t stage_vmask[kStages];
-    __shared__ uint32_t sh_last;
 
     const int group = blockIdx.x, split = blockIdx.y, unit = blockIdx.z;
     const int G = gridDim.x, S = gridDim.y;
@@ -113,12 +125,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&v_ready[s], kConvThreads);
+            mbar_init(&kv_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], kSmThreads);
-            mbar_init(&pv_done[s], 1);
-        }
+        for (int s = 0; s < 2; ++s) mbar_init(&s_full[s], 1);
+        mbar_init(&p_full, kSmThreads);
+        mbar_init(&pv_done, 1);
         fence_mbar_init();
     }
     if (warp == 1) tc::tmem_alloc(&tmem_base_s, LY::kTmemCols);
@@ -131,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % kStages;
-            if (i >= kStages) ok = mbar_wait_bounded(&pv_done[s], ((i - kStages) / 2) & 1);
+            if (i >= kStages) ok = mbar_wait_bounded(&kv_empty[s], ((i / kStages) - 1) & 1);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             const int blk = blk0 + i * kBlocksPerTile + lane;
@@ -200,14 +211,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     issue_qk(i + 1);  // S[(i+1)&1] was released by the softmax of tile i-1
                 }
-                ok = mbar_wait_bounded(&p_full[buf], (i / 2) & 1) &&
+                ok = mbar_wait_bounded(&p_full, i & 1) &&
                      mbar_wait_bounded(&v_ready[s], (i / kStages) & 1);
                 tc::fence_after_sync();
                 if (!ok) break;
                 const uint32_t vt = smem_u32(kv_s + (size_t)s * 2 * LY::kKV + LY::kKV);
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
-                    const uint32_t pt = smem_u32(p_s + (size_t)(2 * buf + mt) * LY::kP);
+                    const uint32_t pt = smem_u32(p_s + (size_t)mt * LY::kP);
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk) {
                         const uint64_t a = tc::smem_desc(pt + kk * 32, 16, 1024);
@@ -216,7 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        (i > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                tc::commit(&pv_done[buf]);
+                tc::commit(&pv_done);
+                tc::commit(&kv_empty[s]);
             }
             if (!ok) set_error(err, RESA_DEVERR_TIMEOUT);
         }
@@ -275,6 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float m_use = -INFINITY, l = 0.f;
         bool ok = true;
+        // Keys every valid row of this CTA may see: tiles entirely below this
+        // limit (and fully loaded) need no mask.
+        const int lim_cta = seq_ok ? start + row0 / g + 1 : 0;
+        const int tend = blk1 * kBlock;
         for (int i = 0; i < ntiles; ++i) {
             const int buf = i & 1;
             ok = mbar_wait_bounded(&s_full[buf], (i / 2) & 1);
@@ -288,26 +304,58 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tmem_wait_ld();
             const int t0 = (blk0 + i * kBlocksPerTile) * kBlock;
             const uint32_t vmask = stage_vmask[i % kStages];
-            const int tend = blk1 * kBlock;
-            float x[64];
-            float mtile = -INFINITY;
+            const bool full_tile = vmask == 0xFu && t0 + kKeys <= tend && t0 + kKeys <= lim_cta;
+            float x[64];  // raw logits; -inf where masked
+            float mraw = -INFINITY;
+            if (full_tile) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const int t = t0 + j;
-                const bool valid = t < lim && t < tend && ((vmask >> (j / kBlock)) & 1u);
-                x[j] = valid ? __uint_as_float(sv[j >> 5][j & 31]) * scale_log2 : -INFINITY;
-                mtile = fmaxf(mtile, x[j]);
+                for (int j = 0; j < 64; ++j) {
+                    x[j] = __uint_as_float(sv[j >> 5][j & 31]);
+                    mraw = fmaxf(mraw, x[j]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const int t = t0 + j;
+                    const bool valid = t < lim && t < tend && ((vmask >> (j / kBlock)) & 1u);
+                    x[j] = valid ? __uint_as_float(sv[j >> 5][j & 31]) : -INFINITY;
+                    mraw = fmaxf(mraw, x[j]);
+                }
             }
+            const float mtile = mraw * scale_log2;  // scale > 0 keeps the maximum
             const bool need = mtile > m_use + kRescaleSlack;
-            if (__any_sync(0xffffffffu, need)) {
+            const bool rescale = __any_sync(0xffffffffu, need);
+            float alpha = 1.f;
+            if (rescale) {
                 const float m_new = fmaxf(m_use, mtile);
-                const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_new);
+                alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_new);
+                m_use = m_new;
                 l *= alpha;
-                if (i > 0) {  // O holds earlier tiles: wait for the last P.V, scale it
-                    ok = mbar_wait_bounded(&pv_done[(i - 1) & 1], ((i - 1) / 2) & 1);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc::fence_after_sync();
+            }
+            // Weights in registers (fp16 pairs) before touching the shared P tile.
+            uint32_t pw[32];
+            float psum = 0.f;
+            if (m_use == -INFINITY) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pw[e] = 0u;
+            } else {
+                const float nm = -m_use;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = ex2(fmaf(x[2 * e], scale_log2, nm));
+                    const float p1 = ex2(fmaf(x[2 * e + 1], scale_log2, nm));
+                    psum += p0 + p1;
+                    pw[e] = f16x2(p0, p1);
+                }
+            }
+            l += psum;
+            // The single P tile and O are free once the P.V of tile i-1 completed.
+            if (i > 0) {
+                ok = mbar_wait_bounded(&pv_done, (i - 1) & 1);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc::fence_after_sync();
+                if (rescale) {
 #pragma unroll
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         uint32_t ov[32];
@@ -321,34 +369,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc::tmem_wait_st();
                 }
-                m_use = m_new;
             }
-            // P buffer `buf` is free once the P.V of tile i-2 completed.
-            if (i >= 2) {
-                ok = mbar_wait_bounded(&pv_done[buf], ((i - 2) / 2) & 1);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-            }
-            uint8_t *prow = p_s + (size_t)(2 * buf + mt) * LY::kP;
-            float psum = 0.f;
+            uint8_t *prow = p_s + (size_t)mt * LY::kP;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = m_use == -INFINITY ? 0.f : exp2f(x[c * 8 + 2 * e] - m_use);
-                    const float p1 = m_use == -INFINITY ? 0.f : exp2f(x[c * 8 + 2 * e + 1] - m_use);
-                    const __half2 hp = __floats2half2_rn(p0, p1);
-                    w[e] = *reinterpret_cast<const uint32_t *>(&hp);
-                    const float2 back = __half22float2(hp);
-                    psum += back.x + back.y;  // the sum of the weights the MMA sees
-                }
-                *reinterpret_cast<uint4 *>(prow + swz128(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            l += psum;
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(prow + swz128(r, c)) =
+                    make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             fence_proxy_async_smem();
             tc::fence_before_sync();
-            mbar_arrive(&p_full[buf]);
+            mbar_arrive(&p_full);
         }
         if (!ok && lane == 0) set_error(err, RESA_DEVERR_TIMEOUT);
         // Final O row (all P.V done), normalised; partial or final output.
@@ -356,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float inv = 0.f;
         bool have = false;
         if (ok && ntiles > 0) {
-            ok = mbar_wait_bounded(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) / 2) & 1);
+            ok = mbar_wait_bounded(&pv_done, (ntiles - 1) & 1);
             ok = __all_sync(0xffffffffu, ok);
             tc::fence_after_sync();
             have = ok;
@@ -407,46 +436,94 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tc::tmem_dealloc(tmem, LY::kTmemCols);
     if (S == 1) return;
 
+    // Every CTA of the (cooperatively launched, co-resident) grid has written
+    // its partials: bounded grid barrier, then each CTA merges its share of
+    // all rows.  tickets[0] counts arrivals, tickets[1] is the generation.
     __threadfence();
     __syncthreads();
+    __shared__ uint32_t sh_ok;
+    const uint32_t nctas = gridDim.x * gridDim.y * gridDim.z;
     if (threadIdx.x == 0) {
-        const uint32_t ticket = atomicAdd(&tickets[(size_t)unit * kMaxRowTiles + group], 1u);
-        sh_last = ticket == (uint32_t)(S - 1);
-    }
-    __syncthreads();
-    if (!sh_last) return;
-    __threadfence();
-    const size_t slot0 = ((size_t)unit * G + group) * S;
-    const int nrows = min(kRows, R - row0);
-    constexpr int C4 = D / 4;
-    for (int e = threadIdx.x; e < nrows * C4; e += kThreads) {
-        const int rl = e / C4, c4 = e % C4;
-        float mstar = -INFINITY;
-        for (int s = 0; s < S; ++s) mstar = fmaxf(mstar, __ldcg(&part_lse[(slot0 + s) * kRows + rl]));
-        float wsum = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (mstar != -INFINITY) {
-#pragma unroll 4
-            for (int s = 0; s < S; ++s) {
-                const float w = exp2f(__ldcg(&part_lse[(slot0 + s) * kRows + rl]) - mstar);
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(
-                                            part_o + ((slot0 + s) * kRows + rl) * D) + c4);
-                wsum += w;
-                acc.x += w * v.x;
-                acc.y += w * v.y;
-                acc.z += w * v.z;
-                acc.w += w * v.w;
+        volatile uint32_t *gen_p = tickets + 1;
+        const uint32_t gen = *gen_p;
+        __threadfence();
+        const uint32_t ticket = atomicAdd(&tickets[0], 1u);
+        uint32_t ok = 1;
+        if (ticket == nctas - 1) {
+            tickets[0] = 0;
+            __threadfence();
+            atomicAdd(&tickets[1], 1u);
+        } else {
+            uint32_t polls = 0;
+            while (*gen_p == gen) {
+                if (++polls > (1u << 24)) {
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(64);
             }
         }
-        const float iw = wsum > 0.f ? 1.f / wsum : 0.f;
-        const int rho = row0 + rl;
-        const size_t orow = ((size_t)b * f + rho / g) * hq + (size_t)h * g + rho % g;
-        reinterpret_cast<float4 *>(out + orow * D)[c4] =
-            make_float4(acc.x * iw, acc.y * iw, acc.z * iw, acc.w * iw);
-        if (lse_out && c4 == 0)
-            lse_out[orow] = wsum > 0.f ? (mstar + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+        sh_ok = ok;
     }
-    if (threadIdx.x == 0) tickets[(size_t)unit * kMaxRowTiles + group] = 0;
+    __syncthreads();
+    if (!sh_ok) {
+        if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+        return;
+    }
+    __threadfence();
+    const int units = gridDim.z;
+    const int total = units * R;
+    const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    const int per_cta = (total + nctas - 1) / nctas;
+    const int i0 = cta * per_cta, i1 = min(total, i0 + per_cta);
+    float *wts = reinterpret_cast<float *>(smem);  // [per_cta][S] merge weights
+    float *lse_s = wts + per_cta * S;              // [per_cta]
+    auto slot_row = [&](int item, int sp) -> size_t {
+        const int u = item / R, rho = item % R;
+        return (((size_t)u * G + rho / kRows) * S + sp) * kRows + rho % kRows;
+    };
+    for (int e = threadIdx.x; e < (i1 - i0) * S; e += kThreads) {
+        const int it = e / S, sp = e % S;
+        wts[it * S + sp] = __ldcg(&part_lse[slot_row(i0 + it, sp)]);
+    }
+    __syncthreads();
+    for (int it = warp; it < i1 - i0; it += kThreads / 32) {
+        float mstar = -INFINITY;
+        for (int sp = lane; sp < S; sp += 32) mstar = fmaxf(mstar, wts[it * S + sp]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
+        float sum = 0.f;
+        if (mstar != -INFINITY)
+            for (int sp = lane; sp < S; sp += 32) sum += exp2f(wts[it * S + sp] - mstar);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        __syncwarp();
+        for (int sp = lane; sp < S; sp += 32)
+            wts[it * S + sp] = sum > 0.f ? exp2f(wts[it * S + sp] - mstar) / sum : 0.f;
+        if (lane == 0) lse_s[it] = sum > 0.f ? mstar + log2f(sum) : -INFINITY;
+    }
+    __syncthreads();
+    constexpr int C4 = D / 4;
+    for (int e = threadIdx.x; e < (i1 - i0) * C4; e += kThreads) {
+        const int it = e / C4, c4 = e % C4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int sp = 0; sp < S; ++sp) {
+            const float w = wts[it * S + sp];
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                                        part_o + slot_row(i0 + it, sp) * D) + c4);
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+        }
+        const int item = i0 + it;
+        const int u = item / R, rho = item % R;
+        const int ub = u / hkv, uh = u % hkv;
+        const size_t orow = ((size_t)ub * f + rho / g) * hq + (size_t)uh * g + rho % g;
+        reinterpret_cast<float4 *>(out + orow * D)[c4] = acc;
+        if (lse_out && c4 == 0) lse_out[orow] = lse_s[it] * 0.6931471805599453f;
+    }
 }
 
 template <int D>
@@ -460,11 +537,23 @@ cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *pa
     if (e != cudaSuccess) return e;
     const float scale_log2 = s.sm_scale * 1.4426950408889634f;
     dim3 grid(groups, splits, s.batch * s.hkv);
-    rectify_tc_kernel<D><<<grid, kThreads, smem, st>>>(
-        maps[0], maps[1], maps[2], maps[3], page_table, seq_len, f, (const uint16_t *)q_chunk,
-        s.hkv, s.g, s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out, lse,
-        err);
-    return cudaGetLastError();
+    // With several splits the CTAs meet at a grid barrier before merging, so
+    // they must be co-resident: cooperative launch (one CTA per SM; the split
+    // count keeps the grid within the SM count).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = splits > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, rectify_tc_kernel<D>, maps[0], maps[1], maps[2], maps[3],
+                              page_table, seq_len, f, (const uint16_t *)q_chunk, s.hkv, s.g,
+                              s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out,
+                              lse, err);
 }
 
 }  // namespace

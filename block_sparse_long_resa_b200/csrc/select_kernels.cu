@@ -15,11 +15,18 @@
 // digit.  In decode steps an extra warp of the first CTA of each sequence
 // appends the decode token (K/V write, descriptor fold) in the same launch.
 //
-// select_kernel is one 1024-thread CTA per (sequence, kv head): it finds the
-// histogram bin holding the k-th largest key (scanning only the touched bins,
-// clearing them for the next call), gathers that bin's keys, radix-selects
-// their low 16 bits, and compacts the blocks with key > T plus the
-// lowest-index blocks with key == T in ascending order (warp ballots).
+// select_kernel runs one thread-block cluster of eight CTAs per (sequence, kv
+// head), each CTA owning one eighth of the keys.  Every CTA finds the
+// histogram bin holding the k-th largest key (only the touched bins are
+// read; the first CTA clears them for the next call); one pass over its slice
+// counts the keys above that bin and gathers the bin's keys; the cluster's
+// candidates are exchanged through distributed shared memory and a radix
+// select of their low 16 bits gives the threshold T; per-CTA counts of keys
+// above / equal to T give each CTA its output offset, and a ballot pass
+// writes the blocks with key > T plus the lowest-index blocks with key == T
+// in ascending order.
+#include <cooperative_groups.h>
+
 #include "resa_common.cuh"
 
 namespace resa {
@@ -95,25 +102,18 @@ __global__ void __launch_bounds__(kScoreThreads)
         }
         fence_mbar_init();
     }
-    if (warp >= 1 && warp <= kScoreConsumers) {
-        // Group pooling: mean of the g query heads, fp32, head order, then / g.
-        for (int e = threadIdx.x - 32; e < HKV * D; e += 32 * kScoreConsumers) {
-            const int h = e / D, j = e % D;
-            const uint16_t *col = q + ((size_t)b * hq + (size_t)h * g) * D + j;
-            uint16_t v[kMaxGroup];
-#pragma unroll
-            for (int r = 0; r < kMaxGroup; ++r) v[r] = r < g ? col[(size_t)r * D] : (uint16_t)0;
-            float s = 0.f;
-#pragma unroll
-            for (int r = 0; r < kMaxGroup; ++r)
-                if (r < g) s += bf16_bits_to_f32(v[r]);
-            qbar_s[h][j] = s / (float)g;
-        }
-    }
     __syncthreads();
 
     if (warp == 0) {  // ------------------------------------------------ producer
-        pdl_wait();
+        static_assert(kScoreStages * kScoreGroup == 32, "one lane per page of the first stages");
+        // Page ids of the first kScoreStages groups (the page table is an
+        // input of the call): lane = group * kScoreGroup + slot.
+        int pg_first = -1;
+        {
+            const int p = p_begin + lane;
+            if (p < p_end) pg_first = page_table[(size_t)b * max_pages + p];
+        }
+        pdl_wait();  // descriptors and workspace may be written by the preceding kernels
         if (!seq_ok && x == 0 && lane == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
         for (int i = 0; i < n_groups; ++i) {
             const int s = i % kScoreStages;
@@ -124,12 +124,15 @@ __global__ void __launch_bounds__(kScoreThreads)
             const int p0 = p_begin + i * kScoreGroup;
             const int npg = min(kScoreGroup, p_end - p0);
             int pg = -1;
-            if (lane < npg) {
+            if (i < kScoreStages) {
+                pg = __shfl_sync(0xffffffffu, pg_first, (i * kScoreGroup + lane) & 31);
+                if (lane >= npg) pg = -1;
+            } else if (lane < npg) {
                 pg = page_table[(size_t)b * max_pages + p0 + lane];
-                if (pg < 0 || pg >= num_pages) {
-                    set_error(err, RESA_DEVERR_PAGE);
-                    pg = -1;
-                }
+            }
+            if (lane < npg && (pg < 0 || pg >= num_pages)) {
+                set_error(err, RESA_DEVERR_PAGE);
+                pg = -1;
             }
             const uint32_t all = (1u << npg) - 1u;  // npg <= kScoreGroup < 32
             const uint32_t vmask = __ballot_sync(0xffffffffu, lane < npg && pg >= 0);
@@ -157,6 +160,21 @@ __global__ void __launch_bounds__(kScoreThreads)
             }
         }
     } else if (warp <= kScoreConsumers) {  // ------------------------- consumers
+        // Group pooling: mean of the g query heads, fp32, head order, then / g
+        // (q is an input of the call, read while the first copies are in flight).
+        for (int e = threadIdx.x - 32; e < HKV * D; e += 32 * kScoreConsumers) {
+            const int h = e / D, j = e % D;
+            const uint16_t *col = q + ((size_t)b * hq + (size_t)h * g) * D + j;
+            uint16_t v[kMaxGroup];
+#pragma unroll
+            for (int r = 0; r < kMaxGroup; ++r) v[r] = r < g ? col[(size_t)r * D] : (uint16_t)0;
+            float s = 0.f;
+#pragma unroll
+            for (int r = 0; r < kMaxGroup; ++r)
+                if (r < g) s += bf16_bits_to_f32(v[r]);
+            qbar_s[h][j] = s / (float)g;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * kScoreConsumers) : "memory");
         pdl_wait();
         const int c = warp - 1;
         float qv[HKV][N];
@@ -279,14 +297,16 @@ __global__ void __launch_bounds__(kScoreThreads)
     }
 }
 
-constexpr int kSelectThreads = 1024;
-constexpr int kSelectWarps = kSelectThreads / 32;
-constexpr int kKeysInSmem = 32 * 1024;  // 128 KB of keys
-constexpr int kCandCap = 8 * 1024;      // keys of the boundary bin
+constexpr int kSelCluster = 8;    // CTAs per (sequence, kv head): one thread-block cluster
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelKeys = 4096;     // keys of its slice a CTA keeps in shared memory
+constexpr int kSelCandCap = 4096;  // boundary-bin keys gathered from the whole cluster
+constexpr int kSelLocalCand = 1024;
 
 // Exclusive scan of one value per thread over the CTA, in thread order.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_tot,
-                                                         uint32_t &total) {
+__device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t *warp_tot,
+                                                       uint32_t &total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t incl = v;
 #pragma unroll
@@ -296,7 +316,7 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
     }
     if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
-    const uint32_t wsum = warp_tot[lane];  // kSelectWarps == 32
+    const uint32_t wsum = lane < kSelWarps ? warp_tot[lane] : 0u;
     uint32_t wincl = wsum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -324,7 +344,7 @@ __device__ __forceinline__ void radix_select(KeyFn key, int n, int bits_left, ui
         const uint32_t nbm = (1u << width) - 1u;
         if (tid < 256) hist[tid] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += kSelectThreads) {
+        for (int i = tid; i < n; i += kSelThreads) {
             const uint32_t x = key(i);
             if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & nbm], 1u);
         }
@@ -366,24 +386,28 @@ __device__ __forceinline__ void radix_select(KeyFn key, int n, int bits_left, ui
     }
 }
 
-// grid (hkv, batch), block kSelectThreads,
-// dynamic smem = (key_cap + kCandCap) * 4 bytes, key_cap = min(max_pages, kKeysInSmem).
-__global__ void __launch_bounds__(kSelectThreads)
+// Grid (kSelCluster, hkv, batch), clusters of kSelCluster CTAs along x: one
+// cluster per (sequence, kv head); CTA rank r owns keys [r*C, (r+1)*C).
+__global__ void __launch_bounds__(kSelThreads)
     select_kernel(const float *__restrict__ scores, uint32_t *__restrict__ hist,
                   uint32_t *__restrict__ hist_range, const int32_t *__restrict__ seq_len,
                   const int32_t *__restrict__ topk, int max_topk, int32_t *__restrict__ block_idx,
-                  int32_t *__restrict__ block_cnt, int hkv, int max_pages, int key_cap,
-                  uint32_t *err) {
-    extern __shared__ uint32_t dsm[];
-    uint32_t *keys_s = dsm;          // [key_cap]
-    uint32_t *cand = dsm + key_cap;  // [kCandCap] low 16 bits of boundary-bin keys
+                  int32_t *__restrict__ block_cnt, int hkv, int max_pages, uint32_t *err) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    __shared__ uint32_t keys_s[kSelKeys];
+    __shared__ uint32_t lc_key[kSelLocalCand];  // this CTA's boundary-bin keys (low 16 bits)
+    __shared__ int32_t lc_idx[kSelLocalCand];   // and their block ids
+    __shared__ uint32_t all_c[kSelCandCap];     // the cluster's boundary-bin keys
     __shared__ uint32_t hist_s[256];
-    __shared__ uint32_t warp_tot[kSelectWarps], warp_gt[kSelectWarps], warp_eq[kSelectWarps];
+    __shared__ uint32_t warp_tot[kSelWarps], warp_gt[kSelWarps], warp_eq[kSelWarps];
     __shared__ uint32_t sh[4];
-    __shared__ uint32_t cand_n;
+    __shared__ uint32_t lc_n;                   // candidates of this CTA
+    __shared__ uint32_t cta_gt, cta_eq;         // keys > T / == T in this CTA's slice
 
     pdl_launch_next();
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int rank = (int)cluster.block_rank();
+    const int h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t unit = (size_t)b * hkv + h;
     int32_t *out = block_idx + unit * (max_topk + 1);
@@ -399,30 +423,27 @@ __global__ void __launch_bounds__(kSelectThreads)
         k = max_topk;
     }
     k = min(k, M);
+    const int C = (M + kSelCluster - 1) / kSelCluster;
+    const int c0 = min(M, rank * C), c1 = min(M, c0 + C);
     pdl_wait();
 
-    // Touched histogram bins [dmin, dmax]; reset the range for the next call.
+    // Boundary bin of the k-th largest key from the scorer's histogram
+    // (every CTA of the cluster computes the same; rank 0 clears it later).
     const uint32_t emin = hist_range[2 * unit], emax = hist_range[2 * unit + 1];
     const int dmin = (int)(kHistBins - emin), dmax = (int)emax - 1;
     const int nbins = dmax >= dmin ? dmax - dmin + 1 : 0;
     uint32_t *hb = hist + unit * kHistBins;
     if (tid == 0) {
-        cand_n = 0;
-        sh[0] = sh[1] = sh[2] = 0;
+        lc_n = 0;
+        sh[0] = sh[1] = 0;
     }
-    __syncthreads();
-    if (tid == 0) {
-        hist_range[2 * unit] = 0;
-        hist_range[2 * unit + 1] = 0;
-    }
-    // Bins in descending order, a contiguous chunk per thread.
-    const int chunk = (nbins + kSelectThreads - 1) / kSelectThreads;
+    const int chunk = (nbins + kSelThreads - 1) / kSelThreads;
     const int top = dmax - tid * chunk;
     const int lo = max(dmin, top - chunk + 1);
     uint32_t local = 0;
     for (int d = top; d >= lo; --d) local += __ldcg(&hb[d]);
     uint32_t total;
-    const uint32_t above_me = block_exclusive_scan(local, warp_tot, total);
+    const uint32_t above_me = cta_exclusive_scan(local, warp_tot, total);
     const bool trivial = !seq_ok || k == M || k == 0;
     if (!trivial && above_me < (uint32_t)k && (uint32_t)k <= above_me + local) {
         uint32_t cum = above_me;
@@ -437,128 +458,181 @@ __global__ void __launch_bounds__(kSelectThreads)
         }
     }
     __syncthreads();
-    for (int d = top; d >= lo; --d) hb[d] = 0;  // leave the histogram clear
-
-    if (tid == 0) {
-        if (!seq_ok) set_error(err, RESA_DEVERR_SEQ_LEN);
-        if (topk_err) set_error(err, RESA_DEVERR_TOPK);
-    }
-    if (!seq_ok) {
-        if (tid == 0) *cnt = 0;
-        return;
-    }
-    if (k == M) {  // every complete block (also k = M = 0)
-        for (int i = tid; i < M; i += kSelectThreads) out[i] = i;
-        if (tid == 0) {
-            out[M] = M;
-            *cnt = M + 1;
-        }
-        return;
-    }
-    if (k == 0) {
-        if (tid == 0) {
-            out[0] = M;
-            *cnt = 1;
-        }
-        return;
-    }
-    const bool hist_ok = total == (uint32_t)M;  // every complete block was scored
-    if (!hist_ok && tid == 0) set_error(err, RESA_DEVERR_PAGE);
+    const bool hist_ok = total == (uint32_t)M;
     const uint32_t d1 = sh[0];
     uint32_t remaining = (uint32_t)k - sh[1];
 
-    // Keys into shared memory; gather the boundary bin's low halves.
+    // One pass over this CTA's slice: keys into shared memory, per-warp count
+    // of keys above the boundary bin, the bin's keys as candidates.
     const float *src = scores + unit * max_pages;
-    const bool in_smem = M <= key_cap;
-    constexpr int U = 8;
-    for (int i0 = warp * 32 * U; i0 < M; i0 += kSelectThreads * U) {
-        uint32_t kv[U];
+    const int n_mine = c1 - c0;
+    const bool in_smem = n_mine <= kSelKeys;
+    const int R = (n_mine + kSelWarps - 1) / kSelWarps;
+    const int w0 = c0 + warp * R, w1 = min(c1, w0 + R);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t above_w = 0;
+    if (!trivial) {
+        constexpr int U = 4;
+        for (int base = w0; base < w1; base += 32 * U) {
+            uint32_t kv[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int i = i0 + u * 32 + lane;
-            kv[u] = i < M ? order_key(src[i]) : 0u;
+            for (int u = 0; u < U; ++u) {
+                const int i = base + u * 32 + lane;
+                kv[u] = i < w1 ? order_key(src[i]) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = base + u * 32 + lane;
+                const bool valid = i < w1;
+                if (valid && in_smem) keys_s[i - c0] = kv[u];
+                const uint32_t dg = kv[u] >> 16;
+                above_w += __popc(__ballot_sync(0xffffffffu, valid && dg > d1));
+                const bool is_c = valid && dg == d1;
+                const uint32_t ball = __ballot_sync(0xffffffffu, is_c);
+                if (ball) {
+                    uint32_t cb = 0;
+                    if (lane == 0) cb = atomicAdd(&lc_n, (uint32_t)__popc(ball));
+                    cb = __shfl_sync(0xffffffffu, cb, 0);
+                    const uint32_t r = cb + __popc(ball & lt_mask);
+                    if (is_c && r < (uint32_t)kSelLocalCand) {
+                        lc_key[r] = kv[u] & 0xffffu;
+                        lc_idx[r] = i;
+                    }
+                }
+            }
         }
+    }
+    if (lane == 0) {
+        warp_gt[warp] = above_w;
+        warp_eq[warp] = 0;
+    }
+    cluster.sync();  // #1: every CTA's candidates are ready; the histogram is read
+
+    if (rank == 0) {  // leave the histogram clear for the next call
+        for (int d = dmin + tid; d <= dmax; d += kSelThreads) hb[d] = 0;
+        if (tid == 0) {
+            hist_range[2 * unit] = 0;
+            hist_range[2 * unit + 1] = 0;
+            if (!seq_ok) set_error(err, RESA_DEVERR_SEQ_LEN);
+            if (topk_err) set_error(err, RESA_DEVERR_TOPK);
+        }
+    }
+    uint32_t T = 0, need_eq = 0;
+    bool fallback = trivial ? false : !hist_ok;
+    if (!trivial) {
+        // Gather the cluster's candidates (distributed shared memory).
+        uint32_t offs[kSelCluster], ntot = 0;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int i = i0 + u * 32 + lane;
-            const bool valid = i < M;
-            if (valid && in_smem) keys_s[i] = kv[u];
-            const bool is_c = valid && (kv[u] >> 16) == d1;
-            const uint32_t ball = __ballot_sync(0xffffffffu, is_c);
-            if (ball) {
-                uint32_t base = 0;
-                if (lane == 0) base = atomicAdd(&cand_n, (uint32_t)__popc(ball));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                const uint32_t r = base + __popc(ball & ((1u << lane) - 1u));
-                if (is_c && r < (uint32_t)kCandCap) cand[r] = kv[u] & 0xffffu;
+        for (int r = 0; r < kSelCluster; ++r) {
+            const uint32_t n = *cluster.map_shared_rank(&lc_n, r);
+            offs[r] = ntot;
+            ntot += n;
+            if (n > (uint32_t)kSelLocalCand) fallback = true;
+        }
+        if (ntot > (uint32_t)kSelCandCap) fallback = true;
+        if (!fallback) {
+#pragma unroll
+            for (int r = 0; r < kSelCluster; ++r) {
+                const uint32_t *peer = cluster.map_shared_rank(lc_key, r);
+                const uint32_t n = (r + 1 < kSelCluster ? offs[r + 1] : ntot) - offs[r];
+                for (uint32_t i = tid; i < n; i += kSelThreads) all_c[offs[r] + i] = peer[i];
+            }
+            __syncthreads();
+            uint32_t cp = 0, cm = 0;
+            radix_select([&](int i) { return all_c[i]; }, (int)ntot, 16, cp, cm, remaining, hist_s,
+                         sh);
+            T = (d1 << 16) | cp;
+            need_eq = remaining;
+            // this CTA's candidates above / at T, per owning warp range
+            const uint32_t myn = lc_n;
+            for (uint32_t c = tid; c < myn; c += kSelThreads) {
+                const uint32_t key = (d1 << 16) | lc_key[c];
+                const int w = (lc_idx[c] - c0) / R;
+                if (key > T) atomicAdd(&warp_gt[w], 1u);
+                else if (key == T) atomicAdd(&warp_eq[w], 1u);
+            }
+        } else {
+            // Degenerate score distribution: radix over every key of the sequence.
+            uint32_t prefix = 0, pmask = 0;
+            remaining = (uint32_t)k;
+            radix_select([&](int i) { return order_key(src[i]); }, M, 32, prefix, pmask,
+                         remaining, hist_s, sh);
+            T = prefix;
+            need_eq = remaining;
+            uint32_t gt = 0, eq = 0;
+            for (int i = w0 + lane; i < w1; i += 32) {
+                const uint32_t x = order_key(src[i]);
+                gt += x > T;
+                eq += x == T;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                gt += __shfl_xor_sync(0xffffffffu, gt, o);
+                eq += __shfl_xor_sync(0xffffffffu, eq, o);
+            }
+            if (lane == 0) {
+                warp_gt[warp] = gt;
+                warp_eq[warp] = eq;
             }
         }
     }
     __syncthreads();
-    auto key_at = [&](int i) -> uint32_t { return in_smem ? keys_s[i] : order_key(src[i]); };
-    uint32_t prefix, pmask;
-    const int nc = (int)cand_n;
-    if (hist_ok && nc <= kCandCap) {
-        uint32_t cp = 0, cm = 0;
-        radix_select([&](int i) { return cand[i]; }, nc, 16, cp, cm, remaining, hist_s, sh);
-        prefix = (d1 << 16) | cp;
-    } else if (hist_ok) {
-        prefix = d1 << 16;
-        pmask = 0xffff0000u;
-        radix_select(key_at, M, 16, prefix, pmask, remaining, hist_s, sh);
-    } else {  // no usable histogram: full radix select over the keys
-        prefix = 0;
-        pmask = 0;
-        remaining = (uint32_t)k;
-        radix_select(key_at, M, 32, prefix, pmask, remaining, hist_s, sh);
-    }
-    const uint32_t T = prefix;
-    const uint32_t need_eq = remaining;
-
-    // Ballot compaction in ascending block order: warp w owns [w*R, (w+1)*R).
-    const int R = (M + kSelectWarps - 1) / kSelectWarps;
-    const int w0 = warp * R, w1 = min(M, w0 + R);
-    uint32_t gt = 0, eq = 0;
-    for (int i = w0 + lane; i < w1; i += 32) {
-        const uint32_t x = key_at(i);
-        gt += x > T;
-        eq += x == T;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        gt += __shfl_xor_sync(0xffffffffu, gt, o);
-        eq += __shfl_xor_sync(0xffffffffu, eq, o);
-    }
-    if (lane == 0) {
-        warp_gt[warp] = gt;
-        warp_eq[warp] = eq;
-    }
-    __syncthreads();
-    uint32_t gt_before = 0, eq_before = 0;
-    for (int w = 0; w < warp; ++w) {
-        gt_before += warp_gt[w];
-        eq_before += warp_eq[w];
-    }
-    uint32_t pos = gt_before + min(eq_before, need_eq);
-    uint32_t eq_seen = eq_before;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int base = w0; base < w1; base += 32) {
-        const int i = base + lane;
-        const uint32_t xk = i < w1 ? key_at(i) : 0u;
-        const bool is_gt = i < w1 && xk > T;
-        const bool is_eq = i < w1 && xk == T;
-        const uint32_t eq_ball = __ballot_sync(0xffffffffu, is_eq);
-        const uint32_t eq_rank = eq_seen + __popc(eq_ball & lt_mask);
-        const bool take = is_gt || (is_eq && eq_rank < need_eq);
-        const uint32_t take_ball = __ballot_sync(0xffffffffu, take);
-        if (take) out[pos + __popc(take_ball & lt_mask)] = i;
-        pos += __popc(take_ball);
-        eq_seen += __popc(eq_ball);
-    }
     if (tid == 0) {
-        out[k] = M;
-        *cnt = k + 1;
+        uint32_t g2 = 0, e2 = 0;
+        for (int w = 0; w < kSelWarps; ++w) {
+            g2 += warp_gt[w];
+            e2 += warp_eq[w];
+        }
+        cta_gt = g2;
+        cta_eq = e2;
     }
+    cluster.sync();  // #2: per-CTA counts visible to the cluster
+
+    if (trivial) {
+        if (seq_ok) {
+            if (k == M)
+                for (int i = c0 + tid; i < c1; i += kSelThreads) out[i] = i;
+            if (rank == 0 && tid == 0) {
+                out[k] = M;
+                *cnt = k + 1;
+            }
+        } else if (rank == 0 && tid == 0) {
+            *cnt = 0;
+        }
+    } else {
+        uint32_t gt_before = 0, eq_before = 0;
+        for (int r = 0; r < rank; ++r) {
+            gt_before += *cluster.map_shared_rank(&cta_gt, r);
+            eq_before += *cluster.map_shared_rank(&cta_eq, r);
+        }
+        for (int w = 0; w < warp; ++w) {
+            gt_before += warp_gt[w];
+            eq_before += warp_eq[w];
+        }
+        auto key_at = [&](int i) -> uint32_t {
+            return (in_smem && !fallback) ? keys_s[i - c0] : order_key(src[i]);
+        };
+        uint32_t pos = gt_before + min(eq_before, need_eq);
+        uint32_t eq_seen = eq_before;
+        for (int base = w0; base < w1; base += 32) {
+            const int i = base + lane;
+            const uint32_t xk = i < w1 ? key_at(i) : 0u;
+            const bool is_gt = i < w1 && xk > T;
+            const bool is_eq = i < w1 && xk == T;
+            const uint32_t eq_ball = __ballot_sync(0xffffffffu, is_eq);
+            const uint32_t eq_rank = eq_seen + __popc(eq_ball & lt_mask);
+            const bool take = is_gt || (is_eq && eq_rank < need_eq);
+            const uint32_t take_ball = __ballot_sync(0xffffffffu, take);
+            if (take) out[pos + __popc(take_ball & lt_mask)] = i;
+            pos += __popc(take_ball);
+            eq_seen += __popc(eq_ball);
+        }
+        if (rank == 0 && tid == 0) {
+            out[k] = M;
+            *cnt = k + 1;
+        }
+    }
+    cluster.sync();  // #3: no CTA leaves while a peer may still read its shared memory
 }
 
 template <int D>
@@ -612,15 +686,22 @@ cudaError_t launch_select(const Shape &s, const float *scores, uint32_t *hist,
                           uint32_t *hist_range, const int32_t *seq_len, const int32_t *topk,
                           int max_topk, int32_t *block_idx, int32_t *block_cnt, uint32_t *err,
                           cudaStream_t st) {
-    const int cap = s.max_pages < kKeysInSmem ? s.max_pages : kKeysInSmem;
-    const size_t smem = (size_t)(cap + kCandCap) * 4;
-    static std::atomic<int> done[64];
-    cudaError_t e = ensure_smem(select_kernel, (kKeysInSmem + kCandCap) * 4, done);
-    if (e != cudaSuccess) return e;
-    dim3 grid(s.hkv, s.batch);
-    return launch_pdl(select_kernel, grid, dim3(kSelectThreads), smem, st, scores, hist,
-                      hist_range, seq_len, topk, max_topk, block_idx, block_cnt, s.hkv,
-                      s.max_pages, cap, err);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kSelCluster, s.hkv, s.batch);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kSelCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, select_kernel, scores, hist, hist_range, seq_len, topk,
+                              max_topk, block_idx, block_cnt, s.hkv, s.max_pages, err);
 }
 
 }  // namespace resa
