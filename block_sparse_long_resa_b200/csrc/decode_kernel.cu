@@ -17,9 +17,12 @@
 // registers with movmatrix and enters the P.V MMA as bf16 hi + lo parts.
 //
 // The CTA merges its warps, then writes the final output (one split) or a
-// partial (o, log2-sum-exp) and draws an atomic ticket; the CTA drawing the
-// last ticket of its (sequence, kv head) merges the splits with vectorised,
-// batched loads and resets the ticket.  No CTA waits on another.
+// partial (o, log2-sum-exp).  When the grid fits one wave it is launched
+// cooperatively and, after a bounded grid barrier, every CTA merges a slice
+// of the outputs.  Otherwise each CTA draws an atomic ticket and the CTA
+// drawing the last ticket of its (sequence, kv head) pulls every split's
+// partial into shared memory with bulk copies, merges them and resets the
+// ticket.
 #include "attn_common.cuh"
 
 namespace resa {
@@ -35,8 +38,8 @@ struct DecodeSmem {
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
     static constexpr int kMergeBytes = kWarps * kMaxGroup * (D + 3) * 4;
-    // split merge: weights [S][16] floats + [threads / (D/4)][16][D/4] float4 partial sums
-    static constexpr int kSplitMergeBytes = (kThreads / (D / 4)) * kMaxGroup * D * 4;
+    static_assert(kRingBytes >= kMaxDecodeSplits * kMaxGroup * 4 + kMaxGroup * D * 4,
+                  "split merge: the weights of every split and one partial tile fit the ring");
     static constexpr int kBytes = (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes) + 1024;
 };
 
@@ -141,6 +144,75 @@ __device__ __forceinline__ void attend_block_swapped(WarpState<D, NT> &st,
     }
 }
 
+// Split merge spread over the whole (co-resident) grid.  Work item = (unit,
+// row, 32 output channels); CTA c takes items c, c + gridsize, ...  Every
+// warp forms the row's log-sum-exp over the S splits in one pass (online max
+// and sum), then takes splits w, w + 8, ... of the item with all its loads in
+// flight together; the eight warps' sums are added through shared memory.
+template <int D>
+__device__ __forceinline__ void merge_splits_spread(const float *__restrict__ part_o,
+                                                    const float *__restrict__ part_lse, int S,
+                                                    int hkv, int g, float *__restrict__ out,
+                                                    float *__restrict__ lse_out, float *red) {
+    constexpr int C32 = D / 32;
+    constexpr int kBatch = 8;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nctas = gridDim.x * gridDim.y * gridDim.z;
+    const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    const int units = gridDim.y * gridDim.z;
+    const int n_items = units * g * C32;
+    const float kLn2 = 0.6931471805599453f;
+    for (int item = cta; item < n_items; item += nctas) {
+        const int u = item / (g * C32), rem = item % (g * C32);
+        const int r = rem / C32, cc = rem % C32;
+        const float *ul = part_lse + (size_t)u * S * kMaxGroup + r;
+        const float *uo = part_o + ((size_t)u * S * kMaxGroup + r) * D + cc * 32 + lane;
+        float m = -INFINITY, l = 0.f;
+        for (int sp = lane; sp < S; sp += 32) {
+            const float x = __ldcg(ul + (size_t)sp * kMaxGroup);
+            if (x == -INFINITY) continue;
+            const float mn = fmaxf(m, x);
+            l = l * exp2f(m - mn) + exp2f(x - mn);
+            m = mn;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+            const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+            const float mn = fmaxf(m, mo);
+            if (mn != -INFINITY) {
+                l = l * exp2f(m - mn) + lo * exp2f(mo - mn);
+                m = mn;
+            }
+        }
+        float acc = 0.f;
+        for (int s0 = warp; s0 < S; s0 += kWarps * kBatch) {
+            float v[kBatch], x[kBatch];
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const int sp = s0 + k * kWarps;
+                v[k] = sp < S ? __ldcg(uo + (size_t)sp * kMaxGroup * D) : 0.f;
+                x[k] = sp < S ? __ldcg(ul + (size_t)sp * kMaxGroup) : -INFINITY;
+            }
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k)
+                if (x[k] != -INFINITY) acc += exp2f(x[k] - m) * v[k];
+        }
+        red[warp * 32 + lane] = acc;
+        __syncthreads();
+        if (warp == 0) {
+            float o = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) o += red[w * 32 + lane];
+            const size_t orow = (size_t)(u / hkv) * hkv * g + (size_t)(u % hkv) * g + r;
+            out[orow * D + cc * 32 + lane] = l > 0.f ? o / l : 0.f;
+            if (lse_out && cc == 0 && lane == 0)
+                lse_out[orow] = (l > 0.f ? m + log2f(l) : -INFINITY) * kLn2;
+        }
+        __syncthreads();
+    }
+}
+
 template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -151,12 +223,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const int32_t *__restrict__ block_cnt, int max_topk, int hkv, int g,
                          int max_pages, int num_pages, float scale_log2, float *__restrict__ part_o,
                          float *__restrict__ part_lse, uint32_t *__restrict__ tickets,
-                         float *__restrict__ out, float *__restrict__ lse_out, uint32_t *err) {
+                         uint32_t *__restrict__ grid_bar, float *__restrict__ out,
+                         float *__restrict__ lse_out, uint32_t *err) {
     using SM = DecodeSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     __shared__ uint64_t bars[kWarps][kStages];
+    __shared__ uint64_t merge_bar;
     __shared__ int2 meta[kMaxBlocksPerSplit];  // (page, valid tokens) of the slice's blocks
     __shared__ uint32_t sh_last;
     __shared__ float sh_lse[kMaxGroup];
@@ -172,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int w = 0; w < kWarps; ++w)
             for (int s = 0; s < kStages; ++s) mbar_init(&bars[w][s], 1);
+        mbar_init(&merge_bar, 1);
         fence_mbar_init();
     }
     // Q^T B fragments: head nt*8 + lane/4 (zero beyond g), channels 2*(lane%4)+{0,1} (+8).
@@ -329,9 +404,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (S == 1) return;
 
-    // Split combine by the CTA that draws the last ticket.
     __threadfence();
     __syncthreads();
+    if (grid_bar != nullptr) {
+        // Cooperative launch (the grid is one wave): bounded grid barrier, then
+        // every CTA merges its share of the outputs.
+        if (threadIdx.x == 0)
+            sh_last = grid_barrier_bounded(grid_bar, gridDim.x * gridDim.y * gridDim.z) ? 1u : 0u;
+        __syncthreads();
+        if (!sh_last) {
+            if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+            return;
+        }
+        __threadfence();
+        merge_splits_spread<D>(part_o, part_lse, S, hkv, g, out, lse_out,
+                               reinterpret_cast<float *>(smem));
+        return;
+    }
+    // Otherwise the CTA that draws the last ticket of the (sequence, head) merges.
     if (threadIdx.x == 0) {
         const uint32_t ticket = atomicAdd(&tickets[unit], 1u);
         sh_last = ticket == (uint32_t)(S - 1);
@@ -339,9 +429,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (!sh_last) return;
     __threadfence();
+    // The other CTAs' partial tiles (rows 0..g-1 of each split, contiguous)
+    // come in through bulk copies into the drained ring, every split's copy in
+    // flight at once; splits that do not fit are taken in further chunks.
     float *wts = reinterpret_cast<float *>(smem);  // [S][16] merge weights
+    const uint32_t wts_bytes = (uint32_t)((S * kMaxGroup * 4 + 127) / 128 * 128);
+    uint8_t *tiles = smem + wts_bytes;
+    const uint32_t tile_bytes = (uint32_t)(g * D * 4);
+    const int chunk = min(S, (int)((SM::kRingBytes - wts_bytes) / tile_bytes));
+    const int nchunks = (S + chunk - 1) / chunk;
     const float *ul = part_lse + unit * S * kMaxGroup;
     const float *uo = part_o + unit * S * kMaxGroup * D;
+    auto issue_chunk = [&](int ci) {  // warp 0
+        const int s0 = ci * chunk, s1 = min(S, s0 + chunk);
+        fence_proxy_async_global();  // generic-proxy partials -> async-proxy reads
+        fence_proxy_async_smem();    // earlier generic use of the ring -> async writes
+        if (lane == 0) mbar_arrive_expect_tx(&merge_bar, (uint32_t)(s1 - s0) * tile_bytes);
+        __syncwarp();
+        for (int sp = s0 + lane; sp < s1; sp += 32)
+            bulk_load(tiles + (size_t)(sp - s0) * tile_bytes, uo + (size_t)sp * kMaxGroup * D,
+                      tile_bytes, &merge_bar);
+    };
+    if (warp == 0) issue_chunk(0);
     for (int i = threadIdx.x; i < S * g; i += kThreads) {
         const int s = i / g, r = i % g;
         wts[s * kMaxGroup + r] = __ldcg(&ul[s * kMaxGroup + r]);
@@ -363,72 +472,117 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) sh_lse[r] = sum > 0.f ? mstar + log2f(sum) : -INFINITY;
     }
     __syncthreads();
-    // (The ring region holds wts then red: S*64 + kSplitMergeBytes <= ring bytes
-    // for every split count the workspace allows.)
-    // Thread (split group sg, float4 column c4) accumulates every row over
-    // splits sg, sg + 8, ...: all its loads are independent and in flight
-    // together; the eight split groups are then summed through shared memory.
+    // Thread item = (row, float4 column); two accumulators (even / odd split)
+    // keep two independent FMA chains per item.
     constexpr int C4 = D / 4;
-    constexpr int SG = kThreads / C4;  // split groups
-    float4 *red = reinterpret_cast<float4 *>(wts + S * kMaxGroup);  // [SG][16][C4]
-    {
-        const int c4 = threadIdx.x % C4, sg = threadIdx.x / C4;
-        float4 acc[kMaxGroup];
+    constexpr int kItems = (kMaxGroup * C4 + kThreads - 1) / kThreads;
+    const int items = g * C4;
+    float4 acc[kItems][2];
 #pragma unroll
-        for (int r = 0; r < kMaxGroup; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = sg; sp < S; sp += SG) {
-            const float4 *src = reinterpret_cast<const float4 *>(uo + (size_t)sp * kMaxGroup * D) + c4;
+    for (int k = 0; k < kItems; ++k)
+        acc[k][0] = acc[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    bool merged = true;
+    for (int ci = 0; ci < nchunks; ++ci) {
+        if (!mbar_wait_bounded(&merge_bar, ci & 1)) {
+            merged = false;
+            break;
+        }
+        const int s0 = ci * chunk, s1 = min(S, s0 + chunk);
+        const float4 *tf = reinterpret_cast<const float4 *>(tiles);
 #pragma unroll
-            for (int r = 0; r < kMaxGroup; ++r) {
-                if (r < g) {
+        for (int k = 0; k < kItems; ++k) {
+            const int item = threadIdx.x + k * kThreads;
+            if (item < items) {
+                const int r = item / C4;
+#pragma unroll 4
+                for (int sp = s0; sp < s1; ++sp) {
                     const float w = wts[sp * kMaxGroup + r];
-                    const float4 v = __ldcg(src + (size_t)r * C4);
-                    acc[r].x += w * v.x;
-                    acc[r].y += w * v.y;
-                    acc[r].z += w * v.z;
-                    acc[r].w += w * v.w;
+                    const float4 v = tf[(size_t)(sp - s0) * items + item];
+                    float4 &a = acc[k][sp & 1];
+                    a.x += w * v.x;
+                    a.y += w * v.y;
+                    a.z += w * v.z;
+                    a.w += w * v.w;
                 }
             }
         }
-#pragma unroll
-        for (int r = 0; r < kMaxGroup; ++r)
-            if (r < g) red[((size_t)sg * kMaxGroup + r) * C4 + c4] = acc[r];
-    }
-    __syncthreads();
-    for (int item = threadIdx.x; item < g * C4; item += kThreads) {
-        const int r = item / C4, c4 = item % C4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int sg = 0; sg < SG; ++sg) {
-            const float4 v = red[((size_t)sg * kMaxGroup + r) * C4 + c4];
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+        if (ci + 1 < nchunks) {
+            __syncthreads();  // every thread is done with this chunk's tiles
+            if (warp == 0) issue_chunk(ci + 1);
         }
-        const size_t orow = (size_t)b * hq + (size_t)h * g + r;
-        reinterpret_cast<float4 *>(out + orow * D)[c4] = acc;
-        if (lse_out && c4 == 0) lse_out[orow] = sh_lse[r] * kLn2;
+    }
+    if (!merged) {
+        if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+        mbar_wait_bounded(&merge_bar, 0);  // let copies in flight land before exit
+        mbar_wait_bounded(&merge_bar, 1);
+    } else {
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+            const int item = threadIdx.x + k * kThreads;
+            if (item < items) {
+                const int r = item / C4, c4 = item % C4;
+                const float4 a0 = acc[k][0], a1 = acc[k][1];
+                const size_t orow = (size_t)b * hq + (size_t)h * g + r;
+                reinterpret_cast<float4 *>(out + orow * D)[c4] =
+                    make_float4(a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w);
+                if (lse_out && c4 == 0) lse_out[orow] = sh_lse[r] * kLn2;
+            }
+        }
     }
     if (threadIdx.x == 0) tickets[unit] = 0;
+}
+
+// CTAs of one wave the device holds for this kernel (cached per device).
+template <int D, int NT>
+int wave_capacity(int smem) {
+    static std::atomic<int> cap[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    int c = cap[dev].load();
+    if (c == 0) {
+        int per_sm = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_decode_kernel<D, NT>,
+                                                          kThreads, smem) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return 0;
+        c = per_sm * sms;
+        cap[dev].store(c);
+    }
+    return c;
 }
 
 template <int D, int NT>
 cudaError_t launch_dn(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
                       const int32_t *page_table, const int32_t *seq_len, const void *q,
                       const int32_t *block_idx, const int32_t *block_cnt, int max_topk, int splits,
-                      float *part_o, float *part_lse, uint32_t *tickets, float *out, float *lse,
-                      uint32_t *err, cudaStream_t st) {
+                      float *part_o, float *part_lse, uint32_t *tickets, uint32_t *grid_bar,
+                      float *out, float *lse, uint32_t *err, cudaStream_t st) {
     constexpr int smem = DecodeSmem<D>::kBytes;
     static std::atomic<int> done[64];
     cudaError_t e = ensure_smem(sparse_decode_kernel<D, NT>, smem, done);
     if (e != cudaSuccess) return e;
     const float scale_log2 = s.sm_scale * 1.4426950408889634f;
     dim3 grid(splits, s.hkv, s.batch);
-    return launch_pdl(sparse_decode_kernel<D, NT>, grid, dim3(kThreads), smem, st, kmap, vmap,
-                      page_table, seq_len, (const uint16_t *)q, block_idx, block_cnt, max_topk,
-                      s.hkv, s.g, s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets,
-                      out, lse, err);
+    const long long ctas = (long long)splits * s.hkv * s.batch;
+    // Split merge across the grid when it fits one wave (cooperative launch);
+    // otherwise by the last CTA of each (sequence, head).
+    const bool spread = grid_bar != nullptr && splits > 1 && ctas <= wave_capacity<D, NT>(smem);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = spread ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, sparse_decode_kernel<D, NT>, kmap, vmap, page_table, seq_len,
+                              (const uint16_t *)q, block_idx, block_cnt, max_topk, s.hkv, s.g,
+                              s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets,
+                              spread ? grid_bar : (uint32_t *)nullptr, out, lse, err);
 }
 
 }  // namespace
@@ -437,10 +591,11 @@ cudaError_t launch_sparse_decode(const Shape &s, const CUtensorMap &kmap, const 
                                  const int32_t *page_table, const int32_t *seq_len, const void *q,
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
-                                 float *out, float *lse, uint32_t *err, cudaStream_t st) {
+                                 uint32_t *grid_bar, float *out, float *lse, uint32_t *err,
+                                 cudaStream_t st) {
 #define RESA_DECODE_ARGS                                                                     \
     s, kmap, vmap, page_table, seq_len, q, block_idx, block_cnt, max_topk, splits, part_o, \
-        part_lse, tickets, out, lse, err, st
+        part_lse, tickets, grid_bar, out, lse, err, st
     if (s.d == 128)
         return s.g <= 8 ? launch_dn<128, 1>(RESA_DECODE_ARGS) : launch_dn<128, 2>(RESA_DECODE_ARGS);
     if (s.d == 64)

@@ -19,7 +19,7 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t(8) << 20;  // 8 MiB per device
 constexpr int kScratchMaxUnits = 4096;             // batch * Hkv
-constexpr size_t kScratchHeader = 256;             // error word
+constexpr size_t kScratchHeader = 256;  // error word; grid barrier at kDecBarrierOffset
 
 // Shared by every call on a device; it keeps the previous call's contents.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
@@ -142,7 +142,8 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     s.num_pages = cache->num_pages;
     const cudaError_t e = launch_sparse_decode(
         s, kmap, vmap, cache->page_table, cache->seq_len, q, block_idx, block_cnt, max_topk,
-        splits, part_o, part_lse, tickets, out, lse_opt, dev_error_opt ? dev_error_opt : err,
-        stream);
+        splits, part_o, part_lse, tickets,
+        reinterpret_cast<uint32_t *>(scratch + kDecBarrierOffset), out, lse_opt,
+        dev_error_opt ? dev_error_opt : err, stream);
     return e == cudaSuccess ? RESA_OK : RESA_ERR_CUDA;
 }

@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_after_sync();
             if (ok) issue_qk(0);
             for (int i = 0; i < ntiles && ok; ++i) {
-                const int s = i % kStages, buf = i & 1;
+                const int s = i % kStages;
                 if (i + 1 < ntiles) {
                     ok = mbar_wait_bounded(&kv_full[(i + 1) % kStages], ((i + 1) / kStages) & 1);
                     tc::fence_after_sync();
@@ -443,28 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     __shared__ uint32_t sh_ok;
     const uint32_t nctas = gridDim.x * gridDim.y * gridDim.z;
-    if (threadIdx.x == 0) {
-        volatile uint32_t *gen_p = tickets + 1;
-        const uint32_t gen = *gen_p;
-        __threadfence();
-        const uint32_t ticket = atomicAdd(&tickets[0], 1u);
-        uint32_t ok = 1;
-        if (ticket == nctas - 1) {
-            tickets[0] = 0;
-            __threadfence();
-            atomicAdd(&tickets[1], 1u);
-        } else {
-            uint32_t polls = 0;
-            while (*gen_p == gen) {
-                if (++polls > (1u << 24)) {
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(64);
-            }
-        }
-        sh_ok = ok;
-    }
+    if (threadIdx.x == 0) sh_ok = grid_barrier_bounded(tickets, nctas) ? 1u : 0u;
     __syncthreads();
     if (!sh_ok) {
         if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);

@@ -151,10 +151,11 @@ resa_status_t decode_impl(const Shape &s, const resa_cache_t *c, const WsLayout 
         return RESA_ERR_CUDA;
     const int splits = decode_splits_for(s.batch * s.hkv, max_topk + 1);
     if (splits > w.dec_splits) return RESA_ERR_RANGE;  // max_topk far above max_pages
+    if (splits > kMaxDecodeSplits) return RESA_ERR_RANGE;
     return cuda_status(launch_sparse_decode(
         s, kmap, vmap, c->page_table, c->seq_len, q, idx, cnt, max_topk, splits,
-        at<float>(ws, w.dec_o), at<float>(ws, w.dec_lse), at<uint32_t>(ws, w.dec_ticket), out, lse,
-        at<uint32_t>(ws, w.err), st));
+        at<float>(ws, w.dec_o), at<float>(ws, w.dec_lse), at<uint32_t>(ws, w.dec_ticket),
+        at<uint32_t>(ws, w.err + kDecBarrierOffset), out, lse, at<uint32_t>(ws, w.err), st));
 }
 
 }  // namespace

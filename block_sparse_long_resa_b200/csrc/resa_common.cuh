@@ -25,9 +25,13 @@ constexpr int kMinBlocksPerSplit = 16;   // two per warp at least
 
 // Decode splits per (sequence, kv head): about one CTA per SM over all units,
 // at least kMinBlocksPerSplit blocks each, at most kMaxBlocksPerSplit.
+// Splits of one (sequence, kv head) the decode merge takes (its weights sit in
+// shared memory next to the partial tiles): max_topk + 1 <= 1024 * 512 blocks.
+constexpr int kMaxDecodeSplits = 1024;
 inline int decode_splits_for(int units, int max_blocks) {
     const int need = (max_blocks + kMaxBlocksPerSplit - 1) / kMaxBlocksPerSplit;
-    const int want = (kNumSms + units - 1) / units;
+    // as many splits as keep the grid within one wave of CTAs (one per SM)
+    const int want = units < kNumSms ? kNumSms / units : 1;
     const int work = (max_blocks + kMinBlocksPerSplit - 1) / kMinBlocksPerSplit;
     int s = want < work ? want : work;
     s = s > need ? s : need;
@@ -59,6 +63,10 @@ inline int rect_splits_for(int batch, int hkv, int groups) {
 // rectification partials come last.
 // ---------------------------------------------------------------------------
 constexpr int kMaxRowTiles = 64;  // rectification row groups per (sequence, kv head)
+
+// Byte offset, inside the 256-byte error header of the workspace, of the
+// decode kernel's grid barrier (arrival count, generation).
+constexpr size_t kDecBarrierOffset = 32;
 
 struct WsLayout {
     size_t err;          // uint32 error word
@@ -95,7 +103,7 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     w.row_tiles = chunk > 0 ? rect_row_groups(chunk, g) : 0;
     w.rect_splits = chunk > 0 ? rect_splits_for(batch, hkv, w.row_tiles) : 0;
     size_t units = (size_t)batch * hkv;
-    w.err = take(256);
+    w.err = take(256);  // error word at 0, decode grid barrier at kDecBarrierOffset
     w.dec_ticket = take(units * 4);
     w.rect_ticket = take(units * kMaxRowTiles * 4);
     w.hist = take(units * 65536 * 4);
@@ -117,6 +125,28 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
     if (err) atomicOr(err, bit);
+}
+
+// Bounded grid barrier of a cooperatively launched (co-resident) grid; thread
+// 0 of every CTA calls it after a __threadfence and a __syncthreads.  bar[0]
+// counts arrivals, bar[1] is the generation.  False when the wait gave up
+// (the count is then left non-zero: the workspace must be re-initialised).
+__device__ __forceinline__ bool grid_barrier_bounded(uint32_t *bar, uint32_t nctas) {
+    volatile uint32_t *gen_p = bar + 1;
+    const uint32_t gen = *gen_p;
+    __threadfence();
+    const uint32_t ticket = atomicAdd(&bar[0], 1u);
+    if (ticket == nctas - 1) {
+        bar[0] = 0;
+        __threadfence();
+        atomicAdd(&bar[1], 1u);
+        return true;
+    }
+    for (uint32_t polls = 0; *gen_p == gen;) {
+        if (++polls > (1u << 24)) return false;
+        __nanosleep(32);
+    }
+    return true;
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t x) {
@@ -174,6 +204,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // TMA: 3-D tiled bulk tensor load into shared memory, completion on an mbarrier.
@@ -312,7 +345,8 @@ cudaError_t launch_sparse_decode(const Shape &s, const CUtensorMap &kmap, const 
                                  const int32_t *page_table, const int32_t *seq_len, const void *q,
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
-                                 float *out, float *lse, uint32_t *err, cudaStream_t st);
+                                 uint32_t *grid_bar, float *out, float *lse, uint32_t *err,
+                                 cudaStream_t st);
 // maps: K half 0, K half 1, V half 0, V half 1 (2-D, 16 x 64 boxes, 128-byte swizzle).
 cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap *maps,
                                      const int32_t *page_table, const int32_t *seq_len, int f,

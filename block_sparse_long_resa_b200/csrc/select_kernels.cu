@@ -3,13 +3,18 @@
 // selection (Eq. 5 count from the caller, ties to the lower block index) with
 // the local block always appended.
 //
-// score_kernel streams the block key cache.  Grid (X, batch); CTA x owns a
-// contiguous range of complete blocks of one sequence.  Its producer warp
-// reads the page ids and issues cp.async.bulk copies of whole descriptor
-// pages (all kv heads, 2*d bf16 each) into a kScoreStages-deep shared-memory
-// ring, one copy per run of physically consecutive pages; four consumer warps
-// score two pages per stage each (lane = d/32 channels, one butterfly per
-// (page, head)).  Every score also bumps a 65536-bin histogram of the top 16
+// score_kernel streams the block key cache.  Grid (X, batch), one CTA per
+// SM; CTA x owns a contiguous range of complete blocks of one sequence, and
+// its 16 scoring warps take every 16th page of it.  Each warp streams its
+// descriptor pages (all kv heads, 2*d bf16 each) through a private ring in
+// shared memory with 16-byte cp.async copies, several pages in flight: these
+// go through the load/store path, which keeps HBM busy at any page size and
+// page order, where one bulk (TMA) copy per 2 KB page would be limited by
+// the copy engine's per-request rate.  Since q-bar is fixed for the call,
+// max(q*max, q*min) is q times the max where q >= 0 and the min elsewhere: a
+// byte permute picks that half, then one multiply and one add per channel
+// (lane = d/32 channels); one transposing shuffle reduction finishes the Hkv
+// sums of a page.  Every score also bumps a 65536-bin histogram of the top 16
 // bits of its order-preserving key, per (sequence, kv head), and the range of
 // touched bins, so the selection never scans the full key range for its first
 // digit.  In decode steps an extra warp of the first CTA of each sequence
@@ -22,9 +27,9 @@
 // counts the keys above that bin and gathers the bin's keys; the cluster's
 // candidates are exchanged through distributed shared memory and a radix
 // select of their low 16 bits gives the threshold T; per-CTA counts of keys
-// above / equal to T give each CTA its output offset, and a ballot pass
-// writes the blocks with key > T plus the lowest-index blocks with key == T
-// in ascending order.
+// above / equal to T, pushed into every CTA of the cluster, give each CTA its
+// output offset, and a ballot pass writes the blocks with key > T plus the
+// lowest-index blocks with key == T in ascending order.
 #include <cooperative_groups.h>
 
 #include "resa_common.cuh"
@@ -32,11 +37,32 @@
 namespace resa {
 namespace {
 
-constexpr int kScoreConsumers = 4;
-constexpr int kScoreGroup = 2 * kScoreConsumers;  // pages per stage: two per consumer warp
-constexpr int kScoreStages = 4;
-constexpr int kScoreThreads = 32 * (1 + kScoreConsumers + 1);  // producer, consumers, append
+constexpr int kScoreWarps = 16;                   // scoring warps per CTA (one CTA per SM)
+constexpr int kScoreRingBytes = 192 * 1024;       // shared-memory ring budget per CTA
+constexpr int kScoreThreads = 32 * (kScoreWarps + 1);  // + the decode-token append warp
 constexpr int kHistBins = 65536;
+constexpr int kHashSlots = 2048;  // per-CTA histogram aggregation table
+constexpr uint32_t kHashEmpty = 0xffffffffu;
+
+template <int D, int HKV>
+struct ScoreCfg {
+    static constexpr int kPageBytes = HKV * 2 * D * 2;  // one descriptor page, all kv heads
+    // pages in flight per warp (cp.async groups outstanding)
+    static constexpr int kFit = kScoreRingBytes / kScoreWarps / kPageBytes;
+    static constexpr int kRing = kFit < 8 ? kFit : 8;
+    static constexpr int kRingBytes = kScoreWarps * kRing * kPageBytes;
+    static_assert(kRing >= 2, "at least two pages in flight per warp");
+};
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ uint32_t order_key(float s) {
     s += 0.0f;  // -0 -> +0: equal scores get equal keys
@@ -66,23 +92,35 @@ __device__ __forceinline__ uint4 pack8(const Bf16x8 &r) {
     return x;
 }
 
-// grid (X, batch), block kScoreThreads, dynamic smem kScoreStages * kScoreGroup * page bytes.
+// Byte-permute selector taking, for the two bf16 channels of a 32-bit word,
+// the max half (from the second operand) where q >= 0 and the min half
+// (first operand) otherwise: q * that value is max(q * max, q * min).
+__device__ __forceinline__ uint32_t upper_bound_selector(float q0, float q1) {
+    const uint32_t b0 = q0 >= 0.f ? 4u : 0u, b1 = q1 >= 0.f ? 4u : 0u;
+    return (b0 + 0u) | ((b0 + 1u) << 4) | ((b1 + 2u) << 8) | ((b1 + 3u) << 12);
+}
+
+// grid (X, batch), block kScoreThreads, dynamic smem ScoreCfg::kRingBytes.
 template <int D, int HKV>
-__global__ void __launch_bounds__(kScoreThreads)
+__global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(uint16_t *__restrict__ desc, const int32_t *__restrict__ page_table,
                  const int32_t *__restrict__ seq_len, const uint16_t *__restrict__ q,
                  float *__restrict__ scores, uint32_t *__restrict__ hist,
                  uint32_t *__restrict__ hist_range, int g, int max_pages, int num_pages,
                  uint4 *__restrict__ K, uint4 *__restrict__ V, const uint4 *__restrict__ k_new,
                  const uint4 *__restrict__ v_new, uint32_t *err) {
+    using CF = ScoreCfg<D, HKV>;
     constexpr int PAGE_ELEMS = HKV * 2 * D;  // bf16 per descriptor page
-    constexpr int PAGE_BYTES = PAGE_ELEMS * 2;
+    constexpr int PAGE_CHUNKS = CF::kPageBytes / 16;
     constexpr int N = D / 32;                // channels per lane
-    extern __shared__ __align__(128) uint8_t ring[];
+    constexpr int RING = CF::kRing;
+    extern __shared__ __align__(128) uint8_t ring_all[];
     __shared__ float qbar_s[HKV][D];
-    __shared__ uint64_t full[kScoreStages], empty[kScoreStages];
-    __shared__ uint32_t stage_mask[kScoreStages];
-    __shared__ int stage_np[kScoreStages];
+    // Per-CTA aggregation of the key histogram: (head, top-16-bit digit) ->
+    // count in an open-addressing table, flushed with one global atomic per
+    // distinct entry; and the touched-digit range per head.
+    __shared__ uint32_t hkey[kHashSlots], hcnt[kHashSlots];
+    __shared__ uint32_t rng_min[HKV], rng_max[HKV];
 
     pdl_launch_next();
     const int b = blockIdx.y, x = blockIdx.x, X = gridDim.x;
@@ -91,78 +129,67 @@ __global__ void __launch_bounds__(kScoreThreads)
     const int L = seq_len[b];
     const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
     const int M = seq_ok ? (L - 1) / kBlock : 0;
-    const int per = ((M + X - 1) / X + kScoreGroup - 1) / kScoreGroup * kScoreGroup;
+    const int per = (M + X - 1) / X;
     const int p_begin = min(M, x * per), p_end = min(M, p_begin + per);
-    const int n_groups = (p_end - p_begin + kScoreGroup - 1) / kScoreGroup;
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kScoreStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kScoreConsumers);
+    if (warp < kScoreWarps) {
+        for (int i = threadIdx.x; i < kHashSlots; i += 32 * kScoreWarps) {
+            hkey[i] = kHashEmpty;
+            hcnt[i] = 0;
         }
-        fence_mbar_init();
-    }
-    __syncthreads();
+        if (threadIdx.x < HKV) {
+            rng_min[threadIdx.x] = 0xffffffffu;
+            rng_max[threadIdx.x] = 0;
+        }
+        // This warp's pages: p_begin + warp + kScoreWarps * t.  Lane t holds
+        // the id of the warp's page t of the current batch of 32 (the page
+        // table is an input of the call: read before waiting).
+        const int n_mine = p_end - p_begin > warp ? (p_end - p_begin - warp + kScoreWarps - 1) / kScoreWarps : 0;
+        auto batch_ids = [&](int t0) {
+            const int t = t0 + lane;
+            return t < n_mine ? page_table[(size_t)b * max_pages + p_begin + warp + kScoreWarps * t] : -1;
+        };
+        int ids = batch_ids(0);
+        pdl_wait();  // descriptors may be written by the preceding kernels
+        if (!seq_ok && x == 0 && warp == 0 && lane == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
 
-    if (warp == 0) {  // ------------------------------------------------ producer
-        static_assert(kScoreStages * kScoreGroup == 32, "one lane per page of the first stages");
-        // Page ids of the first kScoreStages groups (the page table is an
-        // input of the call): lane = group * kScoreGroup + slot.
-        int pg_first = -1;
-        {
-            const int p = p_begin + lane;
-            if (p < p_end) pg_first = page_table[(size_t)b * max_pages + p];
-        }
-        pdl_wait();  // descriptors and workspace may be written by the preceding kernels
-        if (!seq_ok && x == 0 && lane == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
-        for (int i = 0; i < n_groups; ++i) {
-            const int s = i % kScoreStages;
-            if (i >= kScoreStages && !mbar_wait_bounded(&empty[s], ((i / kScoreStages) - 1) & 1)) {
-                if (lane == 0) set_error(err, RESA_DEVERR_TIMEOUT);
-                break;
-            }
-            const int p0 = p_begin + i * kScoreGroup;
-            const int npg = min(kScoreGroup, p_end - p0);
-            int pg = -1;
-            if (i < kScoreStages) {
-                pg = __shfl_sync(0xffffffffu, pg_first, (i * kScoreGroup + lane) & 31);
-                if (lane >= npg) pg = -1;
-            } else if (lane < npg) {
-                pg = page_table[(size_t)b * max_pages + p0 + lane];
-            }
-            if (lane < npg && (pg < 0 || pg >= num_pages)) {
-                set_error(err, RESA_DEVERR_PAGE);
-                pg = -1;
-            }
-            const uint32_t all = (1u << npg) - 1u;  // npg <= kScoreGroup < 32
-            const uint32_t vmask = __ballot_sync(0xffffffffu, lane < npg && pg >= 0);
-            const int first = __shfl_sync(0xffffffffu, pg, 0);
-            const bool contiguous =
-                vmask == all && __ballot_sync(0xffffffffu, lane < npg && pg == first + lane) == all;
-            const uint32_t bytes = (uint32_t)__popc(vmask) * PAGE_BYTES;
-            uint8_t *dst = ring + (size_t)s * kScoreGroup * PAGE_BYTES;
-            if (lane == 0) {
-                stage_mask[s] = vmask;
-                stage_np[s] = npg;
-                if (bytes == 0)
-                    mbar_arrive(&full[s]);
-                else
-                    mbar_arrive_expect_tx(&full[s], bytes);
-            }
-            __syncwarp();
-            if (bytes > 0) {
-                if (contiguous) {
-                    if (lane == 0) bulk_load(dst, desc + (size_t)first * PAGE_ELEMS, bytes, &full[s]);
-                } else if (lane < npg && pg >= 0) {
-                    bulk_load(dst + (size_t)lane * PAGE_BYTES, desc + (size_t)pg * PAGE_ELEMS,
-                              PAGE_BYTES, &full[s]);
+        uint8_t *ring = ring_all + (size_t)warp * RING * CF::kPageBytes;
+        uint32_t valid_b = 0;
+        auto check_batch = [&](int t0) {
+            const bool v = ids >= 0 && ids < num_pages;
+            if (t0 + lane < n_mine && !v) set_error(err, RESA_DEVERR_PAGE);
+            valid_b = __ballot_sync(0xffffffffu, t0 + lane < n_mine && v);
+        };
+        check_batch(0);
+        // Copy of page t into ring slot t % RING, one cp.async group per page
+        // (empty groups past the end keep the group count uniform).  Pages are
+        // issued in order; the ids of batch t >> 5 are in `ids`.
+        uint32_t slot_valid = 0;  // bit t % RING: page t's id was valid (uniform over the warp)
+        auto issue_page = [&](int t) {
+            if (t < n_mine) {
+                if ((t & 31) == 0 && t > 0) {
+                    ids = batch_ids(t);
+                    check_batch(t);
+                }
+                const int pg = __shfl_sync(0xffffffffu, ids, t & 31);
+                const uint32_t ok = (valid_b >> (t & 31)) & 1u;
+                const int slot = t % RING;
+                slot_valid = (slot_valid & ~(1u << slot)) | (ok << slot);
+                if (ok) {
+                    const uint8_t *src = reinterpret_cast<const uint8_t *>(desc + (size_t)pg * PAGE_ELEMS);
+                    uint8_t *dst = ring + (size_t)(t % RING) * CF::kPageBytes;
+#pragma unroll
+                    for (int c = lane; c < PAGE_CHUNKS; c += 32) cp_async16(dst + c * 16, src + c * 16);
                 }
             }
-        }
-    } else if (warp <= kScoreConsumers) {  // ------------------------- consumers
-        // Group pooling: mean of the g query heads, fp32, head order, then / g
-        // (q is an input of the call, read while the first copies are in flight).
-        for (int e = threadIdx.x - 32; e < HKV * D; e += 32 * kScoreConsumers) {
+            cp_async_commit();
+        };
+#pragma unroll
+        for (int t = 0; t < RING - 1; ++t) issue_page(t);
+
+        // Group pooling while the first pages are in flight: mean of the g
+        // query heads, fp32, head order, then / g.
+        for (int e = threadIdx.x; e < HKV * D; e += 32 * kScoreWarps) {
             const int h = e / D, j = e % D;
             const uint16_t *col = q + ((size_t)b * hq + (size_t)h * g) * D + j;
             uint16_t v[kMaxGroup];
@@ -174,89 +201,117 @@ __global__ void __launch_bounds__(kScoreThreads)
                 if (r < g) s += bf16_bits_to_f32(v[r]);
             qbar_s[h][j] = s / (float)g;
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(32 * kScoreConsumers) : "memory");
-        pdl_wait();
-        const int c = warp - 1;
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * kScoreWarps) : "memory");
         float qv[HKV][N];
+        uint32_t sel[HKV][N / 2];
 #pragma unroll
-        for (int h = 0; h < HKV; ++h)
+        for (int h = 0; h < HKV; ++h) {
 #pragma unroll
             for (int n = 0; n < N; ++n) qv[h][n] = qbar_s[h][lane * N + n];
-        // lane t < 2*HKV owns output (page c*2 + t / HKV, head t % HKV)
-        const int my_pp = lane / HKV, my_h = lane % HKV;
-        const bool owner = lane < 2 * HKV;
+#pragma unroll
+            for (int n = 0; n < N / 2; ++n) sel[h][n] = upper_bound_selector(qv[h][2 * n], qv[h][2 * n + 1]);
+        }
+
+        // Head h of a page is value h; after the transposing reduction lane
+        // l holds the full sum of head l >> (5 - kLogP) and lane h << (5 - kLogP)
+        // owns head h's output.
+        constexpr int kLogP = HKV == 1 ? 0 : HKV == 2 ? 1 : HKV == 4 ? 2 : 3;
+        static_assert((1 << kLogP) == HKV, "power-of-two kv heads");
+        const int my_h = lane >> (5 - kLogP);
+        const bool owner = (lane & ((1 << (5 - kLogP)) - 1)) == 0;
+        const size_t unit = (size_t)b * HKV + my_h;
         uint32_t dmin = 0xffffffffu, dmax = 0;
-        for (int i = 0; i < n_groups; ++i) {
-            const int s = i % kScoreStages;
-            if (!mbar_wait_bounded(&full[s], (i / kScoreStages) & 1)) {
-                if (lane == 0) set_error(err, RESA_DEVERR_TIMEOUT);
-                break;
+        for (int t = 0; t < n_mine; ++t) {
+            issue_page(t + RING - 1);  // refills the slot of page t - 1
+            cp_async_wait<RING - 1>();
+            __syncwarp();
+            const uint8_t *pgp = ring + (size_t)(t % RING) * CF::kPageBytes;
+            // Partial sums of this lane's channels: sum over n of q_n * (max_n
+            // if q_n >= 0 else min_n), products rounded, added in channel order.
+            float v[HKV];
+#pragma unroll
+            for (int h = 0; h < HKV; ++h) {
+                const uint16_t *row = reinterpret_cast<const uint16_t *>(pgp + (size_t)h * 2 * D * 2);
+                uint32_t mnw[N / 2], mxw[N / 2];
+                if constexpr (N == 4) {
+                    const uint2 a = *reinterpret_cast<const uint2 *>(row + lane * 4);
+                    const uint2 z = *reinterpret_cast<const uint2 *>(row + D + lane * 4);
+                    mnw[0] = a.x;
+                    mnw[1] = a.y;
+                    mxw[0] = z.x;
+                    mxw[1] = z.y;
+                } else {
+                    mnw[0] = *reinterpret_cast<const uint32_t *>(row + lane * 2);
+                    mxw[0] = *reinterpret_cast<const uint32_t *>(row + D + lane * 2);
+                }
+                float sum = 0.f;
+#pragma unroll
+                for (int n = 0; n < N / 2; ++n) {
+                    const uint32_t w = __byte_perm(mnw[n], mxw[n], sel[h][n]);
+                    sum = __fadd_rn(sum, __fmul_rn(qv[h][2 * n], __uint_as_float(w << 16)));
+                    sum = __fadd_rn(sum, __fmul_rn(qv[h][2 * n + 1], __uint_as_float(w & 0xffff0000u)));
+                }
+                v[h] = sum;
             }
-            const uint32_t vmask = stage_mask[s];
-            const int npg = stage_np[s];
-            const uint8_t *st = ring + (size_t)s * kScoreGroup * PAGE_BYTES;
-            float mine = 0.f;
+            __syncwarp();  // the slot is refilled by the next issue
+            // Transposing reduction: each step halves the values a lane keeps
+            // (upper half where the step's lane bit is set) and adds the
+            // partner's copy of the same heads.
 #pragma unroll
-            for (int pp = 0; pp < 2; ++pp) {
-                const int j = c * 2 + pp;
-                const bool present = j < npg && ((vmask >> j) & 1u);
+            for (int k = 0; k < kLogP; ++k) {
+                const int mask = 16 >> k;
+                const int half = HKV >> (k + 1);
+                const bool upper = (lane & mask) != 0;
 #pragma unroll
-                for (int h = 0; h < HKV; ++h) {
-                    float sum = 0.f;
-                    if (present) {
-                        const uint16_t *row = reinterpret_cast<const uint16_t *>(
-                            st + (size_t)j * PAGE_BYTES + (size_t)h * 2 * D * 2);
-                        float mn[N], mx[N];
-                        if constexpr (N == 4) {
-                            const uint2 a = *reinterpret_cast<const uint2 *>(row + lane * 4);
-                            const uint2 z = *reinterpret_cast<const uint2 *>(row + D + lane * 4);
-                            mn[0] = bf_lo(a.x);
-                            mn[1] = bf_hi(a.x);
-                            mn[2] = bf_lo(a.y);
-                            mn[3] = bf_hi(a.y);
-                            mx[0] = bf_lo(z.x);
-                            mx[1] = bf_hi(z.x);
-                            mx[2] = bf_lo(z.y);
-                            mx[3] = bf_hi(z.y);
-                        } else {
-                            const uint32_t a = *reinterpret_cast<const uint32_t *>(row + lane * 2);
-                            const uint32_t z = *reinterpret_cast<const uint32_t *>(row + D + lane * 2);
-                            mn[0] = bf_lo(a);
-                            mn[1] = bf_hi(a);
-                            mx[0] = bf_lo(z);
-                            mx[1] = bf_hi(z);
-                        }
-#pragma unroll
-                        for (int n = 0; n < N; ++n) sum += fmaxf(qv[h][n] * mx[n], qv[h][n] * mn[n]);
-                    }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                    if (pp == my_pp && h == my_h) mine = sum;
+                for (int j = 0; j < half; ++j) {
+                    const float send = upper ? v[j] : v[j + half];
+                    const float keep = upper ? v[j + half] : v[j];
+                    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-            const int j = c * 2 + my_pp;
-            if (owner && j < npg && ((vmask >> j) & 1u)) {
-                const size_t unit = (size_t)b * HKV + my_h;
-                scores[unit * max_pages + p_begin + i * kScoreGroup + j] = mine;
+#pragma unroll
+            for (int mask = 16 >> kLogP; mask > 0; mask >>= 1)
+                v[0] += __shfl_xor_sync(0xffffffffu, v[0], mask);
+            const int page_idx = p_begin + warp + kScoreWarps * t;
+            const bool page_ok = ((slot_valid >> (t % RING)) & 1u) != 0;
+            if (owner && page_ok) {
+                const float mine = v[0];
+                scores[unit * max_pages + page_idx] = mine;
                 const uint32_t digit = order_key(mine) >> 16;
-                atomicAdd(&hist[unit * kHistBins + digit], 1u);
+                const uint32_t key = ((uint32_t)my_h << 16) | digit;
+                uint32_t slot = (digit * 0x9E3779B1u + (uint32_t)my_h * 0x85EBCA77u) >> 21;  // 11 bits
+                bool placed = false;
+                for (int probe = 0; probe < 64; ++probe) {
+                    const uint32_t old = atomicCAS(&hkey[slot], kHashEmpty, key);
+                    if (old == kHashEmpty || old == key) {
+                        atomicAdd(&hcnt[slot], 1u);
+                        placed = true;
+                        break;
+                    }
+                    slot = (slot + 1) & (kHashSlots - 1);
+                }
+                if (!placed) atomicAdd(&hist[unit * kHistBins + digit], 1u);  // crowded table
                 dmin = min(dmin, digit);
                 dmax = max(dmax, digit);
             }
         }
-        // touched-bin range per (sequence, head): lanes h and h + HKV share head h
-        const uint32_t omin = __shfl_down_sync(0xffffffffu, dmin, HKV);
-        const uint32_t omax = __shfl_down_sync(0xffffffffu, dmax, HKV);
-        if (lane < HKV) {
-            dmin = min(dmin, omin);
-            dmax = max(dmax, omax);
-            if (dmin <= dmax) {
-                const size_t unit = (size_t)b * HKV + lane;
-                atomicMax(&hist_range[2 * unit], (uint32_t)kHistBins - dmin);  // 0 = untouched
-                atomicMax(&hist_range[2 * unit + 1], dmax + 1u);
-            }
+        cp_async_wait<0>();
+        if (owner && dmin <= dmax) {
+            atomicMin(&rng_min[my_h], dmin);
+            atomicMax(&rng_max[my_h], dmax);
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * kScoreWarps) : "memory");
+        // Flush: one global atomic per distinct (head, digit) of the CTA, and
+        // the touched-bin range once per head.
+        for (int i = threadIdx.x; i < kHashSlots; i += 32 * kScoreWarps) {
+            const uint32_t key = hkey[i];
+            if (key != kHashEmpty)
+                atomicAdd(&hist[((size_t)b * HKV + (key >> 16)) * kHistBins + (key & 0xffffu)], hcnt[i]);
+        }
+        if (threadIdx.x < HKV && rng_min[threadIdx.x] <= rng_max[threadIdx.x]) {
+            const size_t u = (size_t)b * HKV + threadIdx.x;
+            atomicMax(&hist_range[2 * u], (uint32_t)kHistBins - rng_min[threadIdx.x]);  // 0 = untouched
+            atomicMax(&hist_range[2 * u + 1], rng_max[threadIdx.x] + 1u);
         }
     } else if (K != nullptr && x == 0) {  // ------------------------ decode-token append
         pdl_wait();
@@ -403,7 +458,8 @@ __global__ void __launch_bounds__(kSelThreads)
     __shared__ uint32_t warp_tot[kSelWarps], warp_gt[kSelWarps], warp_eq[kSelWarps];
     __shared__ uint32_t sh[4];
     __shared__ uint32_t lc_n;                   // candidates of this CTA
-    __shared__ uint32_t cta_gt, cta_eq;         // keys > T / == T in this CTA's slice
+    __shared__ uint32_t cta_gt[kSelCluster];    // keys > T / == T in each CTA's slice
+    __shared__ uint32_t cta_eq[kSelCluster];
 
     pdl_launch_next();
     const int rank = (int)cluster.block_rank();
@@ -427,8 +483,23 @@ __global__ void __launch_bounds__(kSelThreads)
     const int c0 = min(M, rank * C), c1 = min(M, c0 + C);
     pdl_wait();
 
+    // This CTA's first slice keys are requested before the histogram is read.
+    const float *src = scores + unit * max_pages;
+    const int n_mine = c1 - c0;
+    const bool in_smem = n_mine <= kSelKeys;
+    const int R = (n_mine + kSelWarps - 1) / kSelWarps;
+    const int w0 = c0 + warp * R, w1 = min(c1, w0 + R);
+    constexpr int U = 4;
+    float first[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int i = w0 + u * 32 + lane;
+        first[u] = i < w1 ? src[i] : 0.f;
+    }
+
     // Boundary bin of the k-th largest key from the scorer's histogram
     // (every CTA of the cluster computes the same; rank 0 clears it later).
+    // Thread t sums bins dmax - t*chunk down to dmax - (t+1)*chunk + 1.
     const uint32_t emin = hist_range[2 * unit], emax = hist_range[2 * unit + 1];
     const int dmin = (int)(kHistBins - emin), dmax = (int)emax - 1;
     const int nbins = dmax >= dmin ? dmax - dmin + 1 : 0;
@@ -437,24 +508,44 @@ __global__ void __launch_bounds__(kSelThreads)
         lc_n = 0;
         sh[0] = sh[1] = 0;
     }
+    constexpr int kBinRegs = 8;
     const int chunk = (nbins + kSelThreads - 1) / kSelThreads;
     const int top = dmax - tid * chunk;
     const int lo = max(dmin, top - chunk + 1);
+    uint32_t binc[kBinRegs];
     uint32_t local = 0;
-    for (int d = top; d >= lo; --d) local += __ldcg(&hb[d]);
+    if (chunk <= kBinRegs) {
+#pragma unroll
+        for (int j = 0; j < kBinRegs; ++j) binc[j] = (j < chunk && top - j >= lo) ? __ldcg(&hb[top - j]) : 0u;
+#pragma unroll
+        for (int j = 0; j < kBinRegs; ++j) local += binc[j];
+    } else {
+        for (int d = top; d >= lo; --d) local += __ldcg(&hb[d]);
+    }
     uint32_t total;
     const uint32_t above_me = cta_exclusive_scan(local, warp_tot, total);
     const bool trivial = !seq_ok || k == M || k == 0;
     if (!trivial && above_me < (uint32_t)k && (uint32_t)k <= above_me + local) {
         uint32_t cum = above_me;
-        for (int d = top; d >= lo; --d) {
-            const uint32_t c = __ldcg(&hb[d]);
-            if (cum + c >= (uint32_t)k) {
-                sh[0] = (uint32_t)d;  // boundary digit
-                sh[1] = cum;          // keys above it
-                break;
+        if (chunk <= kBinRegs) {
+#pragma unroll
+            for (int j = 0; j < kBinRegs; ++j) {
+                if (j < chunk && top - j >= lo && cum < (uint32_t)k && cum + binc[j] >= (uint32_t)k) {
+                    sh[0] = (uint32_t)(top - j);  // boundary digit
+                    sh[1] = cum;                  // keys above it
+                }
+                cum += binc[j];
             }
-            cum += c;
+        } else {
+            for (int d = top; d >= lo; --d) {
+                const uint32_t c = __ldcg(&hb[d]);
+                if (cum + c >= (uint32_t)k) {
+                    sh[0] = (uint32_t)d;
+                    sh[1] = cum;
+                    break;
+                }
+                cum += c;
+            }
         }
     }
     __syncthreads();
@@ -464,21 +555,15 @@ __global__ void __launch_bounds__(kSelThreads)
 
     // One pass over this CTA's slice: keys into shared memory, per-warp count
     // of keys above the boundary bin, the bin's keys as candidates.
-    const float *src = scores + unit * max_pages;
-    const int n_mine = c1 - c0;
-    const bool in_smem = n_mine <= kSelKeys;
-    const int R = (n_mine + kSelWarps - 1) / kSelWarps;
-    const int w0 = c0 + warp * R, w1 = min(c1, w0 + R);
     const uint32_t lt_mask = (1u << lane) - 1u;
     uint32_t above_w = 0;
     if (!trivial) {
-        constexpr int U = 4;
         for (int base = w0; base < w1; base += 32 * U) {
             uint32_t kv[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int i = base + u * 32 + lane;
-                kv[u] = i < w1 ? order_key(src[i]) : 0u;
+                kv[u] = i < w1 ? order_key(base == w0 ? first[u] : src[i]) : 0u;
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -521,21 +606,30 @@ __global__ void __launch_bounds__(kSelThreads)
     bool fallback = trivial ? false : !hist_ok;
     if (!trivial) {
         // Gather the cluster's candidates (distributed shared memory).
-        uint32_t offs[kSelCluster], ntot = 0;
+        uint32_t nr[kSelCluster], offs[kSelCluster + 1];
+#pragma unroll
+        for (int r = 0; r < kSelCluster; ++r) nr[r] = *cluster.map_shared_rank(&lc_n, r);
+        offs[0] = 0;
 #pragma unroll
         for (int r = 0; r < kSelCluster; ++r) {
-            const uint32_t n = *cluster.map_shared_rank(&lc_n, r);
-            offs[r] = ntot;
-            ntot += n;
-            if (n > (uint32_t)kSelLocalCand) fallback = true;
+            offs[r + 1] = offs[r] + nr[r];
+            if (nr[r] > (uint32_t)kSelLocalCand) fallback = true;
         }
+        const uint32_t ntot = offs[kSelCluster];
         if (ntot > (uint32_t)kSelCandCap) fallback = true;
         if (!fallback) {
+            // one flattened loop over the cluster's candidates: the remote
+            // loads of all ranks are in flight together
+            for (uint32_t j = tid; j < ntot; j += kSelThreads) {
+                int r = 0;
+                uint32_t base = 0;
 #pragma unroll
-            for (int r = 0; r < kSelCluster; ++r) {
-                const uint32_t *peer = cluster.map_shared_rank(lc_key, r);
-                const uint32_t n = (r + 1 < kSelCluster ? offs[r + 1] : ntot) - offs[r];
-                for (uint32_t i = tid; i < n; i += kSelThreads) all_c[offs[r] + i] = peer[i];
+                for (int q = 1; q < kSelCluster; ++q)
+                    if (j >= offs[q]) {
+                        r = q;
+                        base = offs[q];
+                    }
+                all_c[j] = cluster.map_shared_rank(lc_key, r)[j - base];
             }
             __syncthreads();
             uint32_t cp = 0, cm = 0;
@@ -577,16 +671,19 @@ __global__ void __launch_bounds__(kSelThreads)
         }
     }
     __syncthreads();
-    if (tid == 0) {
+    // This CTA's counts go into every CTA's table (remote stores), so that
+    // after the next cluster barrier no CTA reads a peer's shared memory and
+    // each may leave when done.
+    if (tid < kSelCluster) {
         uint32_t g2 = 0, e2 = 0;
         for (int w = 0; w < kSelWarps; ++w) {
             g2 += warp_gt[w];
             e2 += warp_eq[w];
         }
-        cta_gt = g2;
-        cta_eq = e2;
+        cluster.map_shared_rank(cta_gt, tid)[rank] = g2;
+        cluster.map_shared_rank(cta_eq, tid)[rank] = e2;
     }
-    cluster.sync();  // #2: per-CTA counts visible to the cluster
+    cluster.sync();  // #2: every CTA has read its peers' candidates; count tables complete
 
     if (trivial) {
         if (seq_ok) {
@@ -602,8 +699,8 @@ __global__ void __launch_bounds__(kSelThreads)
     } else {
         uint32_t gt_before = 0, eq_before = 0;
         for (int r = 0; r < rank; ++r) {
-            gt_before += *cluster.map_shared_rank(&cta_gt, r);
-            eq_before += *cluster.map_shared_rank(&cta_eq, r);
+            gt_before += cta_gt[r];
+            eq_before += cta_eq[r];
         }
         for (int w = 0; w < warp; ++w) {
             gt_before += warp_gt[w];
@@ -632,7 +729,6 @@ __global__ void __launch_bounds__(kSelThreads)
             *cnt = k + 1;
         }
     }
-    cluster.sync();  // #3: no CTA leaves while a peer may still read its shared memory
 }
 
 template <int D>
@@ -640,14 +736,14 @@ cudaError_t launch_score_d(const Shape &s, void *desc, const int32_t *page_table
                            const int32_t *seq_len, const void *q, float *scores, uint32_t *hist,
                            uint32_t *hist_range, void *K, void *V, const void *k_new,
                            const void *v_new, uint32_t *err, cudaStream_t st) {
-    // ~2 CTAs per SM over all sequences, at least 4 stages of pages each
-    const int by_work = (s.max_pages + 4 * kScoreGroup - 1) / (4 * kScoreGroup);
-    const int by_sm = (2 * kNumSms + s.batch - 1) / s.batch;
+    // One CTA per SM over all sequences, at least two pages per scoring warp.
+    const int by_work = (s.max_pages + 2 * kScoreWarps - 1) / (2 * kScoreWarps);
+    const int by_sm = s.batch < kNumSms ? kNumSms / s.batch : 1;
     const int X = max(1, min(by_work, by_sm));
     dim3 grid(X, s.batch);
 #define RESA_SCORE_CASE(H)                                                                    \
     case H: {                                                                                 \
-        constexpr int smem = kScoreStages * kScoreGroup * H * 2 * D * 2;                      \
+        constexpr int smem = ScoreCfg<D, H>::kRingBytes;                                      \
         static std::atomic<int> done[64];                                                     \
         cudaError_t e = ensure_smem(score_kernel<D, H>, smem, done);                          \
         if (e != cudaSuccess) return e;                                                       \

@@ -149,7 +149,8 @@ RESA_API resa_status_t resa_select_blocks(const resa_config_t *cfg, const resa_c
  * sm_scale * q.k, split across SMs with a log-sum-exp combine.  K/V of a
  * block are fetched once per group.  q [batch][Hq][d] bf16; out
  * [batch][Hq][d] fp32; lse_opt (nullable) [batch][Hq] fp32, natural log.
- * Block ids outside the sequence set RESA_DEVERR_BLOCK and are skipped. */
+ * Block ids outside the sequence set RESA_DEVERR_BLOCK and are skipped.
+ * max_topk + 1 above 1024 * 512 blocks returns RESA_ERR_RANGE. */
 RESA_API resa_status_t resa_sparse_decode(const resa_config_t *cfg, const resa_cache_t *cache,
                                  const void *q, const int32_t *block_idx,
                                  const int32_t *block_cnt, int32_t max_topk, float *out,

@@ -82,6 +82,8 @@ RAGGED = dict(seed=3, batch=5, num_q_heads=28, num_kv_heads=4, head_dim=128, blo
               ctx_lens=[1, 15, 16, 300, 5003], topk=[4, 16, 16, 7, 500], paged=True)
 RAGGED64 = dict(seed=4, batch=3, num_q_heads=8, num_kv_heads=1, head_dim=64, block_size=16,
                 ctx_lens=[33, 257, 1111], topk=[100, 3, 60], paged=True)
+GQA8 = dict(seed=5, batch=2, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+            ctx_lens=[20000, 7777], topk=[125, 48], paged=True)  # 8 kv heads: 16 KB stages
 
 
 def make(case, device="cpu", **over):
@@ -117,8 +119,8 @@ def test_build_descriptors_from_first_block(cuda_device):
     np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
 
 
-@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED, RAGGED64], ids=["tiny", "qwen32k",
-                                                                         "ragged", "ragged64"])
+@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED, RAGGED64, GQA8],
+                         ids=["tiny", "qwen32k", "ragged", "ragged64", "gqa8"])
 def test_decode_step_matches_oracle(cuda_device, case):
     p = make(case)
     cfg, lc, ws = setup_layer(p, cuda_device)
@@ -157,7 +159,8 @@ def test_decode_step_matches_oracle(cuda_device, case):
                 assert set(p.needle_blocks[b, h].tolist()) <= sel
 
 
-@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED], ids=["tiny", "qwen32k", "ragged"])
+@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED, GQA8],
+                         ids=["tiny", "qwen32k", "ragged", "gqa8"])
 def test_select_blocks_scores(cuda_device, case):
     p = make(case)
     cfg, lc, ws = setup_layer(p, cuda_device)
@@ -236,6 +239,36 @@ def test_sparse_decode_given_blocks(cuda_device):
                          torch.from_numpy(cnt).to(cuda_device), 301, out, lse, ws)
     code = R.resa_check_device_status(ws, raise_on_error=False)
     assert code & R.DEVERR_BLOCK
+
+
+def test_sparse_decode_split_merge_beyond_one_wave(cuda_device):
+    """38 sequences x 4 kv heads = 152 (sequence, head) units with 520+1 blocks
+    each: two splits per unit (512-block cap) give 304 CTAs, more than one
+    wave, so the splits are merged by the last CTA of each unit instead of
+    across the grid."""
+    p = make(dict(seed=9, batch=38, num_q_heads=8, num_kv_heads=4, head_dim=128,
+                  block_size=16, ctx_lens=[8400] * 38, topk=[16] * 38))
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len.clone()
+    B, Hkv = p.batch, p.num_kv_heads
+    M = (int(L[0]) - 1) // 16
+    rng = np.random.default_rng(11)
+    n = 520
+    idx = np.full((B, Hkv, n + 1), -1, dtype=np.int32)
+    cnt = np.full((B, Hkv), n + 1, dtype=np.int32)
+    for b in range(B):
+        for h in range(Hkv):
+            idx[b, h, :n] = np.sort(rng.choice(M, size=n, replace=False))
+            idx[b, h, n] = M
+    out = torch.empty(B, 8, 128, device=cuda_device)
+    lse = torch.empty(B, 8, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_sparse_decode(cfg, lc.struct(), dev(p.q), dev(torch.from_numpy(idx)),
+                         dev(torch.from_numpy(cnt)), n, out, lse, ws)
+    assert_no_device_error(ws)
+    ref, ref_lse = oracle_of(p).sparse_attention(p.q, idx, cnt, L)
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
 
 
 def test_all_blocks_equals_dense(cuda_device):
