@@ -6,10 +6,12 @@
 // every eighth block of the slice and keeps its own online-softmax state for
 // the group's g query heads, so the K/V of a block are fetched once for the
 // whole group.  Each warp streams its blocks through a private ring of
-// kStages shared-memory stages: lane 0 issues two 3-D TMA loads per block
-// (the (page, head) K and V tiles of 16 x D bf16, 128-byte swizzled) that
-// complete on the stage's mbarrier.  Block ids and pages of the slice are
-// staged in shared memory once, up front.
+// kStages shared-memory stages with 16-byte cp.async copies (the (page,
+// head) K and V tiles of 16 x D bf16, laid out 128-byte swizzled for
+// ldmatrix): copies through the load/store path keep HBM busy with 4 KB
+// tiles, where one TMA request per tile is limited by the copy engine's
+// per-request rate.  Block ids and pages of the slice are staged in shared
+// memory once, up front.
 //
 // The MMAs run with the operands swapped, S^T = K Q^T and O^T = V^T P^T
 // (bf16 m16n8k16, fp32 accumulate), so the g <= 8 heads of a group fill the
@@ -28,7 +30,7 @@
 namespace resa {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = kDecodeWarps;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 3;
 
@@ -144,59 +146,105 @@ __device__ __forceinline__ void attend_block_swapped(WarpState<D, NT> &st,
     }
 }
 
-// Split merge spread over the whole (co-resident) grid.  Work item = (unit,
-// row, 32 output channels); CTA c takes items c, c + gridsize, ...  Every
-// warp forms the row's log-sum-exp over the S splits in one pass (online max
-// and sum), then takes splits w, w + 8, ... of the item with all its loads in
-// flight together; the eight warps' sums are added through shared memory.
+// Block-wide reductions through shared memory (red: kWarps floats + 1).
+__device__ __forceinline__ float block_max(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        float x = lane < kWarps ? red[lane] : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+        if (lane == 0) red[kWarps] = x;
+    }
+    __syncthreads();
+    const float r = red[kWarps];
+    __syncthreads();
+    return r;
+}
+__device__ __forceinline__ float block_sum(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        float x = lane < kWarps ? red[lane] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) red[kWarps] = x;
+    }
+    __syncthreads();
+    const float r = red[kWarps];
+    __syncthreads();
+    return r;
+}
+
+// Merge of per-warp partials spread over the whole (co-resident) grid.
+// Partial p of unit u holds, per query row, the row max m (log2 domain), the
+// sum l of 2^(x - m) and the unnormalised sum o of 2^(x - m) * v over the
+// warp's blocks.  Work item = (unit, row, 32 output channels); CTA c takes
+// items c, c + gridsize, ...  Each warp first requests its partials' o
+// values (w, w + 8, ...: up to kB loads in flight per lane, independent of
+// the weights), then the CTA reads every partial's (m, l), forms M = max m
+// and the weights 2^(m - M), L = sum of l * 2^(m - M), and each warp adds
+// its weighted o values; out = (sum of the eight warps) / L.
 template <int D>
-__device__ __forceinline__ void merge_splits_spread(const float *__restrict__ part_o,
-                                                    const float *__restrict__ part_lse, int S,
+__device__ __forceinline__ void merge_warp_partials(const float *__restrict__ part_o,
+                                                    const float2 *__restrict__ part_ml, int P,
                                                     int hkv, int g, float *__restrict__ out,
-                                                    float *__restrict__ lse_out, float *red) {
+                                                    float *__restrict__ lse_out, float *smem_f) {
     constexpr int C32 = D / 32;
-    constexpr int kBatch = 8;
+    constexpr int kB = 40;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nctas = gridDim.x * gridDim.y * gridDim.z;
     const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
     const int units = gridDim.y * gridDim.z;
     const int n_items = units * g * C32;
     const float kLn2 = 0.6931471805599453f;
+    float *msm = smem_f;             // [P] row max of each partial
+    float *wsm = msm + P;            // [P] its weight 2^(m - M) (0 without data)
+    float *lsm = wsm + P;            // [P] its l
+    float *red = lsm + P;            // [kWarps * 32] warp sums, reduction scratch
     for (int item = cta; item < n_items; item += nctas) {
         const int u = item / (g * C32), rem = item % (g * C32);
         const int r = rem / C32, cc = rem % C32;
-        const float *ul = part_lse + (size_t)u * S * kMaxGroup + r;
-        const float *uo = part_o + ((size_t)u * S * kMaxGroup + r) * D + cc * 32 + lane;
-        float m = -INFINITY, l = 0.f;
-        for (int sp = lane; sp < S; sp += 32) {
-            const float x = __ldcg(ul + (size_t)sp * kMaxGroup);
-            if (x == -INFINITY) continue;
-            const float mn = fmaxf(m, x);
-            l = l * exp2f(m - mn) + exp2f(x - mn);
-            m = mn;
-        }
+        const float2 *ml = part_ml + (size_t)u * P * kMaxGroup + r;
+        const float *uo = part_o + ((size_t)u * P * kMaxGroup + r) * D + cc * 32 + lane;
+        float v[kB];
+        auto load_pass = [&](int base) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-            const float lo = __shfl_xor_sync(0xffffffffu, l, o);
-            const float mn = fmaxf(m, mo);
-            if (mn != -INFINITY) {
-                l = l * exp2f(m - mn) + lo * exp2f(mo - mn);
-                m = mn;
+            for (int k = 0; k < kB; ++k) {
+                const int pp = base + kWarps * k;
+                v[k] = pp < P ? __ldcg(uo + (size_t)pp * kMaxGroup * D) : 0.f;
             }
+        };
+        load_pass(warp);
+        float tmax = -INFINITY;
+        for (int pp = threadIdx.x; pp < P; pp += kThreads) {
+            const float2 x = __ldcg(ml + (size_t)pp * kMaxGroup);
+            msm[pp] = x.x;
+            lsm[pp] = x.y;
+            if (x.y > 0.f) tmax = fmaxf(tmax, x.x);
         }
+        const float M = block_max(tmax, red);
+        float tl = 0.f;
+        for (int pp = threadIdx.x; pp < P; pp += kThreads) {
+            const float w = lsm[pp] > 0.f ? exp2f(msm[pp] - M) : 0.f;
+            wsm[pp] = w;
+            tl += lsm[pp] * w;
+        }
+        const float Lsum = block_sum(tl, red);  // its barriers also publish wsm
         float acc = 0.f;
-        for (int s0 = warp; s0 < S; s0 += kWarps * kBatch) {
-            float v[kBatch], x[kBatch];
+        for (int base = warp; base < P; base += kWarps * kB) {
+            if (base != warp) load_pass(base);
 #pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-                const int sp = s0 + k * kWarps;
-                v[k] = sp < S ? __ldcg(uo + (size_t)sp * kMaxGroup * D) : 0.f;
-                x[k] = sp < S ? __ldcg(ul + (size_t)sp * kMaxGroup) : -INFINITY;
+            for (int k = 0; k < kB; ++k) {
+                const int pp = base + kWarps * k;
+                if (pp < P) acc += wsm[pp] * v[k];
             }
-#pragma unroll
-            for (int k = 0; k < kBatch; ++k)
-                if (x[k] != -INFINITY) acc += exp2f(x[k] - m) * v[k];
         }
         red[warp * 32 + lane] = acc;
         __syncthreads();
@@ -205,9 +253,9 @@ __device__ __forceinline__ void merge_splits_spread(const float *__restrict__ pa
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) o += red[w * 32 + lane];
             const size_t orow = (size_t)(u / hkv) * hkv * g + (size_t)(u % hkv) * g + r;
-            out[orow * D + cc * 32 + lane] = l > 0.f ? o / l : 0.f;
+            out[orow * D + cc * 32 + lane] = Lsum > 0.f ? o / Lsum : 0.f;
             if (lse_out && cc == 0 && lane == 0)
-                lse_out[orow] = (l > 0.f ? m + log2f(l) : -INFINITY) * kLn2;
+                lse_out[orow] = (Lsum > 0.f ? M + log2f(Lsum) : -INFINITY) * kLn2;
         }
         __syncthreads();
     }
@@ -215,8 +263,7 @@ __device__ __forceinline__ void merge_splits_spread(const float *__restrict__ pa
 
 template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_decode_kernel(const __grid_constant__ CUtensorMap kmap,
-                         const __grid_constant__ CUtensorMap vmap,
+    sparse_decode_kernel(const uint8_t *__restrict__ k_cache, const uint8_t *__restrict__ v_cache,
                          const int32_t *__restrict__ page_table,
                          const int32_t *__restrict__ seq_len, const uint16_t *__restrict__ q,
                          const int32_t *__restrict__ block_idx,
@@ -229,7 +276,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    __shared__ uint64_t bars[kWarps][kStages];
     __shared__ uint64_t merge_bar;
     __shared__ int2 meta[kMaxBlocksPerSplit];  // (page, valid tokens) of the slice's blocks
     __shared__ uint32_t sh_last;
@@ -244,8 +290,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_launch_next();
     const int L = seq_len[b];
     if (threadIdx.x == 0) {
-        for (int w = 0; w < kWarps; ++w)
-            for (int s = 0; s < kStages; ++s) mbar_init(&bars[w][s], 1);
         mbar_init(&merge_bar, 1);
         fence_mbar_init();
     }
@@ -296,50 +340,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    // This warp's blocks: slice entries warp + kWarps * t.
+    // This warp's blocks: slice entries warp + kWarps * t.  Block t goes to
+    // ring slot t % kStages: its K and V tiles (16 x D bf16 each, contiguous
+    // in the cache) are copied with 16-byte cp.async, lane chunk q to the
+    // 128-byte-swizzled position of (row q / 8, chunk q % 8), one copy group
+    // per block (empty groups keep the count uniform).
     const int n_mine = warp < nslice ? (nslice - warp + kWarps - 1) / kWarps : 0;
     uint8_t *ring = smem + (size_t)warp * kStages * SM::kStageBytes;
-    auto issue = [&](int t) {  // lane 0
-        const int2 mt = meta[warp + kWarps * t];
-        uint64_t *bar = &bars[warp][t % kStages];
-        if (mt.y > 0) {
-            uint8_t *st = ring + (size_t)(t % kStages) * SM::kStageBytes;
-            const int row = (mt.x * hkv + h) * kBlock;
-            mbar_arrive_expect_tx(bar, SM::kStageBytes);
-            tma_load_3d(st, &kmap, 0, 0, row, bar);
-            tma_load_3d(st + SM::kTileBytes, &vmap, 0, 0, row, bar);
-        } else {
-            mbar_arrive(bar);  // skipped block: complete the phase without data
+    constexpr int kPerLane = SM::kTileBytes / 16 / 32;
+    auto issue = [&](int t) {
+        if (t < n_mine) {
+            const int2 mt = meta[warp + kWarps * t];
+            if (mt.y > 0) {
+                const size_t tile = ((size_t)mt.x * hkv + h) * SM::kTileBytes;
+                uint8_t *st = ring + (size_t)(t % kStages) * SM::kStageBytes;
+#pragma unroll
+                for (int k = 0; k < kPerLane; ++k) {
+                    const uint32_t qc = lane + 32 * k;
+                    const uint32_t so = swz128(qc >> 3, qc & 7);
+                    cp_async16(st + so, k_cache + tile + qc * 16);
+                    cp_async16(st + SM::kTileBytes + so, v_cache + tile + qc * 16);
+                }
+            }
         }
+        cp_async_commit();
     };
-    if (lane == 0)
-        for (int t = 0; t < n_mine && t < kStages; ++t) issue(t);
+#pragma unroll
+    for (int t = 0; t < kStages - 1; ++t) issue(t);
 
     WarpState<D, NT> st;
     st.init();
-    bool ok = true;
-    int t_done = 0;
     for (int t = 0; t < n_mine; ++t) {
-        const int stage = t % kStages;
-        if (!mbar_wait_bounded(&bars[warp][stage], (t / kStages) & 1)) {
-            ok = false;
-            break;
-        }
+        issue(t + kStages - 1);  // refills the slot of block t - 1
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
         const int ntok = meta[warp + kWarps * t].y;
         if (ntok > 0) {
-            const uint32_t ks = smem_u32(ring + (size_t)stage * SM::kStageBytes);
+            const uint32_t ks = smem_u32(ring + (size_t)(t % kStages) * SM::kStageBytes);
             attend_block_swapped<D, NT>(st, qb, ks, ks + SM::kTileBytes, ntok, scale_log2, lane);
         }
-        t_done = t + 1;
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && t + kStages < n_mine) issue(t + kStages);
     }
-    if (!ok) {
-        if (lane == 0) set_error(err, RESA_DEVERR_TIMEOUT);
-        for (int t = t_done; t < n_mine && t < t_done + kStages; ++t)
-            mbar_wait_bounded(&bars[warp][t % kStages], (t / kStages) & 1);
-    }
+    cp_async_wait<0>();
     // Row sums over the eight lanes that share each head.
 #pragma unroll
     for (int n = 0; n < NT; ++n)
@@ -350,6 +392,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             st.l[n][k] += __shfl_xor_sync(0xffffffffu, st.l[n][k], 16);
         }
     __syncthreads();  // every ring is drained: reuse it for the merge
+
+    if (grid_bar != nullptr) {
+        // Spread mode (the grid is one wave, S >= 2): each warp's partial goes
+        // straight to global memory; after a bounded grid barrier every CTA
+        // merges a share of the outputs over all S * kWarps warp partials.
+        const int P = S * kWarps;
+        const size_t pidx = unit * P + (size_t)split * kWarps + warp;
+        float *pw = part_o + pidx * kMaxGroup * D;
+        float2 *pml = reinterpret_cast<float2 *>(part_lse) + pidx * kMaxGroup;
+        const int hb = 2 * (lane & 3), d0 = lane >> 2;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int h0 = n * 8 + hb;
+            if (lane < 4) {
+                if (h0 < g) pml[h0] = make_float2(st.m[n][0], st.l[n][0]);
+                if (h0 + 1 < g) pml[h0 + 1] = make_float2(st.m[n][1], st.l[n][1]);
+            }
+#pragma unroll
+            for (int t = 0; t < D / 16; ++t) {
+                float *o0 = pw + (size_t)h0 * D + t * 16 + d0;
+                if (h0 < g) {
+                    o0[0] = st.o[t][n][0];
+                    o0[8] = st.o[t][n][2];
+                }
+                if (h0 + 1 < g) {
+                    o0[D] = st.o[t][n][1];
+                    o0[D + 8] = st.o[t][n][3];
+                }
+            }
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            sh_last = grid_barrier_bounded(reinterpret_cast<unsigned long long *>(grid_bar), gridDim.x * gridDim.y * gridDim.z) ? 1u : 0u;
+        __syncthreads();
+        if (!sh_last) {
+            if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+            return;
+        }
+        __threadfence();
+        merge_warp_partials<D>(part_o, reinterpret_cast<const float2 *>(part_lse), P, hkv, g, out,
+                               lse_out, reinterpret_cast<float *>(smem));
+        return;
+    }
 
     float *mw = reinterpret_cast<float *>(smem);  // [kWarps][16]
     float *lw = mw + kWarps * kMaxGroup;          // [kWarps][16]
@@ -406,22 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     __threadfence();
     __syncthreads();
-    if (grid_bar != nullptr) {
-        // Cooperative launch (the grid is one wave): bounded grid barrier, then
-        // every CTA merges its share of the outputs.
-        if (threadIdx.x == 0)
-            sh_last = grid_barrier_bounded(grid_bar, gridDim.x * gridDim.y * gridDim.z) ? 1u : 0u;
-        __syncthreads();
-        if (!sh_last) {
-            if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);
-            return;
-        }
-        __threadfence();
-        merge_splits_spread<D>(part_o, part_lse, S, hkv, g, out, lse_out,
-                               reinterpret_cast<float *>(smem));
-        return;
-    }
-    // Otherwise the CTA that draws the last ticket of the (sequence, head) merges.
+    // The CTA that draws the last ticket of the (sequence, head) merges.
     if (threadIdx.x == 0) {
         const uint32_t ticket = atomicAdd(&tickets[unit], 1u);
         sh_last = ticket == (uint32_t)(S - 1);
@@ -552,7 +623,7 @@ int wave_capacity(int smem) {
 }
 
 template <int D, int NT>
-cudaError_t launch_dn(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
+cudaError_t launch_dn(const Shape &s, const void *k, const void *v,
                       const int32_t *page_table, const int32_t *seq_len, const void *q,
                       const int32_t *block_idx, const int32_t *block_cnt, int max_topk, int splits,
                       float *part_o, float *part_lse, uint32_t *tickets, uint32_t *grid_bar,
@@ -566,7 +637,9 @@ cudaError_t launch_dn(const Shape &s, const CUtensorMap &kmap, const CUtensorMap
     const long long ctas = (long long)splits * s.hkv * s.batch;
     // Split merge across the grid when it fits one wave (cooperative launch);
     // otherwise by the last CTA of each (sequence, head).
-    const bool spread = grid_bar != nullptr && splits > 1 && ctas <= wave_capacity<D, NT>(smem);
+    // (kSpreadMaxCtas bounds the warp partials the caller's scratch holds.)
+    const bool spread = grid_bar != nullptr && splits > 1 && ctas <= kSpreadMaxCtas &&
+                        ctas <= wave_capacity<D, NT>(smem);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kThreads);
@@ -579,7 +652,8 @@ cudaError_t launch_dn(const Shape &s, const CUtensorMap &kmap, const CUtensorMap
     attr[1].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = spread ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, sparse_decode_kernel<D, NT>, kmap, vmap, page_table, seq_len,
+    return cudaLaunchKernelEx(&cfg, sparse_decode_kernel<D, NT>, (const uint8_t *)k,
+                              (const uint8_t *)v, page_table, seq_len,
                               (const uint16_t *)q, block_idx, block_cnt, max_topk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets,
                               spread ? grid_bar : (uint32_t *)nullptr, out, lse, err);
@@ -587,14 +661,14 @@ cudaError_t launch_dn(const Shape &s, const CUtensorMap &kmap, const CUtensorMap
 
 }  // namespace
 
-cudaError_t launch_sparse_decode(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
+cudaError_t launch_sparse_decode(const Shape &s, const void *k, const void *v,
                                  const int32_t *page_table, const int32_t *seq_len, const void *q,
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
                                  uint32_t *grid_bar, float *out, float *lse, uint32_t *err,
                                  cudaStream_t st) {
 #define RESA_DECODE_ARGS                                                                     \
-    s, kmap, vmap, page_table, seq_len, q, block_idx, block_cnt, max_topk, splits, part_o, \
+    s, k, v, page_table, seq_len, q, block_idx, block_cnt, max_topk, splits, part_o,       \
         part_lse, tickets, grid_bar, out, lse, err, st
     if (s.d == 128)
         return s.g <= 8 ? launch_dn<128, 1>(RESA_DECODE_ARGS) : launch_dn<128, 2>(RESA_DECODE_ARGS);

@@ -17,7 +17,7 @@
 namespace resa {
 namespace {
 
-constexpr size_t kScratchBytes = size_t(8) << 20;  // 8 MiB per device
+constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB per device
 constexpr int kScratchMaxUnits = 4096;             // batch * Hkv
 constexpr size_t kScratchHeader = 256;  // error word; grid barrier at kDecBarrierOffset
 
@@ -42,34 +42,6 @@ resa_status_t scratch_address(void **out) {
     }
     *out = g_scratch_addr[dev];
     return RESA_OK;
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// Same K/V tensor-map geometry as the workspace path: one (page, head) block
-// of 16 x d per box, 128-byte swizzled.
-bool kv_map(CUtensorMap *map, void *base, int num_pages, int hkv, int d) {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return false;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    const cuuint64_t dims[3] = {64, (cuuint64_t)(d / 64), (cuuint64_t)num_pages * hkv * kBlock};
-    const cuuint64_t strides[2] = {128, (cuuint64_t)d * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)(d / 64), (cuuint32_t)kBlock};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
 }
 
 bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -109,8 +81,16 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     const int d = cfg->head_dim;
     const int splits = decode_splits_for(units, max_topk + 1);
     const size_t tickets_bytes = align_up((size_t)units * 4, 256);
-    const size_t lse_bytes = align_up((size_t)units * splits * kMaxGroup * 4, 256);
-    const size_t o_bytes = (size_t)units * splits * kMaxGroup * d * 4;
+    // Per-warp partials for a grid-wide merge when they fit the array, else
+    // per-split partials and the last-CTA merge.
+    const size_t spread_parts = (size_t)units * splits * kDecodeWarps;
+    const bool spread_fits = kScratchHeader + tickets_bytes +
+                                 align_up(spread_parts * kMaxGroup * 8, 256) +
+                                 spread_parts * kMaxGroup * d * 4 <=
+                             kScratchBytes;
+    const size_t parts = spread_fits ? spread_parts : (size_t)units * splits;
+    const size_t lse_bytes = align_up(parts * kMaxGroup * 8, 256);
+    const size_t o_bytes = parts * kMaxGroup * d * 4;
     if (kScratchHeader + tickets_bytes + lse_bytes + o_bytes > kScratchBytes) return RESA_ERR_SHAPE;
 
     void *base = nullptr;
@@ -126,10 +106,6 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     if (cudaMemsetAsync(scratch, 0, kScratchHeader + tickets_bytes, stream) != cudaSuccess)
         return RESA_ERR_CUDA;
 
-    CUtensorMap kmap, vmap;
-    if (!kv_map(&kmap, cache->k, cache->num_pages, hkv, d) ||
-        !kv_map(&vmap, cache->v, cache->num_pages, hkv, d))
-        return RESA_ERR_CUDA;
     Shape s{};
     s.hq = cfg->num_q_heads;
     s.hkv = hkv;
@@ -141,9 +117,10 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     s.max_pages = cache->max_pages;
     s.num_pages = cache->num_pages;
     const cudaError_t e = launch_sparse_decode(
-        s, kmap, vmap, cache->page_table, cache->seq_len, q, block_idx, block_cnt, max_topk,
+        s, cache->k, cache->v, cache->page_table, cache->seq_len, q, block_idx, block_cnt, max_topk,
         splits, part_o, part_lse, tickets,
-        reinterpret_cast<uint32_t *>(scratch + kDecBarrierOffset), out, lse_opt,
+        spread_fits ? reinterpret_cast<uint32_t *>(scratch + kDecBarrierOffset) : nullptr, out,
+        lse_opt,
         dev_error_opt ? dev_error_opt : err, stream);
     return e == cudaSuccess ? RESA_OK : RESA_ERR_CUDA;
 }

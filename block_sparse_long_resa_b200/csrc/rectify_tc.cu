@@ -438,12 +438,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Every CTA of the (cooperatively launched, co-resident) grid has written
     // its partials: bounded grid barrier, then each CTA merges its share of
-    // all rows.  tickets[0] counts arrivals, tickets[1] is the generation.
+    // all rows.  tickets[0..1] hold the barrier's 64-bit (generation, arrivals) word.
     __threadfence();
     __syncthreads();
     __shared__ uint32_t sh_ok;
     const uint32_t nctas = gridDim.x * gridDim.y * gridDim.z;
-    if (threadIdx.x == 0) sh_ok = grid_barrier_bounded(tickets, nctas) ? 1u : 0u;
+    if (threadIdx.x == 0) sh_ok = grid_barrier_bounded(reinterpret_cast<unsigned long long *>(tickets), nctas) ? 1u : 0u;
     __syncthreads();
     if (!sh_ok) {
         if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);

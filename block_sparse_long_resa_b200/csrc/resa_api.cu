@@ -26,22 +26,6 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// K or V cache [num_pages][Hkv][16][d] bf16 seen as a 3-D tensor
-// (64 channels, d/64 channel halves, num_pages*Hkv*16 token rows); one box is
-// one (page, head) block of 16 x d, landing 128-byte swizzled in shared memory.
-bool make_kv_map(CUtensorMap *map, void *base, int num_pages, int hkv, int d) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {64, (cuuint64_t)(d / 64), (cuuint64_t)num_pages * hkv * kBlock};
-    const cuuint64_t strides[2] = {128, (cuuint64_t)d * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)(d / 64), (cuuint32_t)kBlock};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // One channel half (64 columns) of a K or V cache as a 2-D tensor: rows are
 // tokens of every (page, head) block (row stride d*2 bytes); one box is the
 // 16 rows x 64 channels of one block, 128-byte swizzled.
@@ -145,15 +129,11 @@ resa_status_t select_impl(const Shape &s, const resa_cache_t *c, const WsLayout 
 resa_status_t decode_impl(const Shape &s, const resa_cache_t *c, const WsLayout &w, void *ws,
                           const void *q, const int32_t *idx, const int32_t *cnt, int max_topk,
                           float *out, float *lse, cudaStream_t st) {
-    CUtensorMap kmap, vmap;
-    if (!make_kv_map(&kmap, c->k, s.num_pages, s.hkv, s.d) ||
-        !make_kv_map(&vmap, c->v, s.num_pages, s.hkv, s.d))
-        return RESA_ERR_CUDA;
     const int splits = decode_splits_for(s.batch * s.hkv, max_topk + 1);
     if (splits > w.dec_splits) return RESA_ERR_RANGE;  // max_topk far above max_pages
     if (splits > kMaxDecodeSplits) return RESA_ERR_RANGE;
     return cuda_status(launch_sparse_decode(
-        s, kmap, vmap, c->page_table, c->seq_len, q, idx, cnt, max_topk, splits,
+        s, c->k, c->v, c->page_table, c->seq_len, q, idx, cnt, max_topk, splits,
         at<float>(ws, w.dec_o), at<float>(ws, w.dec_lse), at<uint32_t>(ws, w.dec_ticket),
         at<uint32_t>(ws, w.err + kDecBarrierOffset), out, lse, at<uint32_t>(ws, w.err), st));
 }

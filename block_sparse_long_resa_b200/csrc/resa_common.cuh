@@ -37,6 +37,15 @@ inline int decode_splits_for(int units, int max_blocks) {
     s = s > need ? s : need;
     return s < 1 ? 1 : s;
 }
+// Decode grids of at most this many CTAs may merge their splits across the
+// grid from per-warp partials (8 warps per CTA): the scratch for partials
+// holds max(units * splits, kSpreadMaxCtas * 8) of them.
+constexpr int kSpreadMaxCtas = kNumSms;
+constexpr int kDecodeWarps = 8;
+inline size_t decode_partials(int units, int splits) {
+    const size_t a = (size_t)units * splits, b = (size_t)kSpreadMaxCtas * kDecodeWarps;
+    return a > b ? a : b;
+}
 // Partial-result capacity of the workspace: enough for any top-k up to max_pages.
 inline int decode_max_splits(int batch, int hkv, int max_pages) {
     const int units = batch * hkv;
@@ -65,7 +74,7 @@ inline int rect_splits_for(int batch, int hkv, int groups) {
 constexpr int kMaxRowTiles = 64;  // rectification row groups per (sequence, kv head)
 
 // Byte offset, inside the 256-byte error header of the workspace, of the
-// decode kernel's grid barrier (arrival count, generation).
+// decode kernel's grid barrier word (64-bit: generation, arrivals).
 constexpr size_t kDecBarrierOffset = 32;
 
 struct WsLayout {
@@ -77,8 +86,8 @@ struct WsLayout {
     size_t scores;       // f32 [B][Hkv][max_pages]
     size_t sel_idx;      // i32 [B][Hkv][max_pages + 1]
     size_t sel_cnt;      // i32 [B][Hkv]
-    size_t dec_o;        // f32 [B][Hkv][dec_splits][kMaxGroup][d]
-    size_t dec_lse;      // f32 [B][Hkv][dec_splits][kMaxGroup]
+    size_t dec_o;        // f32 [partials][kMaxGroup][d]: per split, or per warp when spread
+    size_t dec_lse;      // f32 [partials][kMaxGroup] lse, or float2 (row max, row sum) when spread
     size_t rect_o;       // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta][d]
     size_t rect_lse;     // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta]
     size_t total;
@@ -111,8 +120,9 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     w.scores = take(units * max_pages * 4);
     w.sel_idx = take(units * (max_pages + 1) * 4);
     w.sel_cnt = take(units * 4);
-    w.dec_o = take(units * w.dec_splits * kMaxGroup * d * 4);
-    w.dec_lse = take(units * w.dec_splits * kMaxGroup * 4);
+    const size_t parts = decode_partials((int)units, w.dec_splits);
+    w.dec_o = take(parts * kMaxGroup * d * 4);
+    w.dec_lse = take(parts * kMaxGroup * 2 * 4);  // (lse) or (row max, row sum) pairs
     size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerCta;
     w.rect_o = take(rect_rows * d * 4);
     w.rect_lse = take(rect_rows * 4);
@@ -128,23 +138,23 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
 }
 
 // Bounded grid barrier of a cooperatively launched (co-resident) grid; thread
-// 0 of every CTA calls it after a __threadfence and a __syncthreads.  bar[0]
-// counts arrivals, bar[1] is the generation.  False when the wait gave up
-// (the count is then left non-zero: the workspace must be re-initialised).
-__device__ __forceinline__ bool grid_barrier_bounded(uint32_t *bar, uint32_t nctas) {
-    volatile uint32_t *gen_p = bar + 1;
-    const uint32_t gen = *gen_p;
-    __threadfence();
-    const uint32_t ticket = atomicAdd(&bar[0], 1u);
-    if (ticket == nctas - 1) {
-        bar[0] = 0;
-        __threadfence();
-        atomicAdd(&bar[1], 1u);
+// 0 of every CTA calls it after a __threadfence and a __syncthreads.  One
+// 64-bit word holds (generation << 32) | arrivals: each CTA adds 1; the last
+// arriver's single add of 2^32 - nctas returns the count to zero and bumps
+// the generation, which the others poll for.  The count is zero between
+// barriers, so grids of different sizes may share the word.  False when the
+// wait gave up (the word is then left mid-barrier: the workspace must be
+// re-initialised).
+__device__ __forceinline__ bool grid_barrier_bounded(unsigned long long *bar, uint32_t nctas) {
+    const unsigned long long old = atomicAdd(bar, 1ull);
+    const uint32_t gen = (uint32_t)(old >> 32);
+    if ((uint32_t)old == nctas - 1) {
+        atomicAdd(bar, (1ull << 32) - nctas);
         return true;
     }
-    for (uint32_t polls = 0; *gen_p == gen;) {
-        if (++polls > (1u << 24)) return false;
-        __nanosleep(32);
+    volatile unsigned long long *vp = bar;
+    for (uint32_t polls = 0; (uint32_t)(*vp >> 32) == gen;) {
+        if (++polls > (1u << 22)) return false;  // each poll is an L2 round trip
     }
     return true;
 }
@@ -207,6 +217,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// 16-byte asynchronous copy global -> shared through the load/store path
+// (cp.async), grouped per thread with commit_group / wait_group.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // TMA: 3-D tiled bulk tensor load into shared memory, completion on an mbarrier.
@@ -341,7 +363,7 @@ cudaError_t launch_select(const Shape &s, const float *scores, uint32_t *hist,
                           uint32_t *hist_range, const int32_t *seq_len, const int32_t *topk,
                           int max_topk, int32_t *block_idx, int32_t *block_cnt, uint32_t *err,
                           cudaStream_t st);
-cudaError_t launch_sparse_decode(const Shape &s, const CUtensorMap &kmap, const CUtensorMap &vmap,
+cudaError_t launch_sparse_decode(const Shape &s, const void *k, const void *v,
                                  const int32_t *page_table, const int32_t *seq_len, const void *q,
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,

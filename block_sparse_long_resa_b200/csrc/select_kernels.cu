@@ -54,16 +54,6 @@ struct ScoreCfg {
     static_assert(kRing >= 2, "at least two pages in flight per warp");
 };
 
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ uint32_t order_key(float s) {
     s += 0.0f;  // -0 -> +0: equal scores get equal keys
     const uint32_t u = __float_as_uint(s);

@@ -189,12 +189,13 @@ RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cac
  * at start-up, or a plugin interface that forbids device allocations after
  * initialisation, and so cannot provide a workspace.
  *   - Takes the arguments of resa_sparse_decode minus the workspace; the
- *     decode scratch (split partials, split tickets, error word) lives in a
- *     fixed 8 MiB device array inside the library, held by every GPU that
- *     loads it until the process exits.  Nothing is allocated or freed.
- *   - Limit: batch * Hkv <= 4096 and batch * Hkv * splits * 16 * (d + 1) * 4
- *     bytes of partials must fit the array (about 8 MiB); larger calls return
- *     RESA_ERR_SHAPE.  Splits are chosen as in resa_sparse_decode.
+ *     decode scratch (split or warp partials, split tickets, grid barrier,
+ *     error word) lives in a fixed 16 MiB device array inside the library,
+ *     held by every GPU that loads it until the process exits.  Nothing is
+ *     allocated or freed.
+ *   - Limit: batch * Hkv <= 4096 and batch * Hkv * splits * 16 * (d + 2) * 4
+ *     bytes of partials must fit the array (about 16 MiB); larger calls
+ *     return RESA_ERR_SHAPE.  Splits are chosen as in resa_sparse_decode.
  *   - The first call on each device looks up the array's device address
  *     (a runtime query, done once per device with that device current); make
  *     that first call before any stream capture.
