@@ -324,6 +324,26 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+def decode_dram_traffic():
+    """DRAM bytes per launch of the decode kernel from the committed ncu record,
+    or None when the kernel's sources changed since the counters were taken."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    path = os.path.join(here, "profiles", "sparse_decode_dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(here, src), "rb") as f:
+                h.update(f.read())
+    except (OSError, KeyError, ValueError):
+        return None, None
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None, "kernel changed since profiles/sparse_decode_dram_traffic.json"
+    return int(rec["dram_bytes_per_launch"]), "profiles/sparse_decode_dram_traffic.json (ncu, layer256k)"
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -520,9 +540,10 @@ def run_resa(args):
     last_dec_L = w.sched.decode_L(cycles - 1, wl["f"] - 2)
     dec_bytes = w.decode_kernel_bytes(last_dec_L)
     dec_gbs = dec_bytes / (bd["sparse_decode_us"] * 1e-6) / 1e9
+    traffic, traffic_src = decode_dram_traffic()
     roofline = {"kernel": "sparse_decode_kernel (resa_sparse_decode)", "bound": "hbm",
                 "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": dec_gbs / hbm_peak, "traffic": None,
+                "frac": dec_gbs / hbm_peak, "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes_per_launch": dec_bytes,
                 "launch_us": bd["sparse_decode_us"], "peak_source": peak_src}
     # whole-step roofline: algorithmic bytes of every kernel in the cycle
