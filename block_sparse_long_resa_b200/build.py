@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libresa.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 SOURCES = ["resa_api.cu", "desc_kernels.cu", "select_kernels.cu", "decode_kernel.cu",
-           "rectify_tc.cu", "decode_noalloc.cu"]
+           "rectify_tc.cu", "decode_noalloc.cu", "step_kernel.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
               "-Xcompiler", "-fvisibility=hidden"]

@@ -11,36 +11,6 @@
 namespace resa {
 namespace {
 
-struct Bf16x8 {
-    uint16_t v[8];
-};
-
-__device__ __forceinline__ Bf16x8 unpack(uint4 x) {
-    Bf16x8 r;
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        r.v[2 * i] = (uint16_t)(w[i] & 0xffffu);
-        r.v[2 * i + 1] = (uint16_t)(w[i] >> 16);
-    }
-    return r;
-}
-__device__ __forceinline__ uint4 pack(const Bf16x8 &r) {
-    uint4 x;
-    x.x = (uint32_t)r.v[0] | ((uint32_t)r.v[1] << 16);
-    x.y = (uint32_t)r.v[2] | ((uint32_t)r.v[3] << 16);
-    x.z = (uint32_t)r.v[4] | ((uint32_t)r.v[5] << 16);
-    x.w = (uint32_t)r.v[6] | ((uint32_t)r.v[7] << 16);
-    return x;
-}
-__device__ __forceinline__ void fold(Bf16x8 &mn, Bf16x8 &mx, const Bf16x8 &x) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        mn.v[i] = bf_min(mn.v[i], x.v[i]);
-        mx.v[i] = bf_max(mx.v[i], x.v[i]);
-    }
-}
-
 __device__ __forceinline__ size_t kv_off(int page, int h, int slot, int c, int hkv, int d) {
     return ((((size_t)page * hkv + h) * kBlock + slot) * d) / 8 + c;  // in uint4 units
 }
@@ -81,10 +51,10 @@ __global__ void append_kernel(uint4 *__restrict__ K, uint4 *__restrict__ V,
         *pmn = kx;
         *pmx = kx;
     } else {
-        Bf16x8 mn = unpack(*pmn), mx = unpack(*pmx);
-        fold(mn, mx, unpack(kx));
-        *pmn = pack(mn);
-        *pmx = pack(mx);
+        Bf16x8 mn = unpack8(*pmn), mx = unpack8(*pmx);
+        fold8(mn, mx, unpack8(kx));
+        *pmn = pack8(mn);
+        *pmx = pack8(mx);
     }
 }
 
@@ -125,12 +95,12 @@ __global__ void __launch_bounds__(kBuildThreads)
 #pragma unroll
         for (int t = 0; t < kBlock; ++t)
             if (t < nt) x[t] = K[kv_off(page, h, t, c, hkv, d)];
-        Bf16x8 mn = unpack(x[0]), mx = mn;
+        Bf16x8 mn = unpack8(x[0]), mx = mn;
 #pragma unroll
         for (int t = 1; t < kBlock; ++t)
-            if (t < nt) fold(mn, mx, unpack(x[t]));
-        desc[desc_off(page, h, 0, c, hkv, d)] = pack(mn);
-        desc[desc_off(page, h, 1, c, hkv, d)] = pack(mx);
+            if (t < nt) fold8(mn, mx, unpack8(x[t]));
+        desc[desc_off(page, h, 0, c, hkv, d)] = pack8(mn);
+        desc[desc_off(page, h, 1, c, hkv, d)] = pack8(mx);
     }
 }
 
@@ -182,7 +152,7 @@ __global__ void rectify_writeback_kernel(uint4 *__restrict__ K, uint4 *__restric
             }
         }
     }
-    Bf16x8 mn = unpack(kx[0]), mx = mn;
+    Bf16x8 mn = unpack8(kx[0]), mx = mn;
 #pragma unroll
     for (int t = 0; t < kBlock; ++t) {
         const int pos = blk * kBlock + t;
@@ -191,10 +161,10 @@ __global__ void rectify_writeback_kernel(uint4 *__restrict__ K, uint4 *__restric
             K[o] = kx[t];
             V[o] = vx[t];
         }
-        if (t > 0 && t < nt) fold(mn, mx, unpack(kx[t]));
+        if (t > 0 && t < nt) fold8(mn, mx, unpack8(kx[t]));
     }
-    desc[desc_off(page, h, 0, c, hkv, d)] = pack(mn);
-    desc[desc_off(page, h, 1, c, hkv, d)] = pack(mx);
+    desc[desc_off(page, h, 0, c, hkv, d)] = pack8(mn);
+    desc[desc_off(page, h, 1, c, hkv, d)] = pack8(mx);
 }
 
 }  // namespace

@@ -126,6 +126,25 @@ resa_status_t select_impl(const Shape &s, const resa_cache_t *c, const WsLayout 
     return RESA_OK;
 }
 
+int sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    int c = cache[dev].load();
+    if (c == 0) {
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev].store(c);
+    }
+    return c;
+}
+
+// CTAs per (sequence, kv head) of the fused decode step for this shape, 0 when
+// the step runs as three launches (score + append, select, decode).
+int fused_step_ctas(const Shape &s) {
+    if ((long long)s.num_pages >= (1LL << 27)) return 0;  // packed (page, tokens) work items
+    return step_ctas_per_unit(s.batch * s.hkv, s.g, s.max_pages, sm_count());
+}
+
 resa_status_t decode_impl(const Shape &s, const resa_cache_t *c, const WsLayout &w, void *ws,
                           const void *q, const int32_t *idx, const int32_t *cnt, int max_topk,
                           float *out, float *lse, cudaStream_t st) {
@@ -294,11 +313,42 @@ resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cac
     RESA_TRY(check_ws(ws, ws_bytes, w));
     int32_t *idx = block_idx_opt && block_cnt_opt ? block_idx_opt : at<int32_t>(ws, w.sel_idx);
     int32_t *cnt = block_idx_opt && block_cnt_opt ? block_cnt_opt : at<int32_t>(ws, w.sel_cnt);
+    const int G = fused_step_ctas(s);
+    if (G > 0) {
+        StepBuffers buf;
+        buf.block_idx = idx;
+        buf.block_cnt = cnt;
+        buf.hist = at<uint32_t>(ws, w.hist);
+        buf.hist_range = at<uint32_t>(ws, w.hist_range);
+        buf.bars = at<unsigned long long>(ws, w.step_bars);
+        buf.tickets = at<uint32_t>(ws, w.dec_ticket);
+        buf.counts = at<int2>(ws, w.step_counts);
+        buf.ovf = at<int32_t>(ws, w.step_ovf);
+        buf.cand = at<uint32_t>(ws, w.step_cand);
+        buf.part_o = at<float>(ws, w.dec_o);
+        buf.part_lse = at<float>(ws, w.dec_lse);
+        buf.err = at<uint32_t>(ws, w.err);
+        return cuda_status(launch_decode_step_fused(s, G, cache->k, cache->v, cache->desc,
+                                                    cache->page_table, cache->seq_len, q, k_new,
+                                                    v_new, topk, max_topk, out, lse_opt, buf,
+                                                    stream));
+    }
     // append + scores in one launch (the append touches only the current
     // block, which is never scored), then select, then attend
     RESA_TRY(select_impl(s, cache, w, ws, q, topk, max_topk, idx, cnt, at<float>(ws, w.scores),
                          k_new, v_new, stream));
     return decode_impl(s, cache, w, ws, q, idx, cnt, max_topk, out, lse_opt, stream);
+}
+
+int32_t resa_decode_step_launches(const resa_config_t *cfg, int32_t batch, int32_t max_pages,
+                                  int32_t num_pages) {
+    Shape s{};
+    if (check_config(cfg, &s) != RESA_OK || batch <= 0 || max_pages <= 0 || num_pages <= 0)
+        return -1;
+    s.batch = batch;
+    s.max_pages = max_pages;
+    s.num_pages = num_pages;
+    return fused_step_ctas(s) > 0 ? 1 : 3;
 }
 
 int32_t resa_kernels_per_call(const char *entry_point) {
@@ -308,7 +358,7 @@ int32_t resa_kernels_per_call(const char *entry_point) {
         int n;
     } table[] = {{"resa_build_descriptors", 1}, {"resa_append_token", 1},
                  {"resa_select_blocks", 2},     {"resa_sparse_decode", 1},
-                 {"resa_rectify_attention", 2}, {"resa_decode_step", 3},
+                 {"resa_rectify_attention", 2}, {"resa_decode_step", 1},
                  {"resa_sparse_decode_noalloc", 1}};
     for (auto &e : table)
         if (strcmp(e.name, entry_point) == 0) return e.n;

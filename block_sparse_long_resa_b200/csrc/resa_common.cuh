@@ -53,6 +53,28 @@ inline int decode_max_splits(int batch, int hkv, int max_pages) {
     const int want = (kNumSms + units - 1) / units;
     return want > need ? want : need;
 }
+// Fused decode step (one persistent launch per step): G CTAs per (sequence,
+// kv head) unit, G * units <= kNumSms; a CTA scores at most kStepMaxBlocks
+// complete blocks; a unit resolves up to kStepCandCap boundary candidates in
+// shared memory (more are read from the workspace); block ids must fit 16
+// bits (composite selection keys), so max_pages <= 65536.
+constexpr int kStepMaxBlocks = 1024;
+constexpr int kStepCandCap = 2048;
+constexpr int kStepMaxPages = 65536;
+constexpr int kStepMaxGroup = 8;  // one n8 MMA tile of query heads (register budget)
+// CTAs per unit of the fused step, or 0 when the shape needs the unfused path.
+inline int step_ctas_per_unit(int units, int g, int max_pages, int sms) {
+    if (g > kStepMaxGroup || max_pages > kStepMaxPages || units <= 0) return 0;
+    const int cap = sms < kNumSms ? sms : kNumSms;
+    const int by_sm = cap / units;
+    const int by_work = (max_pages + 63) / 64;  // about 64 blocks per CTA at least
+    int G = by_sm < by_work ? by_sm : by_work;
+    if (G < 2) G = by_sm >= 2 ? 2 : G;
+    if (G < 2) return 0;
+    if ((max_pages + G - 1) / G > kStepMaxBlocks) return 0;
+    return G;
+}
+
 constexpr int kRectRowsPerCta = 256;  // query rows (chunk position x group head) per CTA
 inline int rect_row_groups(int chunk, int group) {
     const int rows = chunk * group;
@@ -88,6 +110,10 @@ struct WsLayout {
     size_t sel_cnt;      // i32 [B][Hkv]
     size_t dec_o;        // f32 [partials][kMaxGroup][d]: per split, or per warp when spread
     size_t dec_lse;      // f32 [partials][kMaxGroup] lse, or float2 (row max, row sum) when spread
+    size_t step_bars;    // u64 [B][Hkv][2] unit barriers of the fused step (zero between calls)
+    size_t step_counts;  // int2 [kNumSms] per-CTA (definite, candidate) counts
+    size_t step_ovf;     // i32 [kNumSms][kStepMaxBlocks] definite blocks beyond a CTA's share
+    size_t step_cand;    // u32 [kNumSms][kStepMaxBlocks] boundary candidates (composite keys)
     size_t rect_o;       // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta][d]
     size_t rect_lse;     // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta]
     size_t total;
@@ -123,6 +149,10 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     const size_t parts = decode_partials((int)units, w.dec_splits);
     w.dec_o = take(parts * kMaxGroup * d * 4);
     w.dec_lse = take(parts * kMaxGroup * 2 * 4);  // (lse) or (row max, row sum) pairs
+    w.step_bars = take(units * 2 * 8);
+    w.step_counts = take((size_t)kNumSms * 8);
+    w.step_ovf = take((size_t)kNumSms * kStepMaxBlocks * 4);
+    w.step_cand = take((size_t)kNumSms * kStepMaxBlocks * 4);
     size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerCta;
     w.rect_o = take(rect_rows * d * 4);
     w.rect_lse = take(rect_rows * 4);
@@ -171,6 +201,55 @@ __device__ __forceinline__ uint16_t bf_min(uint16_t cur, uint16_t x) {
 }
 __device__ __forceinline__ uint16_t bf_max(uint16_t cur, uint16_t x) {
     return bf16_bits_to_f32(x) > bf16_bits_to_f32(cur) ? x : cur;
+}
+
+// Eight bf16 channels (one 16-byte vector) as raw bit patterns.
+struct Bf16x8 {
+    uint16_t v[8];
+};
+__device__ __forceinline__ Bf16x8 unpack8(uint4 x) {
+    Bf16x8 r;
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        r.v[2 * i] = (uint16_t)(w[i] & 0xffffu);
+        r.v[2 * i + 1] = (uint16_t)(w[i] >> 16);
+    }
+    return r;
+}
+__device__ __forceinline__ uint4 pack8(const Bf16x8 &r) {
+    uint4 x;
+    x.x = (uint32_t)r.v[0] | ((uint32_t)r.v[1] << 16);
+    x.y = (uint32_t)r.v[2] | ((uint32_t)r.v[3] << 16);
+    x.z = (uint32_t)r.v[4] | ((uint32_t)r.v[5] << 16);
+    x.w = (uint32_t)r.v[6] | ((uint32_t)r.v[7] << 16);
+    return x;
+}
+// Fold x into a running element-wise (min, max) pair (Eq. 3).
+__device__ __forceinline__ void fold8(Bf16x8 &mn, Bf16x8 &mx, const Bf16x8 &x) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        mn.v[i] = bf_min(mn.v[i], x.v[i]);
+        mx.v[i] = bf_max(mx.v[i], x.v[i]);
+    }
+}
+
+// Block scores as unsigned keys with the same order as the fp32 values
+// (-0 and +0 map to one key, so equal scores get equal keys).
+constexpr int kHistBins = 65536;  // histogram of the top 16 key bits
+__device__ __forceinline__ uint32_t order_key(float s) {
+    s += 0.0f;
+    const uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Byte-permute selector taking, for the two bf16 channels of a 32-bit word,
+// the max half (from the second operand) where q >= 0 and the min half
+// (first operand) otherwise: q * that value is max(q * max, q * min), the
+// per-channel term of Eq. 4.
+__device__ __forceinline__ uint32_t upper_bound_selector(float q0, float q1) {
+    const uint32_t b0 = q0 >= 0.f ? 4u : 0u, b1 = q1 >= 0.f ? 4u : 0u;
+    return (b0 + 0u) | ((b0 + 1u) << 4) | ((b1 + 2u) << 8) | ((b1 + 3u) << 12);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -369,6 +448,24 @@ cudaError_t launch_sparse_decode(const Shape &s, const void *k, const void *v,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
                                  uint32_t *grid_bar, float *out, float *lse, uint32_t *err,
                                  cudaStream_t st);
+// Fused decode step: append + scores + selection + sparse attention in one
+// cooperative launch of G CTAs per (sequence, kv head) (step_ctas_per_unit).
+struct StepBuffers {
+    int32_t *block_idx, *block_cnt;  // selection output [B][Hkv][max_topk+1], [B][Hkv]
+    uint32_t *hist, *hist_range;
+    unsigned long long *bars;
+    uint32_t *tickets;
+    int2 *counts;
+    int32_t *ovf;
+    uint32_t *cand;
+    float *part_o, *part_lse;
+    uint32_t *err;
+};
+cudaError_t launch_decode_step_fused(const Shape &s, int G, void *k, void *v, void *desc,
+                                     const int32_t *page_table, const int32_t *seq_len,
+                                     const void *q, const void *k_new, const void *v_new,
+                                     const int32_t *topk, int max_topk, float *out, float *lse,
+                                     const StepBuffers &buf, cudaStream_t st);
 // maps: K half 0, K half 1, V half 0, V half 1 (2-D, 16 x 64 boxes, 128-byte swizzle).
 cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap *maps,
                                      const int32_t *page_table, const int32_t *seq_len, int f,

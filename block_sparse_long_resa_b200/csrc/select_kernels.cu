@@ -40,7 +40,6 @@ namespace {
 constexpr int kScoreWarps = 16;                   // scoring warps per CTA (one CTA per SM)
 constexpr int kScoreRingBytes = 192 * 1024;       // shared-memory ring budget per CTA
 constexpr int kScoreThreads = 32 * (kScoreWarps + 1);  // + the decode-token append warp
-constexpr int kHistBins = 65536;
 constexpr int kHashSlots = 2048;  // per-CTA histogram aggregation table
 constexpr uint32_t kHashEmpty = 0xffffffffu;
 
@@ -53,42 +52,6 @@ struct ScoreCfg {
     static constexpr int kRingBytes = kScoreWarps * kRing * kPageBytes;
     static_assert(kRing >= 2, "at least two pages in flight per warp");
 };
-
-__device__ __forceinline__ uint32_t order_key(float s) {
-    s += 0.0f;  // -0 -> +0: equal scores get equal keys
-    const uint32_t u = __float_as_uint(s);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-struct Bf16x8 {
-    uint16_t v[8];
-};
-__device__ __forceinline__ Bf16x8 unpack8(uint4 x) {
-    Bf16x8 r;
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        r.v[2 * i] = (uint16_t)(w[i] & 0xffffu);
-        r.v[2 * i + 1] = (uint16_t)(w[i] >> 16);
-    }
-    return r;
-}
-__device__ __forceinline__ uint4 pack8(const Bf16x8 &r) {
-    uint4 x;
-    x.x = (uint32_t)r.v[0] | ((uint32_t)r.v[1] << 16);
-    x.y = (uint32_t)r.v[2] | ((uint32_t)r.v[3] << 16);
-    x.z = (uint32_t)r.v[4] | ((uint32_t)r.v[5] << 16);
-    x.w = (uint32_t)r.v[6] | ((uint32_t)r.v[7] << 16);
-    return x;
-}
-
-// Byte-permute selector taking, for the two bf16 channels of a 32-bit word,
-// the max half (from the second operand) where q >= 0 and the min half
-// (first operand) otherwise: q * that value is max(q * max, q * min).
-__device__ __forceinline__ uint32_t upper_bound_selector(float q0, float q1) {
-    const uint32_t b0 = q0 >= 0.f ? 4u : 0u, b1 = q1 >= 0.f ? 4u : 0u;
-    return (b0 + 0u) | ((b0 + 1u) << 4) | ((b1 + 2u) << 8) | ((b1 + 3u) << 12);
-}
 
 // grid (X, batch), block kScoreThreads, dynamic smem ScoreCfg::kRingBytes.
 template <int D, int HKV>

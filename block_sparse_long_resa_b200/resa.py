@@ -63,6 +63,7 @@ _SIGS = {
                          ctypes.c_int),
     "resa_sparse_decode_noalloc": ([_P, _P, _P, _P, _P, _I, _P, _P, _P, _P], ctypes.c_int),
     "resa_kernels_per_call": ([ctypes.c_char_p], ctypes.c_int32),
+    "resa_decode_step_launches": ([_P, _I, _I, _I], ctypes.c_int32),
     "resa_status_string": ([ctypes.c_int], ctypes.c_char_p),
 }
 
@@ -200,6 +201,11 @@ def resa_sparse_decode_noalloc(cfg, cache, q, block_idx, block_cnt, max_topk: in
 
 def resa_kernels_per_call(entry_point: str) -> int:
     return int(lib().resa_kernels_per_call(entry_point.encode()))
+
+
+def resa_decode_step_launches(cfg, batch: int, max_pages: int, num_pages: int) -> int:
+    """1 when resa_decode_step runs as one fused launch for this cache shape, else 3."""
+    return int(lib().resa_decode_step_launches(ctypes.byref(cfg), batch, max_pages, num_pages))
 
 
 def resa_status_string(status: int) -> str:

@@ -171,11 +171,18 @@ RESA_API resa_status_t resa_rectify_attention(const resa_config_t *cfg, const re
                                      size_t ws_bytes, cudaStream_t stream);
 
 /* One sparse decode step of one layer (Algorithm 1 inner body): append the
- * decode token (as resa_append_token, fused into the scoring launch), select
- * blocks (resa_select_blocks) and attend (resa_sparse_decode).  seq_len must
- * already count the decode token.
- * block_idx_opt / block_cnt_opt (nullable) receive the selection; when NULL
- * it lives in the workspace. */
+ * decode token (as resa_append_token), select blocks (as resa_select_blocks)
+ * and attend (as resa_sparse_decode).  seq_len must already count the decode
+ * token.  block_idx_opt / block_cnt_opt (nullable) receive the selection in
+ * the layout of resa_select_blocks; when NULL it lives in the workspace.
+ * When batch * Hkv <= 74, g <= 8 and max_pages <= 65536 (and each of the
+ * G = 148 / (batch * Hkv) CTAs per (sequence, kv head) scores at most 1024
+ * blocks) the whole step is one cooperative launch: the CTAs of a (sequence,
+ * kv head) score their share of the descriptors, agree on the selection
+ * through two bounded barriers in the workspace and split the selected
+ * blocks evenly; other shapes run as three launches (append fused with the
+ * scores, selection, sparse decode).  resa_decode_step_launches tells which.
+ * Both give the same selection; outputs agree to fp32 rounding. */
 RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cache,
                                const void *q, const void *k_new, const void *v_new,
                                const int32_t *topk, int32_t max_topk, float *out, float *lse_opt,
@@ -215,9 +222,16 @@ RESA_API resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
 
 /* Number of kernels each entry point launches per call (for launch
  * accounting): 1 for append and build, 2 for select, 1 for sparse decode,
- * 2 for rectify, 3 for a decode step (append fused with scoring), 1 for the
- * no-allocation decode.  Unknown names return -1. */
+ * 2 for rectify, 1 for a decode step of the fused shapes (see
+ * resa_decode_step_launches for the others), 1 for the no-allocation decode.
+ * Unknown names return -1. */
 RESA_API int32_t resa_kernels_per_call(const char *entry_point);
+
+/* Kernels resa_decode_step launches for caches of `batch` sequences of
+ * max_pages blocks over num_pages physical pages: 1 (fused step) or 3; -1 for
+ * an invalid configuration.  Reads the current device's SM count. */
+RESA_API int32_t resa_decode_step_launches(const resa_config_t *cfg, int32_t batch,
+                                           int32_t max_pages, int32_t num_pages);
 
 /* Human-readable status name. */
 RESA_API const char *resa_status_string(resa_status_t status);

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_status_strings_and_launch_table(lib):
     assert R.resa_status_string(0) == "RESA_OK"
     assert R.resa_status_string(6) == "RESA_ERR_DEVICE_CHECK"
-    assert R.resa_kernels_per_call("resa_decode_step") == 3
+    assert R.resa_kernels_per_call("resa_decode_step") == 1
     assert R.resa_kernels_per_call("resa_rectify_attention") == 2
     assert R.resa_kernels_per_call("nope") == -1
 
