@@ -240,7 +240,8 @@ class GpuWorkload:
 
     def launches_per_cycle(self):
         R = self.R
-        return self.layers * ((self.f - 1) * R.resa_kernels_per_call("resa_decode_step") +
+        step = R.resa_decode_step_launches(self.cfg, self.B, self.max_pages, self.num_pages)
+        return self.layers * ((self.f - 1) * step +
                               R.resa_kernels_per_call("resa_rectify_attention"))
 
     # algorithmic bytes / flops ---------------------------------------------
@@ -324,12 +325,12 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
-def decode_dram_traffic():
-    """DRAM bytes per launch of the decode kernel from the committed ncu record,
-    or None when the kernel's sources changed since the counters were taken."""
+def kernel_dram_traffic(record="decode_step_dram_traffic.json"):
+    """DRAM bytes per launch of a kernel from its committed ncu record, or None
+    when the kernel's sources changed since the counters were taken."""
     import hashlib
     here = os.path.dirname(os.path.abspath(__file__))
-    path = os.path.join(here, "profiles", "sparse_decode_dram_traffic.json")
+    path = os.path.join(here, "profiles", record)
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -340,8 +341,8 @@ def decode_dram_traffic():
     except (OSError, KeyError, ValueError):
         return None, None
     if h.hexdigest() != rec["sources_sha256"]:
-        return None, "kernel changed since profiles/sparse_decode_dram_traffic.json"
-    return int(rec["dram_bytes_per_launch"]), "profiles/sparse_decode_dram_traffic.json (ncu, layer256k)"
+        return None, f"kernel changed since profiles/{record}"
+    return int(rec["dram_bytes_per_launch"]), f"profiles/{record} (ncu, {rec.get('workload_short', 'layer256k')})"
 
 
 def measured_peaks():
@@ -538,14 +539,25 @@ def run_resa(args):
 
     hbm_peak, bf16_peak, bf16_sus, peak_src = measured_peaks()
     last_dec_L = w.sched.decode_L(cycles - 1, wl["f"] - 2)
-    dec_bytes = w.decode_kernel_bytes(last_dec_L)
-    dec_gbs = dec_bytes / (bd["sparse_decode_us"] * 1e-6) / 1e9
-    traffic, traffic_src = decode_dram_traffic()
-    roofline = {"kernel": "sparse_decode_kernel (resa_sparse_decode)", "bound": "hbm",
+    fused = w.R.resa_decode_step_launches(w.cfg, w.B, w.max_pages, w.num_pages) == 1
+    if fused:
+        # the fused decode step is one kernel: q + descriptors + selected K/V + output
+        dec_bytes = w.step_bytes(last_dec_L)
+        dec_us = bd["decode_step_us"]
+        traffic, traffic_src = kernel_dram_traffic("decode_step_dram_traffic.json")
+        kname = "decode_step_kernel (resa_decode_step, one launch per step)"
+    else:
+        dec_bytes = w.decode_kernel_bytes(last_dec_L)
+        dec_us = bd["sparse_decode_us"]
+        traffic, traffic_src = kernel_dram_traffic("sparse_decode_dram_traffic.json")
+        kname = "sparse_decode_kernel (resa_sparse_decode)"
+    dec_gbs = dec_bytes / (dec_us * 1e-6) / 1e9
+    roofline = {"kernel": kname, "bound": "hbm",
                 "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": dec_gbs / hbm_peak, "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes_per_launch": dec_bytes,
-                "launch_us": bd["sparse_decode_us"], "peak_source": peak_src}
+                "launch_us": dec_us, "peak_source": peak_src,
+                "peak_kind": "burst copy (MEASURED_PEAKS hbm_gbs)"}
     # whole-step roofline: algorithmic bytes of every kernel in the cycle
     cyc_bytes = 0
     for c in range(W, cycles):
@@ -584,6 +596,7 @@ def run_resa(args):
                           "peak": hbm_peak, "unit": "GB/s", "frac": step_gbs / hbm_peak},
         "rectify": rect,
         "kernel_breakdown_us": bd,
+        "decode_step_path": "fused (1 launch)" if fused else "3 launches",
         "sparse_vs_dense_step_speedup": bd["dense_decode_step_us"] / bd["decode_step_us"],
         "clocks": clk,
         "e2e": e2e,

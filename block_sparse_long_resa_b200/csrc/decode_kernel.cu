@@ -173,8 +173,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                          float *__restrict__ lse_out, uint32_t *err) {
     using SM = DecodeSmem<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    // 1024-byte aligned base, derived from the shared array itself so that
+    // accesses keep the shared address space (no generic loads)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ uint64_t merge_bar;
     __shared__ int2 meta[kMaxBlocksPerSplit];  // (page, valid tokens) of the slice's blocks
     __shared__ uint32_t sh_last;

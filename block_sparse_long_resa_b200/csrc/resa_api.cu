@@ -142,7 +142,7 @@ int sm_count() {
 // the step runs as three launches (score + append, select, decode).
 int fused_step_ctas(const Shape &s) {
     if ((long long)s.num_pages >= (1LL << 27)) return 0;  // packed (page, tokens) work items
-    return step_ctas_per_unit(s.batch * s.hkv, s.g, s.max_pages, sm_count());
+    return step_ctas_per_unit(s.batch * s.hkv, s.g, s.d, s.max_pages, sm_count());
 }
 
 resa_status_t decode_impl(const Shape &s, const resa_cache_t *c, const WsLayout &w, void *ws,
@@ -321,10 +321,7 @@ resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cac
         buf.hist = at<uint32_t>(ws, w.hist);
         buf.hist_range = at<uint32_t>(ws, w.hist_range);
         buf.bars = at<unsigned long long>(ws, w.step_bars);
-        buf.tickets = at<uint32_t>(ws, w.dec_ticket);
-        buf.counts = at<int2>(ws, w.step_counts);
-        buf.ovf = at<int32_t>(ws, w.step_ovf);
-        buf.cand = at<uint32_t>(ws, w.step_cand);
+        buf.ukeys = at<uint32_t>(ws, w.step_keys);
         buf.part_o = at<float>(ws, w.dec_o);
         buf.part_lse = at<float>(ws, w.dec_lse);
         buf.err = at<uint32_t>(ws, w.err);

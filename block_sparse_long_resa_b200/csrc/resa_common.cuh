@@ -55,16 +55,23 @@ inline int decode_max_splits(int batch, int hkv, int max_pages) {
 }
 // Fused decode step (one persistent launch per step): G CTAs per (sequence,
 // kv head) unit, G * units <= kNumSms; a CTA scores at most kStepMaxBlocks
-// complete blocks; a unit resolves up to kStepCandCap boundary candidates in
-// shared memory (more are read from the workspace); block ids must fit 16
-// bits (composite selection keys), so max_pages <= 65536.
+// complete blocks; block ids must fit 16 bits (composite selection keys), so
+// max_pages <= 65536.
 constexpr int kStepMaxBlocks = 1024;
-constexpr int kStepCandCap = 2048;
 constexpr int kStepMaxPages = 65536;
+// After scoring, every CTA of the fused step holds its unit's keys and the
+// boundary candidates (at most as many) in its K/V rings (8 warps x 3 stages
+// x a 16-token K and V tile): at most this many keys.
+constexpr int step_unit_keys(int d) {
+    return kDecodeWarps * 3 * 2 * kBlock * d * 2 / 8 - 1024 < 32768 ? kDecodeWarps * 3 * 2 * kBlock * d * 2 / 8 - 1024 : 32768;
+}
+// Row stride (in keys) of a unit's key row in the workspace: 16-byte rows.
+inline int step_key_stride(int max_pages) { return (max_pages + 3) & ~3; }
 constexpr int kStepMaxGroup = 8;  // one n8 MMA tile of query heads (register budget)
 // CTAs per unit of the fused step, or 0 when the shape needs the unfused path.
-inline int step_ctas_per_unit(int units, int g, int max_pages, int sms) {
+inline int step_ctas_per_unit(int units, int g, int d, int max_pages, int sms) {
     if (g > kStepMaxGroup || max_pages > kStepMaxPages || units <= 0) return 0;
+    if (max_pages > step_unit_keys(d)) return 0;
     const int cap = sms < kNumSms ? sms : kNumSms;
     const int by_sm = cap / units;
     const int by_work = (max_pages + 63) / 64;  // about 64 blocks per CTA at least
@@ -111,9 +118,7 @@ struct WsLayout {
     size_t dec_o;        // f32 [partials][kMaxGroup][d]: per split, or per warp when spread
     size_t dec_lse;      // f32 [partials][kMaxGroup] lse, or float2 (row max, row sum) when spread
     size_t step_bars;    // u64 [B][Hkv][2] unit barriers of the fused step (zero between calls)
-    size_t step_counts;  // int2 [kNumSms] per-CTA (definite, candidate) counts
-    size_t step_ovf;     // i32 [kNumSms][kStepMaxBlocks] definite blocks beyond a CTA's share
-    size_t step_cand;    // u32 [kNumSms][kStepMaxBlocks] boundary candidates (composite keys)
+    size_t step_keys;    // u32 [B][Hkv][step_key_stride(max_pages)] block score keys of the fused step
     size_t rect_o;       // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta][d]
     size_t rect_lse;     // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta]
     size_t total;
@@ -150,9 +155,7 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     w.dec_o = take(parts * kMaxGroup * d * 4);
     w.dec_lse = take(parts * kMaxGroup * 2 * 4);  // (lse) or (row max, row sum) pairs
     w.step_bars = take(units * 2 * 8);
-    w.step_counts = take((size_t)kNumSms * 8);
-    w.step_ovf = take((size_t)kNumSms * kStepMaxBlocks * 4);
-    w.step_cand = take((size_t)kNumSms * kStepMaxBlocks * 4);
+    w.step_keys = take(units * (size_t)step_key_stride(max_pages) * 4);
     size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerCta;
     w.rect_o = take(rect_rows * d * 4);
     w.rect_lse = take(rect_rows * 4);
@@ -454,10 +457,7 @@ struct StepBuffers {
     int32_t *block_idx, *block_cnt;  // selection output [B][Hkv][max_topk+1], [B][Hkv]
     uint32_t *hist, *hist_range;
     unsigned long long *bars;
-    uint32_t *tickets;
-    int2 *counts;
-    int32_t *ovf;
-    uint32_t *cand;
+    uint32_t *ukeys;
     float *part_o, *part_lse;
     uint32_t *err;
 };

@@ -6,52 +6,55 @@
 //
 // Grid (G, units): G CTAs per (sequence, kv head) unit u, one CTA per SM,
 // launched cooperatively so the G CTAs of a unit are co-resident.  CTA x owns
-// the x-th contiguous range of the unit's complete blocks.
+// the x-th contiguous range of `per` complete blocks of its unit.
 //
 //  1. Scoring.  All 12 warps stream the range's descriptors (this head's min
-//     and max rows, 4d bytes per block) through per-warp cp.async rings; the
-//     order-preserving keys of the fp32 scores stay in shared memory and their
-//     top 16 bits feed the unit's histogram in the workspace (aggregated per
-//     CTA in a shared-memory hash table first).
-//  2. Unit barrier.  Every CTA reads the touched bins and finds the boundary
-//     bin d1 that holds the k-th largest key.  Blocks above it are selected
-//     for certain ("definite"); blocks in it are candidates, published with a
-//     composite key (low 16 key bits, then the complement of the block id, so
-//     larger means higher score or, on equal scores, lower block id).  Each
-//     CTA also publishes its definite count and the definite blocks beyond its
-//     fair share F = ceil((k + 1) / G), then arrives at a second barrier.
-//  3. The eight decode warps start at once on the CTA's own definite blocks
-//     (at most F), each with a 3-stage K/V ring of 16-byte cp.async copies and
-//     swapped m16n8k16 MMAs (attn_common.cuh).
-//  4. Meanwhile the four control warps wait for the second barrier, find the
-//     exact threshold among the unit's candidates by radix select, and build
-//     the residual pool: definite blocks over the fair shares, qualifying
-//     candidates, the current block.  Every CTA computes the same pool and
-//     takes the slice that fills its share, so all CTAs end with F blocks at
-//     most.  They also write the block list (ascending) and its count.
-//  5. The decode warps finish with the residual slice; the CTA merges its
-//     warps and writes a partial (o / l, log2-sum-exp); the last CTA of the
-//     unit to arrive merges the G partials into the output.
+//     and max rows, 4d bytes per block) through per-warp cp.async rings, eight
+//     blocks per warp step, four lanes per block.  The order-preserving keys of
+//     the fp32 scores go to shared memory and to the unit's key row in the
+//     workspace; their top 16 bits feed the unit's histogram (aggregated per
+//     CTA in a shared-memory hash table, then one atomic per distinct digit).
+//  2. Unit barrier.  In one round trip every CTA reads the histogram bins
+//     around its own top digit and the unit's whole key row (into the idle
+//     K/V ring).  The boundary digit d1 holding the k-th largest key splits
+//     the blocks into definite (above d1) and candidates (at d1); a radix
+//     select over the candidates' composite keys (low 16 key bits, then the
+//     complement of the block id: larger = higher score or, on equal scores,
+//     lower block id) gives the exact threshold.  Every CTA holds every key,
+//     so every CTA computes the same canonical work layout without another
+//     exchange: CTA x' keeps its own selected blocks (definite, then
+//     qualifying candidates, each in block order) up to the fair share
+//     F = ceil((k + 1) / G); the rest is the pool (CTA order, then the current
+//     block), and CTA x takes the slice of the pool that fills its share.
+//  3. The eight decode warps attend to their F blocks with per-warp 3-stage
+//     K/V rings of 16-byte cp.async copies and swapped m16n8k16 MMAs
+//     (attn_common.cuh); the other four warps write the block list (ascending)
+//     and the count.
+//  4. The CTA merges its warps into a partial (o / l, log2-sum-exp); after a
+//     second unit barrier each of the first g * d/32 CTAs merges one (query
+//     row, 32 channels) slice of the unit's G partials; the others leave.
 //
 // The append (K/V of the decode token at position L-1 and the fold of its key
-// into the current block's descriptor) is done by a control warp of CTA 0 of
-// each unit before it arrives at the second barrier: only the current block
-// reads it, and that block is decoded after the barrier.
+// into the current block's descriptor) is done by one warp of CTA 0 of each
+// unit during the scoring phase: only the current block reads it, and that
+// block is never scored and is decoded after the barrier.
 #include "attn_common.cuh"
 
 namespace resa {
 namespace {
 
 constexpr int kDW = kDecodeWarps;         // decode warps
-constexpr int kCW = 4;                    // control warps
+constexpr int kCW = 4;                    // the other warps
 constexpr int kWarpsAll = kDW + kCW;
 constexpr int kThreadsAll = 32 * kWarpsAll;
 constexpr int kCtlThreads = 32 * kCW;
 constexpr int kKvStages = 3;
-constexpr int kDescSlots = 16;            // 512-byte descriptor slots per warp in flight
+constexpr int kScoreSlots = 4;            // descriptor ring slots per warp (8 blocks each)
+constexpr int kScoreBlocks = 8;           // blocks per warp step of the scoring loop
 constexpr int kHash = 1024;               // per-CTA digit histogram slots
 constexpr uint32_t kHashEmpty = 0xffffffffu;
 constexpr uint32_t kSkip = 0xffffffffu;   // work item without data (bad page id)
+constexpr uint32_t kLookup = 0x80000000u; // work entry holding a block id (page not yet read)
 constexpr int kModeAll = 0, kModeNone = 1, kModeMid = 2;
 
 template <int D>
@@ -60,16 +63,17 @@ struct StepSmem {
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = kDW * kKvStages * kStageBytes;
     static constexpr int kDescBytes = 4 * D;  // min and max rows of one (block, head)
-    static_assert(kWarpsAll * kDescSlots * 512 <= kRingBytes, "descriptor rings fit the K/V rings");
+    static constexpr int kSlotBytes = kScoreBlocks * kDescBytes;
+    static_assert(kWarpsAll * kScoreSlots * kSlotBytes <= kRingBytes, "score rings fit the K/V rings");
     static_assert(kDW * kMaxGroup * (D + 2) * 4 <= kRingBytes, "warp states fit the rings");
-    static constexpr int kKeysOff = kRingBytes;
-    static constexpr int kPagesOff = kKeysOff + kStepMaxBlocks * 4;
-    static constexpr int kDefOff = kPagesOff + kStepMaxBlocks * 4;
-    static constexpr int kResCap = kStepMaxBlocks + 64;
-    static constexpr int kResOff = kDefOff + kStepMaxBlocks * 2;
-    static constexpr int kCandOff = kResOff + kResCap * 4;
-    static constexpr int kCandBytes = kStepCandCap * 4 > 2 * kHash * 4 ? kStepCandCap * 4 : 2 * kHash * 4;
-    static constexpr int kBytes = kCandOff + kCandBytes + 1024;  // + base alignment
+    static_assert(step_unit_keys(D) * 4 <= kRingBytes, "the unit's keys and candidates fit the rings");
+    static constexpr int kKeysOff = kRingBytes;                      // u32 [kStepMaxBlocks] own keys
+    static constexpr int kPagesOff = kKeysOff + kStepMaxBlocks * 4;  // i32 [kStepMaxBlocks] own pages
+    static constexpr int kItemOff = kPagesOff + kStepMaxBlocks * 4;  // u32 [kStepMaxBlocks] own work
+    static constexpr int kResCap = kStepMaxBlocks + 8;
+    static constexpr int kResOff = kItemOff + kStepMaxBlocks * 4;    // u32 [kResCap] the rest
+    static constexpr int kHashOff = kResOff + kResCap * 4;           // u32 [2][kHash]
+    static constexpr int kBytes = kHashOff + 2 * kHash * 4 + 128;    // + base alignment
 };
 
 struct StepArgs {
@@ -81,22 +85,18 @@ struct StepArgs {
     int32_t *block_idx, *block_cnt;
     float *out, *lse;
     uint32_t *hist, *hist_range;
-    unsigned long long *bars;
-    uint32_t *tickets;
-    int2 *counts;
-    int32_t *ovf;
-    uint32_t *cand;
+    unsigned long long *bars;  // [units][2] unit barriers
+    uint32_t *ukeys;           // [units][key_stride] every block's key
     float *part_o, *part_lse;
     uint32_t *err;
-    int hkv, g, max_pages, num_pages, max_topk;
+    int hkv, g, max_pages, num_pages, max_topk, key_stride;
     float scale_log2;
 };
 
 // ---------------------------------------------------------------------------
 // Unit barrier: one 64-bit word per barrier holds (generation << 32) |
 // arrivals; the last arriver's single add returns the count to zero and bumps
-// the generation.  Arrive and wait are split so that a CTA can work between
-// them.  The caller fences its writes before arriving.
+// the generation.  The caller fences its writes before arriving.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t unit_bar_arrive(unsigned long long *bar, uint32_t n) {
     const unsigned long long old = atomicAdd(bar, 1ull);
@@ -110,10 +110,6 @@ __device__ __forceinline__ bool unit_bar_wait(const unsigned long long *bar, uin
         if ((uint32_t)(v >> 32) != gen) return true;
         if (polls > (1u << 22)) return false;  // each poll is an L2 round trip
     }
-}
-
-__device__ __forceinline__ void ctl_sync() {
-    asm volatile("bar.sync 1, %0;" ::"r"(kCtlThreads) : "memory");
 }
 
 // Exclusive scan of one value per thread over the whole CTA, in thread order.
@@ -139,7 +135,7 @@ __device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t *tmp, uint32_t
     return before + incl - v;
 }
 
-// The same over the control warps (ct = thread index within them).
+// The same over the last kCW warps (ct = thread index within them).
 __device__ __forceinline__ uint32_t ctl_scan(uint32_t v, int ct, uint32_t *tmp, uint32_t &total) {
     const int lane = ct & 31, w = ct >> 5;
     uint32_t incl = v;
@@ -149,7 +145,7 @@ __device__ __forceinline__ uint32_t ctl_scan(uint32_t v, int ct, uint32_t *tmp, 
         if (lane >= o) incl += t;
     }
     if (lane == 31) tmp[w] = incl;
-    ctl_sync();
+    asm volatile("bar.sync 1, %0;" ::"r"(kCtlThreads) : "memory");
     uint32_t before = 0, tot = 0;
 #pragma unroll
     for (int i = 0; i < kCW; ++i) {
@@ -158,56 +154,8 @@ __device__ __forceinline__ uint32_t ctl_scan(uint32_t v, int ct, uint32_t *tmp, 
         tot += t;
     }
     total = tot;
-    ctl_sync();
+    asm volatile("bar.sync 1, %0;" ::"r"(kCtlThreads) : "memory");
     return before + incl - v;
-}
-
-// The kth largest (1-based) of n distinct 32-bit keys key(0 .. n-1), by radix
-// select over four 8-bit digits, most significant first, on the control warps.
-template <typename KeyFn>
-__device__ uint32_t ctl_select_kth(KeyFn key, int n, uint32_t kth, int ct, uint32_t *rh,
-                                   uint32_t *rsh) {
-    uint32_t prefix = 0, pmask = 0, remaining = kth;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = ct; i < 256; i += kCtlThreads) rh[i] = 0;
-        ctl_sync();
-        for (int i = ct; i < n; i += kCtlThreads) {
-            const uint32_t x = key(i);
-            if ((x & pmask) == prefix) atomicAdd(&rh[(x >> shift) & 255u], 1u);
-        }
-        ctl_sync();
-        if (ct < 32) {
-            // lane l holds digits 255 - 8l - j, j = 0..7 (descending)
-            uint32_t c[8], sum = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                c[j] = rh[255 - 8 * ct - j];
-                sum += c[j];
-            }
-            uint32_t incl = sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (ct >= o) incl += t;
-            }
-            uint32_t cum = incl - sum;  // keys in higher digits than this lane's
-            if (cum < remaining && remaining <= incl) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (cum < remaining && remaining <= cum + c[j]) {
-                        rsh[0] = 255u - 8u * ct - j;
-                        rsh[1] = cum;
-                    }
-                    cum += c[j];
-                }
-            }
-        }
-        ctl_sync();
-        remaining -= rsh[1];
-        prefix |= rsh[0] << shift;
-        pmask |= 255u << shift;
-    }
-    return prefix;
 }
 
 // Largest i in [0, n) with a[i] <= v (a ascending, a[0] <= v).
@@ -221,38 +169,44 @@ __device__ __forceinline__ int upper_index(const int *a, int n, int v) {
     return lo;
 }
 
-__device__ __forceinline__ uint32_t pack_item(int page, int ntok) {
-    return ((uint32_t)page << 4) | (uint32_t)(ntok - 1);
+__device__ __forceinline__ uint32_t item_of_page(int page, int num_pages, int ntok) {
+    return (page >= 0 && page < num_pages) ? (((uint32_t)page << 4) | (uint32_t)(ntok - 1)) : kSkip;
+}
+
+// Composite selection key of block i whose score key is k (its top 16 bits
+// are the boundary digit): larger = higher score, then lower block id.
+__device__ __forceinline__ uint32_t composite(uint32_t k, int i) {
+    return ((k & 0xffffu) << 16) | (0xffffu - (uint32_t)i);
 }
 
 // Indices of the small shared values.
 enum {
-    kVD1 = 0, kVAbove, kVDlo, kVDhi, kVHistOk, kVNd, kVNc, kVNres, kVOk, kVOk2, kVLast,
-    kVOV, kVNC, kVAB, kVSpareBefore, kVDefBefore, kVQBefore, kVLo, kVHi, kVCount
+    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVOk3, kVLo, kVHi, kVAB, kVSpareBefore,
+    kVSelBefore, kVCount
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepArgs a) {
     using SM = StepSmem<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    // 128-byte aligned base, derived from the shared array itself so that
+    // accesses keep the shared address space (no generic loads)
+    uint8_t *smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
     uint8_t *ring = smem;
+    uint32_t *ukeys_s = reinterpret_cast<uint32_t *>(ring);  // the unit's keys (after scoring)
     uint32_t *keys = reinterpret_cast<uint32_t *>(smem + SM::kKeysOff);
     int32_t *pages = reinterpret_cast<int32_t *>(smem + SM::kPagesOff);
-    uint16_t *own_def = reinterpret_cast<uint16_t *>(smem + SM::kDefOff);
+    uint32_t *own_item = reinterpret_cast<uint32_t *>(smem + SM::kItemOff);
     uint32_t *res_item = reinterpret_cast<uint32_t *>(smem + SM::kResOff);
-    uint32_t *cand_s = reinterpret_cast<uint32_t *>(smem + SM::kCandOff);
-    uint32_t *hkey = cand_s, *hcnt = cand_s + kHash;  // scoring phase only
+    uint32_t *hkey = reinterpret_cast<uint32_t *>(smem + SM::kHashOff), *hcnt = hkey + kHash;
 
     __shared__ float qbar_s[D];
-    __shared__ __align__(8) uint64_t res_bar;
-    __shared__ int s_coff[kNumSms + 1], s_ovoff[kNumSms + 1];
+    __shared__ int s_nd[kNumSms], s_q[kNumSms], s_poff[kNumSms + 1];
     __shared__ uint32_t s_rh[256];
     __shared__ uint32_t s_scan[kWarpsAll];
-    __shared__ uint32_t s_rsh[2];
+    __shared__ uint32_t s_rsh[3];
     __shared__ int s_v[kVCount];
-    __shared__ float s_lse[kMaxGroup];
+    __shared__ int s_seg[kWarpsAll];
 
     pdl_launch_next();
     const int x = blockIdx.x, G = gridDim.x, u = blockIdx.y;
@@ -276,7 +230,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     const int p0 = min(M, x * per);
     const int nmine = min(min(M, p0 + per) - p0, kStepMaxBlocks);  // the host keeps per <= cap
     const size_t prow = (size_t)b * a.max_pages;
-    const size_t cap_base = (size_t)cta * kStepMaxBlocks;
+    uint32_t *ukeys_g = a.ukeys + (size_t)u * a.key_stride;
 
     // ---- prologue: inputs of the call only (before the dependency wait) ----
     for (int i = tid; i < nmine; i += kThreadsAll) pages[i] = a.page_table[prow + p0 + i];
@@ -292,15 +246,16 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         hkey[i] = kHashEmpty;
         hcnt[i] = 0;
     }
+    for (int i = tid; i < G; i += kThreadsAll) {
+        s_nd[i] = 0;
+        s_q[i] = 0;
+    }
     if (tid == 0) {
-        mbar_init(&res_bar, 1);
-        fence_mbar_init();
         s_v[kVOk] = 1;
-        s_v[kVOk2] = 1;
+        s_v[kVOk3] = 1;
         s_v[kVLo] = 0x7fffffff;
         s_v[kVHi] = -1;
         s_v[kVD1] = 0;
-        s_v[kVAbove] = 0;
         s_v[kVHistOk] = 1;
     }
     // Q^T fragments for the decode warps: head lane/4 (zero beyond g),
@@ -316,113 +271,181 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             qb[ks][0][1] = row ? *reinterpret_cast<const uint32_t *>(row + ks * 16 + c + 8) : 0u;
         }
     }
+    // The current block's page (its tokens are decoded by whichever CTA draws
+    // it) and, for the appending warp, the decode token's K / V chunks.
+    const int cur_page = seq_ok ? a.page_table[prow + M] : -1;
+    constexpr int CPR = D / 8;  // 16-byte chunks per K / V row
     const bool appender = x == 0 && warp == kWarpsAll - 1 && seq_ok;
-    const int app_page = appender ? a.page_table[prow + (L - 1) / kBlock] : -1;
+    uint4 app_k = make_uint4(0, 0, 0, 0), app_v = app_k;
+    if (appender && lane < CPR) {
+        app_k = a.k_new[((size_t)b * hkv + h) * CPR + lane];
+        app_v = a.v_new[((size_t)b * hkv + h) * CPR + lane];
+    }
     __syncthreads();
     pdl_wait();  // descriptors and K/V may be written by the preceding kernels
 
-    // ---- 1. scoring ----
-    const bool need_hist = mode == kModeMid;
+    // ---- 1. scoring (+ the append, whose descriptor loads are issued first) ----
+    uint4 app_mn = make_uint4(0, 0, 0, 0), app_mx = app_mn;
+    const int app_slot = (L - 1) % kBlock;
+    const bool app_ok = appender && cur_page >= 0 && cur_page < a.num_pages;
+    uint4 *app_dmn = nullptr;
+    if (app_ok && lane < CPR) {
+        app_dmn = reinterpret_cast<uint4 *>(a.desc) + (((size_t)cur_page * hkv + h) * 2) * CPR + lane;
+        if (app_slot != 0) {
+            app_mn = app_dmn[0];
+            app_mx = app_dmn[CPR];
+        }
+    }
     {
-        constexpr int LPP = D / 4;     // lanes per block, 4 channels each
-        constexpr int PPI = 32 / LPP;  // blocks per warp iteration
-        const int sub = lane / LPP, c4 = lane % LPP;
-        const int ngroups = (nmine + PPI - 1) / PPI;
-        const int nmy = warp < ngroups ? (ngroups - warp + kWarpsAll - 1) / kWarpsAll : 0;
-        uint8_t *wring = ring + (size_t)warp * kDescSlots * 512;
-        auto blk_of = [&](int it) { return (warp + kWarpsAll * it) * PPI + sub; };
+        constexpr int CPB = SM::kDescBytes / 16;     // 16-byte chunks per block descriptor
+        constexpr int RC = D / 32;                   // chunks of a row one lane reads
+        constexpr int COPIES = kScoreBlocks * CPB / 32;
+        const int nsteps = (nmine + kScoreBlocks - 1) / kScoreBlocks;
+        const int nmy = warp < nsteps ? (nsteps - warp + kWarpsAll - 1) / kWarpsAll : 0;
+        uint8_t *wring = ring + (size_t)warp * kScoreSlots * SM::kSlotBytes;
+        // Block j of a slot sits at j * 4d bytes; its 16-byte chunk c at
+        // (c ^ 4 (j odd)), so the two blocks a quarter-warp reads fall in
+        // different banks.
         auto issue = [&](int it) {
             if (it < nmy) {
-                const int pi = blk_of(it);
-                if (pi < nmine) {
-                    const int pg = pages[pi];
-                    if (pg >= 0 && pg < a.num_pages) {
-                        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.desc) +
-                                             ((size_t)pg * hkv + h) * SM::kDescBytes;
-                        cp_async16(wring + (size_t)(it % kDescSlots) * 512 + lane * 16, src + c4 * 16);
+                const int blk0 = (warp + kWarpsAll * it) * kScoreBlocks;
+                uint8_t *slot = wring + (size_t)(it % kScoreSlots) * SM::kSlotBytes;
+#pragma unroll
+                for (int i = 0; i < COPIES; ++i) {
+                    const int f = i * 32 + lane;
+                    const int j = f / CPB, c = f % CPB;
+                    const int pi = blk0 + j;
+                    if (pi < nmine) {
+                        const int pg = pages[pi];
+                        if (pg >= 0 && pg < a.num_pages)
+                            cp_async16(slot + j * SM::kDescBytes + ((c ^ ((j & 1) << 2)) << 4),
+                                       reinterpret_cast<const uint8_t *>(a.desc) +
+                                           ((size_t)pg * hkv + h) * SM::kDescBytes + c * 16);
                     }
                 }
             }
             cp_async_commit();
         };
 #pragma unroll
-        for (int it = 0; it < kDescSlots - 1; ++it) issue(it);
-        float qv[4];
+        for (int it = 0; it < kScoreSlots - 1; ++it) issue(it);
+        const int j = lane >> 2, s = lane & 3, sw = (j & 1) << 2;
+        float qv[RC][8];
+        uint32_t sel[RC][4];
 #pragma unroll
-        for (int n = 0; n < 4; ++n) qv[n] = qbar_s[4 * c4 + n];
-        const uint32_t sel0 = upper_bound_selector(qv[0], qv[1]);
-        const uint32_t sel1 = upper_bound_selector(qv[2], qv[3]);
-        int lo = 0x7fffffff, hi = -1;  // digits that bypassed the hash table
+        for (int k = 0; k < RC; ++k) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qv[k][e] = qbar_s[(4 * k + s) * 8 + e];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) sel[k][w] = upper_bound_selector(qv[k][2 * w], qv[k][2 * w + 1]);
+        }
         for (int it = 0; it < nmy; ++it) {
-            issue(it + kDescSlots - 1);
-            cp_async_wait<kDescSlots - 1>();
+            issue(it + kScoreSlots - 1);
+            cp_async_wait<kScoreSlots - 1>();
             __syncwarp();
-            const uint8_t *pg = wring + (size_t)(it % kDescSlots) * 512 + sub * SM::kDescBytes;
-            const uint2 mn = *reinterpret_cast<const uint2 *>(pg + 8 * c4);
-            const uint2 mx = *reinterpret_cast<const uint2 *>(pg + 2 * D + 8 * c4);
-            __syncwarp();  // the slot is refilled by the next issue
-            const uint32_t w0 = __byte_perm(mn.x, mx.x, sel0);
-            const uint32_t w1 = __byte_perm(mn.y, mx.y, sel1);
-            float sum = __fmul_rn(qv[0], __uint_as_float(w0 << 16));
-            sum = __fadd_rn(sum, __fmul_rn(qv[1], __uint_as_float(w0 & 0xffff0000u)));
-            sum = __fadd_rn(sum, __fmul_rn(qv[2], __uint_as_float(w1 << 16)));
-            sum = __fadd_rn(sum, __fmul_rn(qv[3], __uint_as_float(w1 & 0xffff0000u)));
+            const uint8_t *bp = wring + (size_t)(it % kScoreSlots) * SM::kSlotBytes + j * SM::kDescBytes;
+            float part[RC];
 #pragma unroll
-            for (int o = LPP / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            const int pi = blk_of(it);
-            if (c4 == 0 && pi < nmine) {
-                const int pgid = pages[pi];
-                const bool ok = pgid >= 0 && pgid < a.num_pages;
+            for (int k = 0; k < RC; ++k) {
+                const int c = 4 * k + s;
+                const uint4 mn = *reinterpret_cast<const uint4 *>(bp + ((c ^ sw) << 4));
+                const uint4 mx = *reinterpret_cast<const uint4 *>(bp + (((c + D / 8) ^ sw) << 4));
+                const uint32_t mnw[4] = {mn.x, mn.y, mn.z, mn.w};
+                const uint32_t mxw[4] = {mx.x, mx.y, mx.z, mx.w};
+                float acc = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const uint32_t pw = __byte_perm(mnw[w], mxw[w], sel[k][w]);
+                    acc = __fadd_rn(acc, __fmul_rn(qv[k][2 * w], __uint_as_float(pw << 16)));
+                    acc = __fadd_rn(acc, __fmul_rn(qv[k][2 * w + 1], __uint_as_float(pw & 0xffff0000u)));
+                }
+                part[k] = acc;
+            }
+            __syncwarp();  // the slot is refilled by the next issue
+            float sum = part[0];
+#pragma unroll
+            for (int k = 1; k < RC; ++k) sum = __fadd_rn(sum, part[k]);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            const int pi = (warp + kWarpsAll * it) * kScoreBlocks + j;
+            if (s == 0 && pi < nmine) {
+                const int pg = pages[pi];
+                const bool ok = pg >= 0 && pg < a.num_pages;
                 if (!ok) set_error(a.err, RESA_DEVERR_PAGE);
                 const uint32_t key = ok ? order_key(sum) : 0u;
                 keys[pi] = key;
-                if (need_hist) {
-                    const uint32_t digit = key >> 16;
-                    uint32_t slot = (digit * 0x9E3779B1u) >> 22;  // 10 bits
-                    bool placed = false;
-                    for (int probe = 0; probe < 64; ++probe) {
-                        const uint32_t old = atomicCAS(&hkey[slot], kHashEmpty, digit);
-                        if (old == kHashEmpty || old == digit) {
-                            atomicAdd(&hcnt[slot], 1u);
-                            placed = true;
-                            break;
-                        }
-                        slot = (slot + 1) & (kHash - 1);
-                    }
-                    if (!placed) {
-                        atomicAdd(&a.hist[(size_t)u * kHistBins + digit], 1u);
-                        lo = min(lo, (int)digit);
-                        hi = max(hi, (int)digit);
-                    }
-                }
+                ukeys_g[p0 + pi] = key;
             }
         }
         cp_async_wait<0>();
-        __syncthreads();
-        if (need_hist) {
-            for (int i = tid; i < kHash; i += kThreadsAll) {
-                const uint32_t k = hkey[i];
-                if (k != kHashEmpty) {
-                    atomicAdd(&a.hist[(size_t)u * kHistBins + k], hcnt[i]);
-                    lo = min(lo, (int)k);
-                    hi = max(hi, (int)k);
+    }
+    if (appender) {
+        // decode-token append: K/V at position L-1, key folded into the
+        // current block's descriptor (a new block starts from the key)
+        if (!app_ok) {
+            if (lane == 0) set_error(a.err, RESA_DEVERR_PAGE);
+        } else if (lane < CPR) {
+            const size_t o = (((size_t)cur_page * hkv + h) * kBlock + app_slot) * CPR + lane;
+            reinterpret_cast<uint4 *>(a.k_cache)[o] = app_k;
+            reinterpret_cast<uint4 *>(a.v_cache)[o] = app_v;
+            if (app_slot == 0) {
+                app_dmn[0] = app_k;
+                app_dmn[CPR] = app_k;
+            } else {
+                Bf16x8 mn = unpack8(app_mn), mx = unpack8(app_mx);
+                fold8(mn, mx, unpack8(app_k));
+                app_dmn[0] = pack8(mn);
+                app_dmn[CPR] = pack8(mx);
+            }
+        }
+    }
+    __syncthreads();
+    const bool need_hist = mode == kModeMid;
+    if (need_hist) {
+        // per-CTA histogram of the keys' top 16 bits, then one global atomic
+        // per distinct digit
+        int lo = 0x7fffffff, hi = -1;
+        for (int i = tid; i < nmine; i += kThreadsAll) {
+            const uint32_t digit = keys[i] >> 16;
+            uint32_t slot = (digit * 0x9E3779B1u) >> 22;  // 10 bits
+            bool placed = false;
+            for (int probe = 0; probe < 64; ++probe) {
+                const uint32_t old = atomicCAS(&hkey[slot], kHashEmpty, digit);
+                if (old == kHashEmpty || old == digit) {
+                    atomicAdd(&hcnt[slot], 1u);
+                    placed = true;
+                    break;
                 }
+                slot = (slot + 1) & (kHash - 1);
             }
-            if (hi >= 0) {
-                atomicMin(&s_v[kVLo], lo);
-                atomicMax(&s_v[kVHi], hi);
+            if (!placed) {
+                atomicAdd(&a.hist[(size_t)u * kHistBins + digit], 1u);
+                lo = min(lo, (int)digit);
+                hi = max(hi, (int)digit);
             }
-            __syncthreads();
-            if (tid == 0 && s_v[kVHi] >= 0) {
-                atomicMax(&a.hist_range[2 * u], (uint32_t)(kHistBins - s_v[kVLo]));  // 0 = untouched
-                atomicMax(&a.hist_range[2 * u + 1], (uint32_t)(s_v[kVHi] + 1));
+        }
+        __syncthreads();
+        for (int i = tid; i < kHash; i += kThreadsAll) {
+            const uint32_t k = hkey[i];
+            if (k != kHashEmpty) {
+                atomicAdd(&a.hist[(size_t)u * kHistBins + k], hcnt[i]);
+                lo = min(lo, (int)k);
+                hi = max(hi, (int)k);
             }
+        }
+        if (hi >= 0) {
+            atomicMin(&s_v[kVLo], lo);
+            atomicMax(&s_v[kVHi], hi);
+        }
+        __syncthreads();
+        if (tid == 0 && s_v[kVHi] >= 0) {
+            atomicMax(&a.hist_range[2 * u], (uint32_t)(kHistBins - s_v[kVLo]));  // 0 = untouched
+            atomicMax(&a.hist_range[2 * u + 1], (uint32_t)(s_v[kVHi] + 1));
         }
     }
     __threadfence();
     __syncthreads();
 
-    // ---- 2. boundary bin, own lists, second barrier ----
+    // ---- 2. unit barrier; the unit's keys and histogram; threshold; layout ----
     if (G > 1 && need_hist) {
         if (tid == 0) {
             const uint32_t gen = unit_bar_arrive(&a.bars[2 * u], G);
@@ -435,48 +458,46 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
         __threadfence();
     }
+    uint32_t d1 = 0;
     if (need_hist) {
-        const uint32_t emin = __ldcg(&a.hist_range[2 * u]), emax = __ldcg(&a.hist_range[2 * u + 1]);
-        const int dlo = kHistBins - (int)emin, dhi = (int)emax - 1;
-        const int nb = dhi >= dlo ? dhi - dlo + 1 : 0;
+        // One round trip in the common case: every key of the unit (into the
+        // idle K/V ring), the touched range and a window of kThreadsAll bins
+        // below (this CTA's top digit + 128); the whole touched range is read
+        // only when the window does not hold it.
+        for (int c = tid; c < (M + 3) / 4; c += kThreadsAll) cp_async16(ukeys_s + 4 * c, ukeys_g + 4 * c);
+        cp_async_commit();
         const uint32_t *hb = a.hist + (size_t)u * kHistBins;
-        const int chunk = (nb + kThreadsAll - 1) / kThreadsAll;
-        const int top = dhi - tid * chunk, bot = max(dlo, top - chunk + 1);
-        constexpr int kBinRegs = 8;
-        uint32_t binc[kBinRegs];
-        uint32_t loc = 0;
-        if (chunk <= kBinRegs) {
-#pragma unroll
-            for (int j = 0; j < kBinRegs; ++j) {
-                binc[j] = (j < chunk && top - j >= bot) ? __ldcg(&hb[top - j]) : 0u;
-                loc += binc[j];
-            }
+        const int wtop = min(kHistBins - 1, s_v[kVHi] + 128);
+        const int wbot = max(0, wtop - (kThreadsAll - 1));
+        const uint32_t emin = __ldcg(&a.hist_range[2 * u]), emax = __ldcg(&a.hist_range[2 * u + 1]);
+        const int wd = wtop - tid;
+        const uint32_t wc = wd >= wbot ? __ldcg(&hb[wd]) : 0u;
+        const int dlo = kHistBins - (int)emin, dhi = (int)emax - 1;
+        const bool covered = dlo >= wbot && dhi <= wtop;  // uniform over the CTA
+        uint32_t total, above_me, loc;
+        int top, bot;
+        if (covered) {
+            loc = wc;
+            top = wd;
+            bot = wd;
         } else {
+            const int nb = dhi >= dlo ? dhi - dlo + 1 : 0;
+            const int chunk = (nb + kThreadsAll - 1) / kThreadsAll;
+            top = dhi - tid * chunk;
+            bot = max(dlo, top - chunk + 1);
+            loc = 0;
             for (int d = top; d >= bot; --d) loc += __ldcg(&hb[d]);
         }
-        uint32_t total;
-        const uint32_t above_me = cta_scan(loc, s_scan, total);
+        above_me = cta_scan(loc, s_scan, total);  // keys in the bins above this thread's
         if (above_me < (uint32_t)keff && (uint32_t)keff <= above_me + loc) {
             uint32_t cum = above_me;
-            if (chunk <= kBinRegs) {
-#pragma unroll
-                for (int j = 0; j < kBinRegs; ++j) {
-                    if (j < chunk && top - j >= bot && cum < (uint32_t)keff && cum + binc[j] >= (uint32_t)keff) {
-                        s_v[kVD1] = top - j;
-                        s_v[kVAbove] = (int)cum;
-                    }
-                    cum += binc[j];
+            for (int d = top; d >= bot; --d) {
+                const uint32_t c = covered ? wc : __ldcg(&hb[d]);
+                if (cum + c >= (uint32_t)keff) {
+                    s_v[kVD1] = d;
+                    break;
                 }
-            } else {
-                for (int d = top; d >= bot; --d) {
-                    const uint32_t c = __ldcg(&hb[d]);
-                    if (cum + c >= (uint32_t)keff) {
-                        s_v[kVD1] = d;
-                        s_v[kVAbove] = (int)cum;
-                        break;
-                    }
-                    cum += c;
-                }
+                cum += c;
             }
         }
         if (tid == 0) {
@@ -484,6 +505,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             s_v[kVDhi] = dhi;
             s_v[kVHistOk] = total == (uint32_t)M ? 1 : 0;
         }
+        cp_async_wait<0>();
         __syncthreads();
         if (!s_v[kVHistOk]) {
             // The histogram was not clean at entry (an earlier call gave up
@@ -493,107 +515,329 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             mode = kModeNone;
             keff = 0;
         }
+        d1 = (uint32_t)s_v[kVD1];
     }
-    const int W = seq_ok ? keff + 1 : 0;
-    const int F = (W + G - 1) / G;
-    const uint32_t d1 = (uint32_t)s_v[kVD1];
-    {
-        // Classify the CTA's blocks: definite (ascending local ids into
-        // own_def) and candidates (composite keys into the workspace).
-        constexpr int R = (kStepMaxBlocks + kThreadsAll - 1) / kThreadsAll;
-        const int i0 = tid * R;
-        uint32_t nd_t = 0, nc_t = 0;
+    const int F = ((seq_ok ? keff + 1 : 0) + G - 1) / G;
+    // Per-CTA counts from the unit's keys, branch-free: each warp takes 32-key
+    // groups (one key a lane, four groups in flight), records the ballots of
+    // the definite keys and of the candidates per group, and appends the
+    // candidates' composite keys to its own segment of the list after the keys.
+    const int ngroups = (M + 31) >> 5;
+    const int KW = (ngroups + kWarpsAll - 1) / kWarpsAll * 32;  // keys one warp sees at most
+    uint32_t *cand_s = ukeys_s + ((M + 3) & ~3);                // [kWarpsAll][KW]
+    uint32_t *defm = hkey, *candm = hcnt;                       // [ngroups] (hash area, free now)
+    if (mode == kModeMid) {
+        const uint32_t lt_mask = (1u << lane) - 1u;
+        uint32_t *seg = cand_s + warp * KW;
+        int nseg = 0;
+        for (int g0 = warp; g0 < ngroups; g0 += 4 * kWarpsAll) {
+            uint32_t kk[4];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
+            for (int u4 = 0; u4 < 4; ++u4) {
+                const int i = (g0 + kWarpsAll * u4) * 32 + lane;
+                kk[u4] = i < M ? ukeys_s[i] : 0u;
+            }
+#pragma unroll
+            for (int u4 = 0; u4 < 4; ++u4) {
+                const int grp = g0 + kWarpsAll * u4;
+                const int i = grp * 32 + lane;
+                const uint32_t dg = kk[u4] >> 16;
+                const bool isc = i < M && dg == d1;
+                const uint32_t bd = __ballot_sync(0xffffffffu, i < M && dg > d1);
+                const uint32_t bc = __ballot_sync(0xffffffffu, isc);
+                if (lane == 0 && grp < ngroups) {
+                    defm[grp] = bd;
+                    candm[grp] = bc;
+                }
+                if (isc) seg[nseg + __popc(bc & lt_mask)] = composite(kk[u4], i);
+                nseg += __popc(bc);
+            }
+        }
+        if (lane == 0) s_seg[warp] = nseg;
+    }
+    __syncthreads();
+    // definite blocks per CTA range: popcounts of the ballots, a warp per range
+    if (mode == kModeMid) {
+        for (int src = warp; src < G; src += kWarpsAll) {
+            const int b0 = min(M, src * per), b1 = min(M, b0 + per);
+            int cnt = 0;
+            if (b1 > b0)
+                for (int gi = (b0 >> 5) + lane; gi <= ((b1 - 1) >> 5); gi += 32) {
+                    const int lo = max(b0, gi * 32) - gi * 32, hi = min(b1, gi * 32 + 32) - gi * 32;
+                    const uint32_t rm = (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~((1u << lo) - 1u);
+                    cnt += __popc(defm[gi] & rm);
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+            if (lane == 0) s_nd[src] = cnt;
+        }
+    } else if (mode == kModeAll) {
+        for (int i = tid; i < G; i += kThreadsAll) s_nd[i] = max(0, min(M, (i + 1) * per) - min(M, i * per));
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int ab = 0;
+        for (int i = lane; i < G; i += 32) ab += s_nd[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ab += __shfl_xor_sync(0xffffffffu, ab, o);
+        if (lane == 0) s_v[kVAB] = ab;
+    }
+    __syncthreads();
+    // exact threshold: radix select over the candidates' composite keys,
+    // stopping at the first digit whose bin is taken whole
+    // candidate f of the list: segment w = the first with f < its end
+    int seg_end[kWarpsAll];
+    {
+        int acc = 0;
+#pragma unroll
+        for (int w = 0; w < kWarpsAll; ++w) {
+            acc += mode == kModeMid ? s_seg[w] : 0;
+            seg_end[w] = acc;
+        }
+    }
+    const int NC = seg_end[kWarpsAll - 1];
+    auto cand_at = [&](int f) -> uint32_t {
+        int w = 0, start = 0;
+#pragma unroll
+        for (int k = 0; k < kWarpsAll - 1; ++k)
+            if (f >= seg_end[k]) {
+                w = k + 1;
+                start = seg_end[k];
+            }
+        return cand_s[w * KW + (f - start)];
+    };
+    int rem = mode == kModeMid ? keff - s_v[kVAB] : 0;
+    if (rem < 0) {  // cannot happen with consistent counts
+        if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
+        rem = 0;
+    }
+    uint32_t tau = 0xffffffffu;
+    if (rem > 0) {
+        uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)rem;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int i = tid; i < 256; i += kThreadsAll) s_rh[i] = 0;
+            __syncthreads();
+            for (int i = tid; i < NC; i += kThreadsAll) {
+                const uint32_t c = cand_at(i);
+                if ((c & pmask) == prefix) atomicAdd(&s_rh[(c >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // lane l holds digits 255 - 8l - j, j = 0..7 (descending)
+                uint32_t cnt[8], sum = 0;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    cnt[jj] = s_rh[255 - 8 * lane - jj];
+                    sum += cnt[jj];
+                }
+                uint32_t incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                uint32_t cum = incl - sum;
+                if (cum < remaining && remaining <= incl) {
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        if (cum < remaining && remaining <= cum + cnt[jj]) {
+                            s_rsh[0] = 255u - 8u * lane - jj;
+                            s_rsh[1] = cum;
+                            s_rsh[2] = cnt[jj];
+                        }
+                        cum += cnt[jj];
+                    }
+                }
+            }
+            __syncthreads();
+            remaining -= s_rsh[1];
+            prefix |= s_rsh[0] << shift;
+            pmask |= 255u << shift;
+            if (remaining == s_rsh[2]) break;  // every key with this prefix is taken
+        }
+        tau = prefix;
+        // qualifying candidates per CTA
+        for (int i = tid; i < NC; i += kThreadsAll) {
+            const uint32_t c = cand_at(i);
+            if (c >= tau) atomicAdd(&s_q[(int)(0xffffu - (c & 0xffffu)) / per], 1);
+        }
+    }
+    __syncthreads();
+    // canonical work layout: CTA x' keeps its own selected blocks (definite,
+    // then qualifying, each in block order) up to F; the rest is the pool (CTA
+    // order, then the current block); CTA x takes the slice of the pool after
+    // the spare capacity of the CTAs before it
+    if (warp == 0) {
+        const int PL = (G + 31) / 32;
+        const int i0 = lane * PL;
+        int sp = 0, pl = 0, ss = 0;
+        for (int r = 0; r < PL; ++r) {
             const int i = i0 + r;
+            if (i < G) {
+                const int sel = s_nd[i] + s_q[i];
+                sp += F - min(sel, F);
+                pl += sel - min(sel, F);
+                ss += sel;
+            }
+        }
+        int ep = sp, el = pl, es = ss;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t1 = __shfl_up_sync(0xffffffffu, ep, o);
+            const int t2 = __shfl_up_sync(0xffffffffu, el, o);
+            const int t3 = __shfl_up_sync(0xffffffffu, es, o);
+            if (lane >= o) {
+                ep += t1;
+                el += t2;
+                es += t3;
+            }
+        }
+        int bp = ep - sp, bl = el - pl, bs = es - ss;
+        for (int r = 0; r < PL; ++r) {
+            const int i = i0 + r;
+            if (i < G) {
+                if (i == x) {
+                    s_v[kVSpareBefore] = bp;
+                    s_v[kVSelBefore] = bs;
+                }
+                s_poff[i] = bl;
+                const int sel = s_nd[i] + s_q[i];
+                bp += F - min(sel, F);
+                bl += sel - min(sel, F);
+                bs += sel;
+            }
+        }
+        if (lane == 31) s_poff[G] = el;
+    }
+    __syncthreads();
+    const int nd = s_nd[x], myq = s_q[x];
+    const int kept_def = min(nd, F);
+    const int qkeep = max(0, min(myq, F - nd));  // own qualifying candidates kept
+    const int pool = seq_ok ? s_poff[G] + 1 : 0;
+    const int S0 = s_v[kVSpareBefore];
+    const int S1 = min(pool, S0 + (F - min(nd + myq, F)));
+    const int nslice = max(0, S1 - S0);
+    const int n_res = qkeep + nslice;
+    // Is own block i (local index) definite / a qualifying candidate?
+    auto own_def = [&](int i) -> bool {
+        return mode == kModeAll || (mode == kModeMid && (keys[i] >> 16) > d1);
+    };
+    auto own_qual = [&](int i) -> bool {
+        const uint32_t k = keys[i];
+        return rem > 0 && (k >> 16) == d1 && composite(k, p0 + i) >= tau;
+    };
+    {
+        // own definite blocks in block order (this CTA keeps the first F) and
+        // the first qkeep own qualifying candidates
+        constexpr int R1 = (kStepMaxBlocks + kThreadsAll - 1) / kThreadsAll;
+        const int j0 = tid * R1;
+        uint32_t nd_t = 0, nq_t = 0;
+#pragma unroll
+        for (int r = 0; r < R1; ++r) {
+            const int i = j0 + r;
             if (i < nmine) {
-                const uint32_t dg = keys[i] >> 16;
-                nd_t += mode == kModeAll || (mode == kModeMid && dg > d1);
-                nc_t += mode == kModeMid && dg == d1;
+                nd_t += own_def(i);
+                nq_t += own_qual(i);
             }
         }
         uint32_t tot;
-        const uint32_t ex = cta_scan(nd_t | (nc_t << 16), s_scan, tot);
-        uint32_t od = ex & 0xffffu, oc = ex >> 16;
+        const uint32_t ex = cta_scan(nd_t | (nq_t << 16), s_scan, tot);
+        uint32_t od = ex & 0xffffu, oq = ex >> 16;
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int i = i0 + r;
+        for (int r = 0; r < R1; ++r) {
+            const int i = j0 + r;
             if (i < nmine) {
-                const uint32_t key = keys[i];
-                const uint32_t dg = key >> 16;
-                if (mode == kModeAll || (mode == kModeMid && dg > d1)) {
-                    own_def[od++] = (uint16_t)i;
-                } else if (mode == kModeMid && dg == d1) {
-                    a.cand[cap_base + oc++] = ((key & 0xffffu) << 16) | (0xffffu - (uint32_t)(p0 + i));
+                if (own_def(i)) {
+                    if ((int)od < F) own_item[od] = item_of_page(pages[i], a.num_pages, kBlock);
+                    ++od;
+                } else if (own_qual(i)) {
+                    if ((int)oq < qkeep) res_item[oq] = item_of_page(pages[i], a.num_pages, kBlock);
+                    ++oq;
                 }
             }
         }
-        if (tid == 0) {
-            s_v[kVNd] = (int)(tot & 0xffffu);
-            s_v[kVNc] = (int)(tot >> 16);
+    }
+    // the slice [S0, S1) of the pool: per source CTA, its definite blocks
+    // past F, then its qualifying candidates past its kept ones, block order
+    if (nslice > 0) {
+        const int last = pool - 1;  // the current block
+        if (tid == 0 && last >= S0 && last < S1)
+            res_item[qkeep + last - S0] = item_of_page(cur_page, a.num_pages, L - M * kBlock);
+        const int s_hi_pos = min(S1, last) - 1;  // last pool position of a source CTA in the slice
+        if (mode == kModeMid && s_hi_pos >= S0) {
+            const int s_lo = upper_index(s_poff, G, S0), s_hi = upper_index(s_poff, G, s_hi_pos);
+            const uint32_t lt_mask = (1u << lane) - 1u;
+            for (int src = s_lo + warp; src <= s_hi; src += kWarpsAll) {
+                const int ovd = max(0, s_nd[src] - F);
+                const int keepq = max(0, min(s_q[src], F - s_nd[src]));
+                const int base = s_poff[src];
+                const int b0 = min(M, src * per), b1 = min(M, b0 + per);
+                int def_seen = 0, q_seen = 0;
+                for (int c0 = b0; c0 < b1; c0 += 32) {
+                    const int i = c0 + lane;
+                    const uint32_t k = i < b1 ? ukeys_s[i] : 0u;
+                    const bool isd = i < b1 && (k >> 16) > d1;
+                    const bool isq = i < b1 && rem > 0 && (k >> 16) == d1 && composite(k, i) >= tau;
+                    const uint32_t bd = __ballot_sync(0xffffffffu, isd);
+                    const uint32_t bq = __ballot_sync(0xffffffffu, isq);
+                    if (isd) {
+                        const int rank = def_seen + __popc(bd & lt_mask);
+                        const int pos = base + rank - F;
+                        if (rank >= F && pos >= S0 && pos < S1) res_item[qkeep + pos - S0] = kLookup | (uint32_t)i;
+                    }
+                    if (isq) {
+                        const int rank = q_seen + __popc(bq & lt_mask);
+                        const int pos = base + ovd + rank - keepq;
+                        if (rank >= keepq && pos >= S0 && pos < S1) res_item[qkeep + pos - S0] = kLookup | (uint32_t)i;
+                    }
+                    def_seen += __popc(bd);
+                    q_seen += __popc(bq);
+                }
+            }
         }
         __syncthreads();
-        const int nd = s_v[kVNd], kept = min(nd, F);
-        for (int j = kept + tid; j < nd; j += kThreadsAll) a.ovf[cap_base + (j - kept)] = p0 + own_def[j];
-        if (tid == 0) a.counts[cta] = make_int2(nd, s_v[kVNc]);
+        // page ids of the pool blocks (other CTAs' ranges): one round trip
+        for (int r = qkeep + tid; r < n_res; r += kThreadsAll) {
+            const uint32_t v = res_item[r];
+            if ((v & 0xffff0000u) == kLookup)
+                res_item[r] = item_of_page(a.page_table[prow + (v & 0xffffu)], a.num_pages, kBlock);
+        }
     }
-    __threadfence();
     __syncthreads();
-    const int nd = s_v[kVNd];
-    const int kept = min(nd, F);
 
     if (warp < kDW) {
-        // ---- 3 / 5. decode warps ----
+        // ---- 3. decode warps: own definite blocks, then the rest ----
         WarpState<D, 1> st;
         st.init();
-        bool ready = false;
-        int nres = 0;
-        auto get_item = [&](int j, uint32_t &item) -> bool {
-            if (j < kept) {
-                const int pg = pages[own_def[j]];
-                item = (pg >= 0 && pg < a.num_pages) ? pack_item(pg, kBlock) : kSkip;
-                return true;
-            }
-            if (!ready) {
-                ready = true;
-                if (mbar_wait_bounded(&res_bar, 0)) {
-                    nres = s_v[kVNres];
-                } else {
-                    if (lane == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
-                    nres = 0;
-                }
-            }
-            if (j - kept < nres) {
-                item = res_item[j - kept];
-                return true;
-            }
-            return false;
-        };
+        const int n_items = kept_def + n_res;
+        auto item_at = [&](int j) -> uint32_t { return j < kept_def ? own_item[j] : res_item[j - kept_def]; };
         uint8_t *wr = ring + (size_t)warp * kKvStages * SM::kStageBytes;
         constexpr int kPerLane = SM::kTileBytes / 16 / 32;
         auto issue = [&](int t) {
-            uint32_t item;
-            if (get_item(warp + kDW * t, item) && item != kSkip) {
-                const size_t tile = ((size_t)(item >> 4) * hkv + h) * SM::kTileBytes;
-                uint8_t *stg = wr + (size_t)(t % kKvStages) * SM::kStageBytes;
+            const int j = warp + kDW * t;
+            if (j < n_items) {
+                const uint32_t item = item_at(j);
+                if (item != kSkip) {
+                    const size_t tile = ((size_t)(item >> 4) * hkv + h) * SM::kTileBytes;
+                    uint8_t *stg = wr + (size_t)(t % kKvStages) * SM::kStageBytes;
 #pragma unroll
-                for (int k = 0; k < kPerLane; ++k) {
-                    const uint32_t qc = lane + 32 * k;
-                    const uint32_t so = swz128(qc >> 3, qc & 7);
-                    cp_async16(stg + so, a.k_cache + tile + qc * 16);
-                    cp_async16(stg + SM::kTileBytes + so, a.v_cache + tile + qc * 16);
+                    for (int k = 0; k < kPerLane; ++k) {
+                        const uint32_t qc = lane + 32 * k;
+                        const uint32_t so = swz128(qc >> 3, qc & 7);
+                        cp_async16(stg + so, a.k_cache + tile + qc * 16);
+                        cp_async16(stg + SM::kTileBytes + so, a.v_cache + tile + qc * 16);
+                    }
                 }
             }
             cp_async_commit();
         };
 #pragma unroll
         for (int t = 0; t < kKvStages - 1; ++t) issue(t);
-        for (int t = 0;; ++t) {
-            uint32_t item;
-            if (!get_item(warp + kDW * t, item)) break;
+        for (int t = 0; warp + kDW * t < n_items; ++t) {
             issue(t + kKvStages - 1);
             cp_async_wait<kKvStages - 1>();
             __syncwarp();
+            const uint32_t item = item_at(warp + kDW * t);
             if (item != kSkip) {
                 const uint32_t ks = smem_u32(wr + (size_t)(t % kKvStages) * SM::kStageBytes);
                 attend_block_swapped<D, 1>(st, qb, ks, ks + SM::kTileBytes, (int)(item & 15u) + 1,
@@ -629,225 +873,23 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             o0[D + 8] = st.o[t][0][3];
         }
     } else {
-        // ---- 4. control warps ----
+        // ---- 3'. the other warps: block list (ascending), count, errors ----
         const int ct = tid - kDW * 32;
-        if (appender) {
-            // decode-token append: K/V at position L-1, key folded into the
-            // current block's descriptor (a new block starts from the key)
-            const int slot = (L - 1) % kBlock;
-            if (app_page < 0 || app_page >= a.num_pages) {
-                if (lane == 0) set_error(a.err, RESA_DEVERR_PAGE);
-            } else {
-                constexpr int CPR = D / 8;
-                uint4 *K4 = reinterpret_cast<uint4 *>(a.k_cache);
-                uint4 *V4 = reinterpret_cast<uint4 *>(a.v_cache);
-                uint4 *D4 = reinterpret_cast<uint4 *>(a.desc);
-                for (int e = lane; e < CPR; e += 32) {
-                    const uint4 kx = a.k_new[((size_t)b * hkv + h) * CPR + e];
-                    const uint4 vx = a.v_new[((size_t)b * hkv + h) * CPR + e];
-                    const size_t o = (((size_t)app_page * hkv + h) * kBlock + slot) * CPR + e;
-                    K4[o] = kx;
-                    V4[o] = vx;
-                    uint4 *pmn = &D4[(((size_t)app_page * hkv + h) * 2) * CPR + e];
-                    uint4 *pmx = pmn + CPR;
-                    if (slot == 0) {
-                        *pmn = kx;
-                        *pmx = kx;
-                    } else {
-                        Bf16x8 mn = unpack8(*pmn), mx = unpack8(*pmx);
-                        fold8(mn, mx, unpack8(kx));
-                        *pmn = pack8(mn);
-                        *pmx = pack8(mx);
-                    }
-                }
-                __threadfence();
-            }
-        }
-        ctl_sync();
-        if (G > 1) {
-            if (ct == 0) {
-                __threadfence();
-                const uint32_t gen = unit_bar_arrive(&a.bars[2 * u + 1], G);
-                s_v[kVOk2] = unit_bar_wait(&a.bars[2 * u + 1], gen) ? 1 : 0;
-            }
-            ctl_sync();
-            __threadfence();
-        }
-        const bool ok2 = s_v[kVOk2] != 0;
-        if (!ok2 && ct == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
-        // Per-CTA counts of the unit -> prefix sums (one warp, <= 5 CTAs per lane).
-        if (ct < 32) {
-            const int PL = (G + 31) / 32;
-            const int i0 = ct * PL, i1 = min(G, i0 + PL);
-            int ndv[5], ncv[5];
-            int s_ov = 0, s_sp = 0, s_nc = 0, s_nd = 0;
-#pragma unroll
-            for (int r = 0; r < 5; ++r) {
-                const int i = i0 + r;
-                int2 c = make_int2(0, 0);
-                if (ok2 && r < PL && i < i1) c = __ldcg(&a.counts[u * G + i]);
-                ndv[r] = c.x;
-                ncv[r] = c.y;
-                if (r < PL && i < i1) {
-                    const int kp = min(c.x, F);
-                    s_ov += c.x - kp;
-                    s_sp += F - kp;
-                    s_nc += c.y;
-                    s_nd += c.x;
-                }
-            }
-            int e_ov = s_ov, e_sp = s_sp, e_nc = s_nc, e_nd = s_nd;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int a1 = __shfl_up_sync(0xffffffffu, e_ov, o);
-                const int a2 = __shfl_up_sync(0xffffffffu, e_sp, o);
-                const int a3 = __shfl_up_sync(0xffffffffu, e_nc, o);
-                const int a4 = __shfl_up_sync(0xffffffffu, e_nd, o);
-                if (ct >= o) {
-                    e_ov += a1;
-                    e_sp += a2;
-                    e_nc += a3;
-                    e_nd += a4;
-                }
-            }
-            int b_ov = e_ov - s_ov, b_sp = e_sp - s_sp, b_nc = e_nc - s_nc, b_nd = e_nd - s_nd;
-#pragma unroll
-            for (int r = 0; r < 5; ++r) {
-                const int i = i0 + r;
-                if (r < PL && i < i1) {
-                    if (i == x) {
-                        s_v[kVSpareBefore] = b_sp;
-                        s_v[kVDefBefore] = b_nd;
-                    }
-                    s_ovoff[i] = b_ov;
-                    s_coff[i] = b_nc;
-                    const int kp = min(ndv[r], F);
-                    b_ov += ndv[r] - kp;
-                    b_sp += F - kp;
-                    b_nc += ncv[r];
-                    b_nd += ndv[r];
-                }
-            }
-            if (ct == 31) {
-                s_ovoff[G] = e_ov;
-                s_coff[G] = e_nc;
-                s_v[kVOV] = e_ov;
-                s_v[kVNC] = e_nc;
-                s_v[kVAB] = e_nd;
-            }
-        }
-        ctl_sync();
-        const int OV = s_v[kVOV], NC = s_v[kVNC], AB = s_v[kVAB];
-        int rem = mode == kModeMid ? keff - AB : 0;
-        if (rem < 0 || rem > NC) {  // cannot happen with consistent counts
-            if (ct == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
-            rem = max(0, min(rem, NC));
-        }
-        const uint32_t *gcand = a.cand + (size_t)u * G * kStepMaxBlocks;
-        auto gkey = [&](int i) -> uint32_t {
-            const int src = upper_index(s_coff, G, i);
-            return __ldcg(&gcand[(size_t)src * kStepMaxBlocks + (i - s_coff[src])]);
-        };
-        const bool in_smem = NC <= kStepCandCap;
-        uint32_t tau = 0xffffffffu;
-        if (rem > 0) {
-            if (in_smem) {
-                for (int i0 = ct; i0 < NC; i0 += 4 * kCtlThreads) {
-                    uint32_t v[4];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int i = i0 + r * kCtlThreads;
-                        v[r] = i < NC ? gkey(i) : 0u;
-                    }
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int i = i0 + r * kCtlThreads;
-                        if (i < NC) cand_s[i] = v[r];
-                    }
-                }
-                ctl_sync();
-                tau = ctl_select_kth([&](int i) { return cand_s[i]; }, NC, (uint32_t)rem, ct, s_rh, s_rsh);
-            } else {
-                tau = ctl_select_kth(gkey, NC, (uint32_t)rem, ct, s_rh, s_rsh);
-            }
-        }
-        auto ckey = [&](int i) -> uint32_t { return in_smem ? cand_s[i] : gkey(i); };
-        // Residual pool: [overflow definite blocks, CTA order][qualifying
-        // candidates, candidate order][current block]; this CTA's slice.
-        const int Q = rem;
-        const int Rpool = seq_ok ? OV + Q + 1 : 0;
-        const int S0 = s_v[kVSpareBefore];
-        const int myspare = F - kept;
-        const int S1 = min(Rpool, S0 + myspare);
-        const int nres = max(0, S1 - S0);
-        auto page_item = [&](int blk, int ntok) -> uint32_t {
-            const int pg = a.page_table[prow + blk];
-            if (pg < 0 || pg >= a.num_pages) {
-                set_error(a.err, RESA_DEVERR_PAGE);
-                return kSkip;
-            }
-            return pack_item(pg, ntok);
-        };
-        for (int pos = S0 + ct; pos < min(S1, OV); pos += kCtlThreads) {
-            const int src = upper_index(s_ovoff, G, pos);
-            const int blk = __ldcg(&a.ovf[((size_t)u * G + src) * kStepMaxBlocks + (pos - s_ovoff[src])]);
-            res_item[pos - S0] = page_item(blk, kBlock);
-        }
-        if (seq_ok && ct == 0 && Rpool - 1 >= S0 && Rpool - 1 < S1)
-            res_item[Rpool - 1 - S0] = page_item(M, L - M * kBlock);
-        uint32_t qbefore_add = 0;
-        if (Q > 0) {
-            // qualifying candidates in array order: chunked scan of the flags
-            const int CH = (NC + kCtlThreads - 1) / kCtlThreads;
-            const int c0 = ct * CH, c1 = min(NC, c0 + CH);
-            uint32_t nq = 0;
-            for (int i = c0; i < c1; ++i) nq += ckey(i) >= tau;
-            uint32_t qtot;
-            uint32_t qp = ctl_scan(nq, ct, s_scan, qtot);
-            const int myc = s_coff[x];
-            for (int i = c0; i < c1; ++i) {
-                const uint32_t kk = ckey(i);
-                if (kk >= tau) {
-                    if (i < myc) ++qbefore_add;
-                    const int pos = OV + (int)qp;
-                    if (pos >= S0 && pos < S1) res_item[pos - S0] = page_item(0xffff - (int)(kk & 0xffffu), kBlock);
-                    ++qp;
-                }
-            }
-        }
-        if (ct == 0) s_v[kVQBefore] = 0;
-        ctl_sync();
-        if (qbefore_add) atomicAdd(&s_v[kVQBefore], (int)qbefore_add);
-        if (ct == 0) s_v[kVNres] = ok2 ? nres : 0;
-        ctl_sync();
-        if (ct == 0) mbar_arrive(&res_bar);  // the decode warps may take the residual slice
-
-        // Block list (ascending) and count.
-        const int off = s_v[kVDefBefore] + s_v[kVQBefore];
         int32_t *list = a.block_idx + (size_t)u * (a.max_topk + 1);
         {
             constexpr int R2 = (kStepMaxBlocks + kCtlThreads - 1) / kCtlThreads;
             const int i0 = ct * R2;
-            auto sel = [&](int i) -> bool {
-                if (mode == kModeAll) return true;
-                if (mode != kModeMid) return false;
-                const uint32_t key = keys[i];
-                const uint32_t dg = key >> 16;
-                if (dg != d1) return dg > d1;
-                return Q > 0 && (((key & 0xffffu) << 16) | (0xffffu - (uint32_t)(p0 + i))) >= tau;
-            };
             uint32_t ns = 0;
             for (int r = 0; r < R2; ++r) {
                 const int i = i0 + r;
-                if (i < nmine && sel(i)) ++ns;
+                if (i < nmine && (own_def(i) || own_qual(i))) ++ns;
             }
             uint32_t tot;
-            uint32_t pos = ctl_scan(ns, ct, s_scan, tot) + (uint32_t)off;
-            if (ok2)
-                for (int r = 0; r < R2; ++r) {
-                    const int i = i0 + r;
-                    if (i < nmine && sel(i) && pos < (uint32_t)keff) list[pos++] = p0 + i;
-                }
+            uint32_t pos = ctl_scan(ns, ct, s_scan, tot) + (uint32_t)s_v[kVSelBefore];
+            for (int r = 0; r < R2; ++r) {
+                const int i = i0 + r;
+                if (i < nmine && (own_def(i) || own_qual(i)) && pos < (uint32_t)keff) list[pos++] = p0 + i;
+            }
         }
         if (x == 0 && ct == 0) {
             if (seq_ok) {
@@ -859,9 +901,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             }
             if (topk_err) set_error(a.err, RESA_DEVERR_TOPK);
         }
-        if (x == 0 && need_hist) {
-            // every CTA of the unit read the histogram before the second
-            // barrier: leave it clear for the next call
+        if (G == 1 && need_hist) {
+            // the only CTA of the unit has read the histogram: clear it
             uint32_t *hb = a.hist + (size_t)u * kHistBins;
             for (int d = s_v[kVDlo] + ct; d <= s_v[kVDhi]; d += kCtlThreads) hb[d] = 0;
             if (ct == 0) {
@@ -872,7 +913,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     __syncthreads();  // warp states are in shared memory
 
-    // ---- 5. merge the warps, then the unit's CTAs ----
+    // ---- 4. merge the warps, then the unit's CTAs ----
     const float kLn2 = 0.6931471805599453f;
     {
         const float *mw = reinterpret_cast<const float *>(ring);
@@ -908,81 +949,86 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
     }
     if (G == 1) return;
+    // The unit's G partials are merged by slices: item (row r, 32 channels)
+    // goes to CTA item % G, after a second unit barrier.  CTAs without an item
+    // arrive and leave.
+    constexpr int C32 = D / 32;
+    const int n_items = g * C32;
+    const bool merger = x < n_items;
     __threadfence();
     __syncthreads();
     if (tid == 0) {
-        const uint32_t t = atomicAdd(&a.tickets[u], 1u);
-        s_v[kVLast] = t == (uint32_t)(G - 1) ? 1 : 0;
+        const uint32_t gen = unit_bar_arrive(&a.bars[2 * u + 1], G);
+        s_v[kVOk3] = merger ? (unit_bar_wait(&a.bars[2 * u + 1], gen) ? 1 : 0) : 1;
     }
     __syncthreads();
-    if (!s_v[kVLast]) return;
+    if (!merger) return;
+    if (!s_v[kVOk3]) {
+        if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
+        return;
+    }
     __threadfence();
-    // The last CTA of the unit: weights from the G partial log-sum-exps, then
-    // the weighted sum of the partial outputs, pulled into shared memory with
-    // cp.async in chunks of as many partials as the rings hold.
-    float *wts = reinterpret_cast<float *>(ring);  // [G][kStepMaxGroup]
-    const size_t wbytes = ((size_t)G * kStepMaxGroup * 4 + 127) / 128 * 128;
-    const float *ul = a.part_lse + (size_t)u * G * kMaxGroup;
-    for (int i = tid; i < G * g; i += kThreadsAll) {
-        const int s = i / g, r = i % g;
-        wts[s * kStepMaxGroup + r] = __ldcg(&ul[s * kMaxGroup + r]);
+    if (x == 0 && need_hist) {
+        // every CTA of the unit read the histogram before this barrier: leave
+        // it clear for the next call
+        uint32_t *hb = a.hist + (size_t)u * kHistBins;
+        for (int d = s_v[kVDlo] + tid; d <= s_v[kVDhi]; d += kThreadsAll) hb[d] = 0;
+        if (tid == 0) {
+            a.hist_range[2 * u] = 0;
+            a.hist_range[2 * u + 1] = 0;
+        }
     }
-    __syncthreads();
-    for (int r = warp; r < g; r += kWarpsAll) {
+    const float *ul = a.part_lse + (size_t)u * G * kMaxGroup;
+    const float *uo = a.part_o + (size_t)u * G * kStepMaxGroup * D;
+    constexpr int kPW = (kNumSms + kWarpsAll - 1) / kWarpsAll;  // partials per warp
+    constexpr int kPL = (kNumSms + 31) / 32;                     // log-sum-exps per lane
+    float *red = reinterpret_cast<float *>(ring);                // [kWarpsAll][33]
+    for (int item = x; item < n_items; item += G) {
+        const int r = item / C32, cc = item % C32;
+        // every load of the item in flight at once: this warp's partials
+        // (warp, warp + 12, ...) and every partial's log2-sum-exp
+        float v[kPW], lv[kPW], la[kPL];
+#pragma unroll
+        for (int k = 0; k < kPW; ++k) {
+            const int sp = warp + kWarpsAll * k;
+            v[k] = sp < G ? __ldcg(&uo[((size_t)sp * kStepMaxGroup + r) * D + cc * 32 + lane]) : 0.f;
+            lv[k] = sp < G ? __ldcg(&ul[sp * kMaxGroup + r]) : -INFINITY;
+        }
         float mstar = -INFINITY;
-        for (int s = lane; s < G; s += 32) mstar = fmaxf(mstar, wts[s * kStepMaxGroup + r]);
+#pragma unroll
+        for (int k = 0; k < kPL; ++k) {
+            const int sp = lane + 32 * k;
+            la[k] = sp < G ? __ldcg(&ul[sp * kMaxGroup + r]) : -INFINITY;
+            mstar = fmaxf(mstar, la[k]);
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
-        float sum = 0.f;
-        if (mstar != -INFINITY)
-            for (int s = lane; s < G; s += 32) sum += exp2f(wts[s * kStepMaxGroup + r] - mstar);
+        float lsum = 0.f, acc = 0.f;
+        if (mstar != -INFINITY) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        __syncwarp();
-        for (int s = lane; s < G; s += 32)
-            wts[s * kStepMaxGroup + r] = sum > 0.f ? exp2f(wts[s * kStepMaxGroup + r] - mstar) / sum : 0.f;
-        if (lane == 0) s_lse[r] = sum > 0.f ? mstar + log2f(sum) : -INFINITY;
-    }
-    __syncthreads();
-    uint8_t *tiles = ring + wbytes;
-    const int tile_bytes = g * D * 4;
-    const int chunk = max(1, (int)((SM::kRingBytes - wbytes) / tile_bytes));
-    const float *uo = a.part_o + (size_t)u * G * kStepMaxGroup * D;
-    constexpr int C4 = D / 4;
-    const int items = g * C4;  // float4 columns of the g rows
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int item = tid;      // g * D / 4 <= 8 * 32 < kThreadsAll
-    for (int s0 = 0; s0 < G; s0 += chunk) {
-        const int s1 = min(G, s0 + chunk);
-        const int n16 = (s1 - s0) * items;  // 16-byte pieces
-        for (int i = tid; i < n16; i += kThreadsAll) {
-            const int s = s0 + i / items, k = i % items;
-            cp_async16(tiles + (size_t)i * 16, uo + (size_t)s * kStepMaxGroup * D + (size_t)k * 4);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncthreads();
-        if (item < items) {
-            const int r = item / C4;
-            const float4 *tf = reinterpret_cast<const float4 *>(tiles);
-            for (int s = s0; s < s1; ++s) {
-                const float w = wts[s * kStepMaxGroup + r];
-                const float4 v = tf[(size_t)(s - s0) * items + item];
-                acc.x += w * v.x;
-                acc.y += w * v.y;
-                acc.z += w * v.z;
-                acc.w += w * v.w;
+            for (int k = 0; k < kPW; ++k) {
+                const float wk = exp2f(lv[k] - mstar);
+                lsum += wk;
+                acc += wk * v[k];
             }
         }
+        red[warp * 33 + lane] = acc;
+        if (lane == 0) red[warp * 33 + 32] = lsum;
+        __syncthreads();
+        if (warp == 0) {
+            float o = 0.f, lt = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarpsAll; ++w) {
+                o += red[w * 33 + lane];
+                lt += red[w * 33 + 32];
+            }
+            const size_t orow = (size_t)b * hkv * g + (size_t)h * g + r;
+            a.out[orow * D + cc * 32 + lane] = lt > 0.f ? o / lt : 0.f;
+            if (a.lse && cc == 0 && lane == 0)
+                a.lse[orow] = (lt > 0.f ? mstar + log2f(lt) : -INFINITY) * kLn2;
+        }
         __syncthreads();
     }
-    if (item < items) {
-        const int r = item / C4, c4 = item % C4;
-        const size_t orow = (size_t)b * hkv * g + (size_t)h * g + r;
-        reinterpret_cast<float4 *>(a.out + orow * D)[c4] = acc;
-        if (a.lse && c4 == 0) a.lse[orow] = s_lse[r] * kLn2;
-    }
-    if (tid == 0) a.tickets[u] = 0;
 }
 
 }  // namespace
@@ -1009,10 +1055,7 @@ cudaError_t launch_decode_step_fused(const Shape &s, int G, void *k, void *v, vo
     a.hist = buf.hist;
     a.hist_range = buf.hist_range;
     a.bars = buf.bars;
-    a.tickets = buf.tickets;
-    a.counts = buf.counts;
-    a.ovf = buf.ovf;
-    a.cand = buf.cand;
+    a.ukeys = buf.ukeys;
     a.part_o = buf.part_o;
     a.part_lse = buf.part_lse;
     a.err = buf.err;
@@ -1021,6 +1064,7 @@ cudaError_t launch_decode_step_fused(const Shape &s, int G, void *k, void *v, vo
     a.max_pages = s.max_pages;
     a.num_pages = s.num_pages;
     a.max_topk = max_topk;
+    a.key_stride = step_key_stride(s.max_pages);
     a.scale_log2 = s.sm_scale * 1.4426950408889634f;
 
     cudaLaunchConfig_t cfg = {};
