@@ -59,11 +59,13 @@ inline int decode_max_splits(int batch, int hkv, int max_pages) {
 // max_pages <= 65536.
 constexpr int kStepMaxBlocks = 1024;
 constexpr int kStepMaxPages = 65536;
-// After scoring, every CTA of the fused step holds its unit's keys and the
-// boundary candidates (at most as many) in its K/V rings (8 warps x 3 stages
-// x a 16-token K and V tile): at most this many keys.
+// After scoring, every CTA of the fused step holds its unit's keys, page ids
+// and boundary candidates (12 warps x 512 at most) in its K/V rings (8 warps x
+// 3 stages x a 16-token K and V tile): at most this many complete blocks.
 constexpr int step_unit_keys(int d) {
-    return kDecodeWarps * 3 * 2 * kBlock * d * 2 / 8 - 1024 < 32768 ? kDecodeWarps * 3 * 2 * kBlock * d * 2 / 8 - 1024 : 32768;
+    return (kDecodeWarps * 3 * 2 * kBlock * d * 2 - 12 * 512 * 4 - 64) / 8 < 32768
+               ? (kDecodeWarps * 3 * 2 * kBlock * d * 2 - 12 * 512 * 4 - 64) / 8
+               : 32768;
 }
 // Row stride (in keys) of a unit's key row in the workspace: 16-byte rows.
 inline int step_key_stride(int max_pages) { return (max_pages + 3) & ~3; }
@@ -308,6 +310,11 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// 4-byte asynchronous copy (through L1) for unaligned tails.
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");

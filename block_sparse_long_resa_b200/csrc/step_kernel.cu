@@ -52,9 +52,10 @@ constexpr int kKvStages = 3;
 constexpr int kScoreSlots = 4;            // descriptor ring slots per warp (8 blocks each)
 constexpr int kScoreBlocks = 8;           // blocks per warp step of the scoring loop
 constexpr int kHash = 1024;               // per-CTA digit histogram slots
+constexpr int kMaxGroups = kHash;         // 32-block groups of a unit (group counts in the hash area)
+constexpr int kCandPerWarp = 512;         // candidate segment of a warp
 constexpr uint32_t kHashEmpty = 0xffffffffu;
 constexpr uint32_t kSkip = 0xffffffffu;   // work item without data (bad page id)
-constexpr uint32_t kLookup = 0x80000000u; // work entry holding a block id (page not yet read)
 constexpr int kModeAll = 0, kModeNone = 1, kModeMid = 2;
 
 template <int D>
@@ -66,12 +67,14 @@ struct StepSmem {
     static constexpr int kSlotBytes = kScoreBlocks * kDescBytes;
     static_assert(kWarpsAll * kScoreSlots * kSlotBytes <= kRingBytes, "score rings fit the K/V rings");
     static_assert(kDW * kMaxGroup * (D + 2) * 4 <= kRingBytes, "warp states fit the rings");
-    static_assert(step_unit_keys(D) * 4 <= kRingBytes, "the unit's keys and candidates fit the rings");
+    static_assert(step_unit_keys(D) * 8 + kWarpsAll * kCandPerWarp * 4 + 64 <= kRingBytes,
+                  "the unit's keys, page ids and candidates fit the rings");
+    static_assert(step_unit_keys(D) <= kMaxGroups * 32, "group counts fit the hash area");
     static constexpr int kKeysOff = kRingBytes;                      // u32 [kStepMaxBlocks] own keys
     static constexpr int kPagesOff = kKeysOff + kStepMaxBlocks * 4;  // i32 [kStepMaxBlocks] own pages
-    static constexpr int kItemOff = kPagesOff + kStepMaxBlocks * 4;  // u32 [kStepMaxBlocks] own work
-    static constexpr int kResCap = kStepMaxBlocks + 8;
-    static constexpr int kResOff = kItemOff + kStepMaxBlocks * 4;    // u32 [kResCap] the rest
+    static constexpr int kResCap = kStepMaxBlocks + 8;               // this CTA's items: at most F
+    static constexpr int kItemOff = kPagesOff + kStepMaxBlocks * 4;  // u32 [kResCap] their block ids
+    static constexpr int kResOff = kItemOff + kResCap * 4;           // u32 [kResCap] (page, tokens) items
     static constexpr int kHashOff = kResOff + kResCap * 4;           // u32 [2][kHash]
     static constexpr int kBytes = kHashOff + 2 * kHash * 4 + 128;    // + base alignment
 };
@@ -135,40 +138,6 @@ __device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t *tmp, uint32_t
     return before + incl - v;
 }
 
-// The same over the last kCW warps (ct = thread index within them).
-__device__ __forceinline__ uint32_t ctl_scan(uint32_t v, int ct, uint32_t *tmp, uint32_t &total) {
-    const int lane = ct & 31, w = ct >> 5;
-    uint32_t incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) tmp[w] = incl;
-    asm volatile("bar.sync 1, %0;" ::"r"(kCtlThreads) : "memory");
-    uint32_t before = 0, tot = 0;
-#pragma unroll
-    for (int i = 0; i < kCW; ++i) {
-        const uint32_t t = tmp[i];
-        before += i < w ? t : 0u;
-        tot += t;
-    }
-    total = tot;
-    asm volatile("bar.sync 1, %0;" ::"r"(kCtlThreads) : "memory");
-    return before + incl - v;
-}
-
-// Largest i in [0, n) with a[i] <= v (a ascending, a[0] <= v).
-__device__ __forceinline__ int upper_index(const int *a, int n, int v) {
-    int lo = 0, hi = n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a[mid] <= v) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
 __device__ __forceinline__ uint32_t item_of_page(int page, int num_pages, int ntok) {
     return (page >= 0 && page < num_pages) ? (((uint32_t)page << 4) | (uint32_t)(ntok - 1)) : kSkip;
 }
@@ -181,8 +150,7 @@ __device__ __forceinline__ uint32_t composite(uint32_t k, int i) {
 
 // Indices of the small shared values.
 enum {
-    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVOk3, kVLo, kVHi, kVAB, kVSpareBefore,
-    kVSelBefore, kVCount
+    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVOk3, kVLo, kVHi, kVAB, kVCount
 };
 
 template <int D>
@@ -201,7 +169,6 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     uint32_t *hkey = reinterpret_cast<uint32_t *>(smem + SM::kHashOff), *hcnt = hkey + kHash;
 
     __shared__ float qbar_s[D];
-    __shared__ int s_nd[kNumSms], s_q[kNumSms], s_poff[kNumSms + 1];
     __shared__ uint32_t s_rh[256];
     __shared__ uint32_t s_scan[kWarpsAll];
     __shared__ uint32_t s_rsh[3];
@@ -245,10 +212,6 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     for (int i = tid; i < kHash; i += kThreadsAll) {
         hkey[i] = kHashEmpty;
         hcnt[i] = 0;
-    }
-    for (int i = tid; i < G; i += kThreadsAll) {
-        s_nd[i] = 0;
-        s_q[i] = 0;
     }
     if (tid == 0) {
         s_v[kVOk] = 1;
@@ -458,14 +421,29 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
         __threadfence();
     }
-    uint32_t d1 = 0;
-    if (need_hist) {
-        // One round trip in the common case: every key of the unit (into the
-        // idle K/V ring), the touched range and a window of kThreadsAll bins
-        // below (this CTA's top digit + 128); the whole touched range is read
-        // only when the window does not hold it.
-        for (int c = tid; c < (M + 3) / 4; c += kThreadsAll) cp_async16(ukeys_s + 4 * c, ukeys_g + 4 * c);
+    // ---- 2'. in one round trip: the unit's keys and page ids (into the idle
+    // K/V rings) and the histogram around this CTA's own top digit ----
+    // page id of block i at upages_s[i + pshift]: the row is copied from the
+    // 16-byte boundary at or below its start; the tail (inside the row) with
+    // 4-byte copies
+    uint32_t *upages_s = ukeys_s + ((M + 3) & ~3);
+    const int pshift = (int)(prow & 3);
+    if (mode == kModeAll || mode == kModeMid) {
+        if (mode == kModeMid)
+            for (int c = tid; c < (M + 3) / 4; c += kThreadsAll) cp_async16(ukeys_s + 4 * c, ukeys_g + 4 * c);
+        const int32_t *prow_al = a.page_table + (prow - pshift);
+        const int nfull = (M + pshift) / 4;
+        for (int c = tid; c < nfull; c += kThreadsAll) cp_async16(upages_s + 4 * c, prow_al + 4 * c);
+        for (int e = 4 * nfull + tid; e < M + pshift; e += kThreadsAll) cp_async4(upages_s + e, prow_al + e);
         cp_async_commit();
+    }
+    auto page_of = [&](int blk) -> int { return (int)upages_s[blk + pshift]; };
+    uint32_t d1 = 0;
+    int above = 0;
+    if (need_hist) {
+        // a window of kThreadsAll bins below (this CTA's top digit + 128) and
+        // the touched range; the whole range is read only when the window
+        // does not hold it
         const uint32_t *hb = a.hist + (size_t)u * kHistBins;
         const int wtop = min(kHistBins - 1, s_v[kVHi] + 128);
         const int wbot = max(0, wtop - (kThreadsAll - 1));
@@ -495,6 +473,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                 const uint32_t c = covered ? wc : __ldcg(&hb[d]);
                 if (cum + c >= (uint32_t)keff) {
                     s_v[kVD1] = d;
+                    s_v[kVAB] = (int)cum;  // keys above the boundary digit
                     break;
                 }
                 cum += c;
@@ -505,8 +484,10 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             s_v[kVDhi] = dhi;
             s_v[kVHistOk] = total == (uint32_t)M ? 1 : 0;
         }
-        cp_async_wait<0>();
-        __syncthreads();
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (need_hist) {
         if (!s_v[kVHistOk]) {
             // The histogram was not clean at entry (an earlier call gave up
             // mid-way): every CTA of the unit sees the same sums and selects
@@ -516,19 +497,28 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             keff = 0;
         }
         d1 = (uint32_t)s_v[kVD1];
+        above = s_v[kVAB];
     }
-    const int F = ((seq_ok ? keff + 1 : 0) + G - 1) / G;
-    // Per-CTA counts from the unit's keys, branch-free: each warp takes 32-key
-    // groups (one key a lane, four groups in flight), records the ballots of
-    // the definite keys and of the candidates per group, and appends the
-    // candidates' composite keys to its own segment of the list after the keys.
+    // Work split: the unit's ordered work list is the selected blocks in
+    // ascending order, then the current block (W = keff + 1 items); CTA x
+    // takes items [x*F, (x+1)*F).
+    const int W = seq_ok ? keff + 1 : 0;
+    const int F = (W + G - 1) / G;
+    const int s0 = min(W, x * F), s1 = min(W, s0 + F);
+    const int n_items = s1 - s0;
+    int *gcnt = reinterpret_cast<int *>(hkey), *gpre = reinterpret_cast<int *>(hcnt);  // [ngroups]
     const int ngroups = (M + 31) >> 5;
-    const int KW = (ngroups + kWarpsAll - 1) / kWarpsAll * 32;  // keys one warp sees at most
-    uint32_t *cand_s = ukeys_s + ((M + 3) & ~3);                // [kWarpsAll][KW]
-    uint32_t *defm = hkey, *candm = hcnt;                       // [ngroups] (hash area, free now)
+    uint32_t tau = 0xffffffffu;
+    int rem = 0;
     if (mode == kModeMid) {
+        // One pass over the unit's keys, a 32-block group per warp step (one
+        // key a lane, four groups in flight): the definite count of each group
+        // and the candidates' composite keys, appended to the warp's segment.
+        const int KW = (ngroups + kWarpsAll - 1) / kWarpsAll * 32;  // keys one warp sees at most
+        uint32_t *cand_s = upages_s + ((M + pshift + 3) & ~3);      // [kWarpsAll][min(KW, cap)]
+        const int cap = min(KW, kCandPerWarp);
         const uint32_t lt_mask = (1u << lane) - 1u;
-        uint32_t *seg = cand_s + warp * KW;
+        uint32_t *seg = cand_s + warp * cap;
         int nseg = 0;
         for (int g0 = warp; g0 < ngroups; g0 += 4 * kWarpsAll) {
             uint32_t kk[4];
@@ -545,278 +535,169 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                 const bool isc = i < M && dg == d1;
                 const uint32_t bd = __ballot_sync(0xffffffffu, i < M && dg > d1);
                 const uint32_t bc = __ballot_sync(0xffffffffu, isc);
-                if (lane == 0 && grp < ngroups) {
-                    defm[grp] = bd;
-                    candm[grp] = bc;
-                }
-                if (isc) seg[nseg + __popc(bc & lt_mask)] = composite(kk[u4], i);
+                if (lane == 0 && grp < ngroups) gcnt[grp] = __popc(bd);
+                const int r = nseg + __popc(bc & lt_mask);
+                if (isc && r < cap) seg[r] = composite(kk[u4], i);
                 nseg += __popc(bc);
             }
         }
         if (lane == 0) s_seg[warp] = nseg;
-    }
-    __syncthreads();
-    // definite blocks per CTA range: popcounts of the ballots, a warp per range
-    if (mode == kModeMid) {
-        for (int src = warp; src < G; src += kWarpsAll) {
-            const int b0 = min(M, src * per), b1 = min(M, b0 + per);
-            int cnt = 0;
-            if (b1 > b0)
-                for (int gi = (b0 >> 5) + lane; gi <= ((b1 - 1) >> 5); gi += 32) {
-                    const int lo = max(b0, gi * 32) - gi * 32, hi = min(b1, gi * 32 + 32) - gi * 32;
-                    const uint32_t rm = (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~((1u << lo) - 1u);
-                    cnt += __popc(defm[gi] & rm);
-                }
+        __syncthreads();
+        // exact threshold: the rem-th largest candidate composite by radix
+        // select, stopping at the first digit whose bin is taken whole
+        int seg_end[kWarpsAll];
+        bool fits = true;
+        {
+            int acc = 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-            if (lane == 0) s_nd[src] = cnt;
-        }
-    } else if (mode == kModeAll) {
-        for (int i = tid; i < G; i += kThreadsAll) s_nd[i] = max(0, min(M, (i + 1) * per) - min(M, i * per));
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int ab = 0;
-        for (int i = lane; i < G; i += 32) ab += s_nd[i];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ab += __shfl_xor_sync(0xffffffffu, ab, o);
-        if (lane == 0) s_v[kVAB] = ab;
-    }
-    __syncthreads();
-    // exact threshold: radix select over the candidates' composite keys,
-    // stopping at the first digit whose bin is taken whole
-    // candidate f of the list: segment w = the first with f < its end
-    int seg_end[kWarpsAll];
-    {
-        int acc = 0;
-#pragma unroll
-        for (int w = 0; w < kWarpsAll; ++w) {
-            acc += mode == kModeMid ? s_seg[w] : 0;
-            seg_end[w] = acc;
-        }
-    }
-    const int NC = seg_end[kWarpsAll - 1];
-    auto cand_at = [&](int f) -> uint32_t {
-        int w = 0, start = 0;
-#pragma unroll
-        for (int k = 0; k < kWarpsAll - 1; ++k)
-            if (f >= seg_end[k]) {
-                w = k + 1;
-                start = seg_end[k];
+            for (int w = 0; w < kWarpsAll; ++w) {
+                fits = fits && s_seg[w] <= cap;
+                acc += s_seg[w];
+                seg_end[w] = acc;
             }
-        return cand_s[w * KW + (f - start)];
-    };
-    int rem = mode == kModeMid ? keff - s_v[kVAB] : 0;
-    if (rem < 0) {  // cannot happen with consistent counts
-        if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
-        rem = 0;
-    }
-    uint32_t tau = 0xffffffffu;
-    if (rem > 0) {
-        uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)rem;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += kThreadsAll) s_rh[i] = 0;
-            __syncthreads();
-            for (int i = tid; i < NC; i += kThreadsAll) {
-                const uint32_t c = cand_at(i);
-                if ((c & pmask) == prefix) atomicAdd(&s_rh[(c >> shift) & 255u], 1u);
+        }
+        const int NC = seg_end[kWarpsAll - 1];
+        // candidate f of the list (segments in warp order); when a segment
+        // overflowed, candidates are found by scanning the keys instead
+        auto for_each_cand = [&](auto fn) {
+            if (fits) {
+                for (int f = tid; f < NC; f += kThreadsAll) {
+                    int w = 0, st0 = 0;
+#pragma unroll
+                    for (int k2 = 0; k2 < kWarpsAll - 1; ++k2)
+                        if (f >= seg_end[k2]) {
+                            w = k2 + 1;
+                            st0 = seg_end[k2];
+                        }
+                    fn(cand_s[w * cap + (f - st0)]);
+                }
+            } else {
+                for (int i = tid; i < M; i += kThreadsAll) {
+                    const uint32_t k = ukeys_s[i];
+                    if ((k >> 16) == d1) fn(composite(k, i));
+                }
             }
-            __syncthreads();
-            if (warp == 0) {
-                // lane l holds digits 255 - 8l - j, j = 0..7 (descending)
-                uint32_t cnt[8], sum = 0;
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    cnt[jj] = s_rh[255 - 8 * lane - jj];
-                    sum += cnt[jj];
-                }
-                uint32_t incl = sum;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += t;
-                }
-                uint32_t cum = incl - sum;
-                if (cum < remaining && remaining <= incl) {
+        };
+        rem = keff - above;
+        if (rem < 1 || rem > NC) {  // cannot happen with consistent counts
+            if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
+            rem = max(0, min(rem, NC));
+        }
+        if (rem > 0) {
+            uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)rem;
+            for (int shift = 24; shift >= 0; shift -= 8) {
+                for (int i = tid; i < 256; i += kThreadsAll) s_rh[i] = 0;
+                __syncthreads();
+                for_each_cand([&](uint32_t c) {
+                    if ((c & pmask) == prefix) atomicAdd(&s_rh[(c >> shift) & 255u], 1u);
+                });
+                __syncthreads();
+                if (warp == 0) {
+                    // lane l holds digits 255 - 8l - j, j = 0..7 (descending)
+                    uint32_t cnt[8], sum = 0;
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj) {
-                        if (cum < remaining && remaining <= cum + cnt[jj]) {
-                            s_rsh[0] = 255u - 8u * lane - jj;
-                            s_rsh[1] = cum;
-                            s_rsh[2] = cnt[jj];
+                        cnt[jj] = s_rh[255 - 8 * lane - jj];
+                        sum += cnt[jj];
+                    }
+                    uint32_t incl = sum;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += t;
+                    }
+                    uint32_t cum = incl - sum;
+                    if (cum < remaining && remaining <= incl) {
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj) {
+                            if (cum < remaining && remaining <= cum + cnt[jj]) {
+                                s_rsh[0] = 255u - 8u * lane - jj;
+                                s_rsh[1] = cum;
+                                s_rsh[2] = cnt[jj];
+                            }
+                            cum += cnt[jj];
                         }
-                        cum += cnt[jj];
                     }
                 }
+                __syncthreads();
+                remaining -= s_rsh[1];
+                prefix |= s_rsh[0] << shift;
+                pmask |= 255u << shift;
+                if (remaining == s_rsh[2]) break;  // every key with this prefix is taken
             }
-            __syncthreads();
-            remaining -= s_rsh[1];
-            prefix |= s_rsh[0] << shift;
-            pmask |= 255u << shift;
-            if (remaining == s_rsh[2]) break;  // every key with this prefix is taken
+            tau = prefix;
+            // the qualifying candidates join their groups' counts
+            for_each_cand([&](uint32_t c) {
+                if (c >= tau) atomicAdd(&gcnt[(int)(0xffffu - (c & 0xffffu)) >> 5], 1);
+            });
         }
-        tau = prefix;
-        // qualifying candidates per CTA
-        for (int i = tid; i < NC; i += kThreadsAll) {
-            const uint32_t c = cand_at(i);
-            if (c >= tau) atomicAdd(&s_q[(int)(0xffffu - (c & 0xffffu)) / per], 1);
-        }
-    }
-    __syncthreads();
-    // canonical work layout: CTA x' keeps its own selected blocks (definite,
-    // then qualifying, each in block order) up to F; the rest is the pool (CTA
-    // order, then the current block); CTA x takes the slice of the pool after
-    // the spare capacity of the CTAs before it
-    if (warp == 0) {
-        const int PL = (G + 31) / 32;
-        const int i0 = lane * PL;
-        int sp = 0, pl = 0, ss = 0;
-        for (int r = 0; r < PL; ++r) {
-            const int i = i0 + r;
-            if (i < G) {
-                const int sel = s_nd[i] + s_q[i];
-                sp += F - min(sel, F);
-                pl += sel - min(sel, F);
-                ss += sel;
-            }
-        }
-        int ep = sp, el = pl, es = ss;
+        __syncthreads();
+        // exclusive prefix of the selected count over the groups
+        {
+            constexpr int RG = (kMaxGroups + kThreadsAll - 1) / kThreadsAll;
+            const int q0 = tid * RG;
+            int v[RG];
+            uint32_t sum = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t1 = __shfl_up_sync(0xffffffffu, ep, o);
-            const int t2 = __shfl_up_sync(0xffffffffu, el, o);
-            const int t3 = __shfl_up_sync(0xffffffffu, es, o);
-            if (lane >= o) {
-                ep += t1;
-                el += t2;
-                es += t3;
+            for (int r = 0; r < RG; ++r) {
+                v[r] = q0 + r < ngroups ? gcnt[q0 + r] : 0;
+                sum += v[r];
             }
-        }
-        int bp = ep - sp, bl = el - pl, bs = es - ss;
-        for (int r = 0; r < PL; ++r) {
-            const int i = i0 + r;
-            if (i < G) {
-                if (i == x) {
-                    s_v[kVSpareBefore] = bp;
-                    s_v[kVSelBefore] = bs;
-                }
-                s_poff[i] = bl;
-                const int sel = s_nd[i] + s_q[i];
-                bp += F - min(sel, F);
-                bl += sel - min(sel, F);
-                bs += sel;
-            }
-        }
-        if (lane == 31) s_poff[G] = el;
-    }
-    __syncthreads();
-    const int nd = s_nd[x], myq = s_q[x];
-    const int kept_def = min(nd, F);
-    const int qkeep = max(0, min(myq, F - nd));  // own qualifying candidates kept
-    const int pool = seq_ok ? s_poff[G] + 1 : 0;
-    const int S0 = s_v[kVSpareBefore];
-    const int S1 = min(pool, S0 + (F - min(nd + myq, F)));
-    const int nslice = max(0, S1 - S0);
-    const int n_res = qkeep + nslice;
-    // Is own block i (local index) definite / a qualifying candidate?
-    auto own_def = [&](int i) -> bool {
-        return mode == kModeAll || (mode == kModeMid && (keys[i] >> 16) > d1);
-    };
-    auto own_qual = [&](int i) -> bool {
-        const uint32_t k = keys[i];
-        return rem > 0 && (k >> 16) == d1 && composite(k, p0 + i) >= tau;
-    };
-    {
-        // own definite blocks in block order (this CTA keeps the first F) and
-        // the first qkeep own qualifying candidates
-        constexpr int R1 = (kStepMaxBlocks + kThreadsAll - 1) / kThreadsAll;
-        const int j0 = tid * R1;
-        uint32_t nd_t = 0, nq_t = 0;
+            uint32_t tot;
+            uint32_t run = cta_scan(sum, s_scan, tot);
 #pragma unroll
-        for (int r = 0; r < R1; ++r) {
-            const int i = j0 + r;
-            if (i < nmine) {
-                nd_t += own_def(i);
-                nq_t += own_qual(i);
-            }
-        }
-        uint32_t tot;
-        const uint32_t ex = cta_scan(nd_t | (nq_t << 16), s_scan, tot);
-        uint32_t od = ex & 0xffffu, oq = ex >> 16;
-#pragma unroll
-        for (int r = 0; r < R1; ++r) {
-            const int i = j0 + r;
-            if (i < nmine) {
-                if (own_def(i)) {
-                    if ((int)od < F) own_item[od] = item_of_page(pages[i], a.num_pages, kBlock);
-                    ++od;
-                } else if (own_qual(i)) {
-                    if ((int)oq < qkeep) res_item[oq] = item_of_page(pages[i], a.num_pages, kBlock);
-                    ++oq;
-                }
-            }
-        }
-    }
-    // the slice [S0, S1) of the pool: per source CTA, its definite blocks
-    // past F, then its qualifying candidates past its kept ones, block order
-    if (nslice > 0) {
-        const int last = pool - 1;  // the current block
-        if (tid == 0 && last >= S0 && last < S1)
-            res_item[qkeep + last - S0] = item_of_page(cur_page, a.num_pages, L - M * kBlock);
-        const int s_hi_pos = min(S1, last) - 1;  // last pool position of a source CTA in the slice
-        if (mode == kModeMid && s_hi_pos >= S0) {
-            const int s_lo = upper_index(s_poff, G, S0), s_hi = upper_index(s_poff, G, s_hi_pos);
-            const uint32_t lt_mask = (1u << lane) - 1u;
-            for (int src = s_lo + warp; src <= s_hi; src += kWarpsAll) {
-                const int ovd = max(0, s_nd[src] - F);
-                const int keepq = max(0, min(s_q[src], F - s_nd[src]));
-                const int base = s_poff[src];
-                const int b0 = min(M, src * per), b1 = min(M, b0 + per);
-                int def_seen = 0, q_seen = 0;
-                for (int c0 = b0; c0 < b1; c0 += 32) {
-                    const int i = c0 + lane;
-                    const uint32_t k = i < b1 ? ukeys_s[i] : 0u;
-                    const bool isd = i < b1 && (k >> 16) > d1;
-                    const bool isq = i < b1 && rem > 0 && (k >> 16) == d1 && composite(k, i) >= tau;
-                    const uint32_t bd = __ballot_sync(0xffffffffu, isd);
-                    const uint32_t bq = __ballot_sync(0xffffffffu, isq);
-                    if (isd) {
-                        const int rank = def_seen + __popc(bd & lt_mask);
-                        const int pos = base + rank - F;
-                        if (rank >= F && pos >= S0 && pos < S1) res_item[qkeep + pos - S0] = kLookup | (uint32_t)i;
-                    }
-                    if (isq) {
-                        const int rank = q_seen + __popc(bq & lt_mask);
-                        const int pos = base + ovd + rank - keepq;
-                        if (rank >= keepq && pos >= S0 && pos < S1) res_item[qkeep + pos - S0] = kLookup | (uint32_t)i;
-                    }
-                    def_seen += __popc(bd);
-                    q_seen += __popc(bq);
-                }
+            for (int r = 0; r < RG; ++r) {
+                if (q0 + r < ngroups) gpre[q0 + r] = (int)run;
+                run += v[r];
             }
         }
         __syncthreads();
-        // page ids of the pool blocks (other CTAs' ranges): one round trip
-        for (int r = qkeep + tid; r < n_res; r += kThreadsAll) {
-            const uint32_t v = res_item[r];
-            if ((v & 0xffff0000u) == kLookup)
-                res_item[r] = item_of_page(a.page_table[prow + (v & 0xffffu)], a.num_pages, kBlock);
+        // this CTA's items among the selected blocks: groups q with
+        // gpre[q] < e and gpre[q] + gcnt[q] > s0, one warp per group
+        const int e_sel = min(s1, keff);
+        if (s0 < e_sel) {
+            int lo = 0, hi = ngroups - 1;  // first group ending past s0
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (gpre[mid] + gcnt[mid] > s0) hi = mid;
+                else lo = mid + 1;
+            }
+            for (int q = lo + warp; q < ngroups && gpre[q] < e_sel; q += kWarpsAll) {
+                const int i = q * 32 + lane;
+                const uint32_t k = i < M ? ukeys_s[i] : 0u;
+                const uint32_t dg = k >> 16;
+                const bool sel = i < M && (dg > d1 || (dg == d1 && rem > 0 && composite(k, i) >= tau));
+                const uint32_t bs = __ballot_sync(0xffffffffu, sel);
+                const int rank = gpre[q] + __popc(bs & lt_mask);
+                if (sel && rank >= s0 && rank < e_sel) {
+                    res_item[rank - s0] = item_of_page(page_of(i), a.num_pages, kBlock);
+                    own_item[rank - s0] = (uint32_t)i;
+                }
+            }
         }
+    } else if (mode == kModeAll) {
+        // every complete block is selected: items are block ids themselves
+        for (int j = tid; j < min(s1, M) - s0; j += kThreadsAll) {
+            res_item[j] = item_of_page(page_of(s0 + j), a.num_pages, kBlock);
+            own_item[j] = (uint32_t)(s0 + j);
+        }
+    }
+    if (tid == 0 && seq_ok && keff >= s0 && keff < s1) {
+        res_item[keff - s0] = item_of_page(cur_page, a.num_pages, L - M * kBlock);
+        own_item[keff - s0] = (uint32_t)M;
     }
     __syncthreads();
 
     if (warp < kDW) {
-        // ---- 3. decode warps: own definite blocks, then the rest ----
+        // ---- 3. decode warps: this CTA's items ----
         WarpState<D, 1> st;
         st.init();
-        const int n_items = kept_def + n_res;
-        auto item_at = [&](int j) -> uint32_t { return j < kept_def ? own_item[j] : res_item[j - kept_def]; };
         uint8_t *wr = ring + (size_t)warp * kKvStages * SM::kStageBytes;
         constexpr int kPerLane = SM::kTileBytes / 16 / 32;
         auto issue = [&](int t) {
             const int j = warp + kDW * t;
             if (j < n_items) {
-                const uint32_t item = item_at(j);
+                const uint32_t item = res_item[j];
                 if (item != kSkip) {
                     const size_t tile = ((size_t)(item >> 4) * hkv + h) * SM::kTileBytes;
                     uint8_t *stg = wr + (size_t)(t % kKvStages) * SM::kStageBytes;
@@ -837,7 +718,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             issue(t + kKvStages - 1);
             cp_async_wait<kKvStages - 1>();
             __syncwarp();
-            const uint32_t item = item_at(warp + kDW * t);
+            const uint32_t item = res_item[warp + kDW * t];
             if (item != kSkip) {
                 const uint32_t ks = smem_u32(wr + (size_t)(t % kKvStages) * SM::kStageBytes);
                 attend_block_swapped<D, 1>(st, qb, ks, ks + SM::kTileBytes, (int)(item & 15u) + 1,
@@ -873,36 +754,17 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             o0[D + 8] = st.o[t][0][3];
         }
     } else {
-        // ---- 3'. the other warps: block list (ascending), count, errors ----
+        // ---- 3'. the other warps: this CTA's part of the block list, the
+        // count, errors, and (a single CTA per unit) the histogram cleanup ----
         const int ct = tid - kDW * 32;
         int32_t *list = a.block_idx + (size_t)u * (a.max_topk + 1);
-        {
-            constexpr int R2 = (kStepMaxBlocks + kCtlThreads - 1) / kCtlThreads;
-            const int i0 = ct * R2;
-            uint32_t ns = 0;
-            for (int r = 0; r < R2; ++r) {
-                const int i = i0 + r;
-                if (i < nmine && (own_def(i) || own_qual(i))) ++ns;
-            }
-            uint32_t tot;
-            uint32_t pos = ctl_scan(ns, ct, s_scan, tot) + (uint32_t)s_v[kVSelBefore];
-            for (int r = 0; r < R2; ++r) {
-                const int i = i0 + r;
-                if (i < nmine && (own_def(i) || own_qual(i)) && pos < (uint32_t)keff) list[pos++] = p0 + i;
-            }
-        }
+        for (int j = ct; j < n_items; j += kCtlThreads) list[s0 + j] = (int32_t)own_item[j];
         if (x == 0 && ct == 0) {
-            if (seq_ok) {
-                list[keff] = M;
-                a.block_cnt[u] = keff + 1;
-            } else {
-                a.block_cnt[u] = 0;
-                set_error(a.err, RESA_DEVERR_SEQ_LEN);
-            }
+            a.block_cnt[u] = seq_ok ? keff + 1 : 0;
+            if (!seq_ok) set_error(a.err, RESA_DEVERR_SEQ_LEN);
             if (topk_err) set_error(a.err, RESA_DEVERR_TOPK);
         }
         if (G == 1 && need_hist) {
-            // the only CTA of the unit has read the histogram: clear it
             uint32_t *hb = a.hist + (size_t)u * kHistBins;
             for (int d = s_v[kVDlo] + ct; d <= s_v[kVDhi]; d += kCtlThreads) hb[d] = 0;
             if (ct == 0) {
@@ -953,8 +815,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     // goes to CTA item % G, after a second unit barrier.  CTAs without an item
     // arrive and leave.
     constexpr int C32 = D / 32;
-    const int n_items = g * C32;
-    const bool merger = x < n_items;
+    const int n_slices = g * C32;
+    const bool merger = x < n_slices;
     __threadfence();
     __syncthreads();
     if (tid == 0) {
@@ -983,7 +845,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     constexpr int kPW = (kNumSms + kWarpsAll - 1) / kWarpsAll;  // partials per warp
     constexpr int kPL = (kNumSms + 31) / 32;                     // log-sum-exps per lane
     float *red = reinterpret_cast<float *>(ring);                // [kWarpsAll][33]
-    for (int item = x; item < n_items; item += G) {
+    for (int item = x; item < n_slices; item += G) {
         const int r = item / C32, cc = item % C32;
         // every load of the item in flight at once: this warp's partials
         // (warp, warp + 12, ...) and every partial's log2-sum-exp
