@@ -88,9 +88,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       float *__restrict__ out, float *__restrict__ lse_out, uint32_t *err) {
     using LY = TcLayout<D>;
     extern __shared__ uint8_t smem_raw[];
-    // 1024-byte aligned base, derived from the shared array itself so that
-    // accesses keep the shared address space (no generic loads)
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
     __shared__ uint64_t q_ready, kv_full[kStages], v_ready[kStages], kv_empty[kStages], s_full[2],
         p_full, pv_done;
     __shared__ uint32_t tmem_base_s;

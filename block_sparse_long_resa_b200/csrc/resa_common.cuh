@@ -59,12 +59,13 @@ inline int decode_max_splits(int batch, int hkv, int max_pages) {
 // max_pages <= 65536.
 constexpr int kStepMaxBlocks = 1024;
 constexpr int kStepMaxPages = 65536;
-// After scoring, every CTA of the fused step holds its unit's keys, page ids
-// and boundary candidates (12 warps x 512 at most) in its K/V rings (8 warps x
-// 3 stages x a 16-token K and V tile): at most this many complete blocks.
+// After scoring, every CTA of the fused step holds its unit's keys, page ids,
+// boundary candidates (12 warps x 512 at most) and a 2048-bin radix
+// histogram in its K/V rings (8 warps x 3 stages x a 16-token K and V tile):
+// at most this many complete blocks.
 constexpr int step_unit_keys(int d) {
-    return (kDecodeWarps * 3 * 2 * kBlock * d * 2 - 12 * 512 * 4 - 64) / 8 < 32768
-               ? (kDecodeWarps * 3 * 2 * kBlock * d * 2 - 12 * 512 * 4 - 64) / 8
+    return (kDecodeWarps * 3 * 2 * kBlock * d * 2 / 4 - 12 * 512 - 2048 - 16) / 2 < 32768
+               ? (kDecodeWarps * 3 * 2 * kBlock * d * 2 / 4 - 12 * 512 - 2048 - 16) / 2
                : 32768;
 }
 // Row stride (in keys) of a unit's key row in the workspace: 16-byte rows.

@@ -67,8 +67,8 @@ struct StepSmem {
     static constexpr int kSlotBytes = kScoreBlocks * kDescBytes;
     static_assert(kWarpsAll * kScoreSlots * kSlotBytes <= kRingBytes, "score rings fit the K/V rings");
     static_assert(kDW * kMaxGroup * (D + 2) * 4 <= kRingBytes, "warp states fit the rings");
-    static_assert(step_unit_keys(D) * 8 + kWarpsAll * kCandPerWarp * 4 + 64 <= kRingBytes,
-                  "the unit's keys, page ids and candidates fit the rings");
+    static_assert((step_unit_keys(D) * 2 + 8 + kWarpsAll * kCandPerWarp + 2048) * 4 <= kRingBytes,
+                  "the unit's keys, page ids, candidates and radix bins fit the rings");
     static_assert(step_unit_keys(D) <= kMaxGroups * 32, "group counts fit the hash area");
     static constexpr int kKeysOff = kRingBytes;                      // u32 [kStepMaxBlocks] own keys
     static constexpr int kPagesOff = kKeysOff + kStepMaxBlocks * 4;  // i32 [kStepMaxBlocks] own pages
@@ -169,7 +169,6 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     uint32_t *hkey = reinterpret_cast<uint32_t *>(smem + SM::kHashOff), *hcnt = hkey + kHash;
 
     __shared__ float qbar_s[D];
-    __shared__ uint32_t s_rh[256];
     __shared__ uint32_t s_scan[kWarpsAll];
     __shared__ uint32_t s_rsh[3];
     __shared__ int s_v[kVCount];
@@ -408,7 +407,20 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     __threadfence();
     __syncthreads();
 
-    // ---- 2. unit barrier; the unit's keys and histogram; threshold; layout ----
+    // ---- 2. the unit's page ids (an input: copied while the unit's CTAs
+    // meet), unit barrier, then the unit's keys and histogram ----
+    // page id of block i at upages_s[i + pshift]: the row is copied from the
+    // 16-byte boundary at or below its start, the tail (inside the row) with
+    // 4-byte copies
+    uint32_t *upages_s = ukeys_s + ((M + 3) & ~3);
+    const int pshift = (int)(prow & 3);
+    if (mode == kModeAll || mode == kModeMid) {
+        const int32_t *prow_al = a.page_table + (prow - pshift);
+        const int nfull = (M + pshift) / 4;
+        for (int c = tid; c < nfull; c += kThreadsAll) cp_async16(upages_s + 4 * c, prow_al + 4 * c);
+        for (int e = 4 * nfull + tid; e < M + pshift; e += kThreadsAll) cp_async4(upages_s + e, prow_al + e);
+    }
+    cp_async_commit();
     if (G > 1 && need_hist) {
         if (tid == 0) {
             const uint32_t gen = unit_bar_arrive(&a.bars[2 * u], G);
@@ -421,20 +433,10 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
         __threadfence();
     }
-    // ---- 2'. in one round trip: the unit's keys and page ids (into the idle
-    // K/V rings) and the histogram around this CTA's own top digit ----
-    // page id of block i at upages_s[i + pshift]: the row is copied from the
-    // 16-byte boundary at or below its start; the tail (inside the row) with
-    // 4-byte copies
-    uint32_t *upages_s = ukeys_s + ((M + 3) & ~3);
-    const int pshift = (int)(prow & 3);
-    if (mode == kModeAll || mode == kModeMid) {
-        if (mode == kModeMid)
-            for (int c = tid; c < (M + 3) / 4; c += kThreadsAll) cp_async16(ukeys_s + 4 * c, ukeys_g + 4 * c);
-        const int32_t *prow_al = a.page_table + (prow - pshift);
-        const int nfull = (M + pshift) / 4;
-        for (int c = tid; c < nfull; c += kThreadsAll) cp_async16(upages_s + 4 * c, prow_al + 4 * c);
-        for (int e = 4 * nfull + tid; e < M + pshift; e += kThreadsAll) cp_async4(upages_s + e, prow_al + e);
+    // in one round trip: the unit's keys (into the idle K/V rings) and the
+    // histogram around this CTA's own top digit
+    if (mode == kModeMid) {
+        for (int c = tid; c < (M + 3) / 4; c += kThreadsAll) cp_async16(ukeys_s + 4 * c, ukeys_g + 4 * c);
         cp_async_commit();
     }
     auto page_of = [&](int blk) -> int { return (int)upages_s[blk + pshift]; };
@@ -501,11 +503,10 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     // Work split: the unit's ordered work list is the selected blocks in
     // ascending order, then the current block (W = keff + 1 items); CTA x
-    // takes items [x*F, (x+1)*F).
+    // takes items [x*W/G, (x+1)*W/G).
     const int W = seq_ok ? keff + 1 : 0;
-    const int F = (W + G - 1) / G;
-    const int s0 = min(W, x * F), s1 = min(W, s0 + F);
-    const int n_items = s1 - s0;
+    const int s0 = (int)((long long)W * x / G), s1 = (int)((long long)W * (x + 1) / G);
+    const int n_items = s1 - s0;  // floor(W / G) or one more
     int *gcnt = reinterpret_cast<int *>(hkey), *gpre = reinterpret_cast<int *>(hcnt);  // [ngroups]
     const int ngroups = (M + 31) >> 5;
     uint32_t tau = 0xffffffffu;
@@ -521,7 +522,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         uint32_t *seg = cand_s + warp * cap;
         int nseg = 0;
         for (int g0 = warp; g0 < ngroups; g0 += 4 * kWarpsAll) {
-            uint32_t kk[4];
+            uint32_t kk[4], bd[4], bc[4];
 #pragma unroll
             for (int u4 = 0; u4 < 4; ++u4) {
                 const int i = (g0 + kWarpsAll * u4) * 32 + lane;
@@ -529,16 +530,23 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             }
 #pragma unroll
             for (int u4 = 0; u4 < 4; ++u4) {
-                const int grp = g0 + kWarpsAll * u4;
-                const int i = grp * 32 + lane;
+                const int i = (g0 + kWarpsAll * u4) * 32 + lane;
                 const uint32_t dg = kk[u4] >> 16;
-                const bool isc = i < M && dg == d1;
-                const uint32_t bd = __ballot_sync(0xffffffffu, i < M && dg > d1);
-                const uint32_t bc = __ballot_sync(0xffffffffu, isc);
-                if (lane == 0 && grp < ngroups) gcnt[grp] = __popc(bd);
-                const int r = nseg + __popc(bc & lt_mask);
-                if (isc && r < cap) seg[r] = composite(kk[u4], i);
-                nseg += __popc(bc);
+                bd[u4] = __ballot_sync(0xffffffffu, i < M && dg > d1);
+                bc[u4] = __ballot_sync(0xffffffffu, i < M && dg == d1);
+            }
+            // lane u4 < 4 stores group u4's definite count
+            uint32_t mine = bd[0];
+#pragma unroll
+            for (int u4 = 1; u4 < 4; ++u4) mine = lane == u4 ? bd[u4] : mine;
+            const int gme = g0 + kWarpsAll * lane;
+            if (lane < 4 && gme < ngroups) gcnt[gme] = __popc(mine);
+#pragma unroll
+            for (int u4 = 0; u4 < 4; ++u4) {
+                const int i = (g0 + kWarpsAll * u4) * 32 + lane;
+                const int r = nseg + __popc(bc[u4] & lt_mask);
+                if (((bc[u4] >> lane) & 1u) && r < cap) seg[r] = composite(kk[u4], i);
+                nseg += __popc(bc[u4]);
             }
         }
         if (lane == 0) s_seg[warp] = nseg;
@@ -584,45 +592,47 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             rem = max(0, min(rem, NC));
         }
         if (rem > 0) {
+            // digits of 11, 8, 8 and 5 bits, most significant first; bins in
+            // the rings after the candidates; the digit holding the remaining-th
+            // largest candidate is found by one CTA-wide scan in descending order
+            uint32_t *rh = cand_s + kWarpsAll * cap;  // [2048]
             uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)rem;
-            for (int shift = 24; shift >= 0; shift -= 8) {
-                for (int i = tid; i < 256; i += kThreadsAll) s_rh[i] = 0;
+            int shift = 32;
+            for (int pass = 0; pass < 4; ++pass) {
+                const int width = pass == 0 ? 11 : pass == 3 ? 5 : 8;
+                shift -= width;
+                const int nb = 1 << width;
+                for (int i = tid; i < nb; i += kThreadsAll) rh[i] = 0;
                 __syncthreads();
                 for_each_cand([&](uint32_t c) {
-                    if ((c & pmask) == prefix) atomicAdd(&s_rh[(c >> shift) & 255u], 1u);
+                    if ((c & pmask) == prefix) atomicAdd(&rh[(c >> shift) & (uint32_t)(nb - 1)], 1u);
                 });
                 __syncthreads();
-                if (warp == 0) {
-                    // lane l holds digits 255 - 8l - j, j = 0..7 (descending)
-                    uint32_t cnt[8], sum = 0;
+                constexpr int kPer = (2048 + kThreadsAll - 1) / kThreadsAll;
+                uint32_t cnt[kPer], sum = 0;
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        cnt[jj] = s_rh[255 - 8 * lane - jj];
-                        sum += cnt[jj];
-                    }
-                    uint32_t incl = sum;
+                for (int jj = 0; jj < kPer; ++jj) {
+                    const int dgt = nb - 1 - (tid * kPer + jj);  // descending digits
+                    cnt[jj] = dgt >= 0 ? rh[dgt] : 0u;
+                    sum += cnt[jj];
+                }
+                uint32_t tot;
+                uint32_t cum = cta_scan(sum, s_scan, tot);  // candidates in higher digits
+                if (cum < remaining && remaining <= cum + sum) {
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += t;
-                    }
-                    uint32_t cum = incl - sum;
-                    if (cum < remaining && remaining <= incl) {
-#pragma unroll
-                        for (int jj = 0; jj < 8; ++jj) {
-                            if (cum < remaining && remaining <= cum + cnt[jj]) {
-                                s_rsh[0] = 255u - 8u * lane - jj;
-                                s_rsh[1] = cum;
-                                s_rsh[2] = cnt[jj];
-                            }
-                            cum += cnt[jj];
+                    for (int jj = 0; jj < kPer; ++jj) {
+                        if (cum < remaining && remaining <= cum + cnt[jj]) {
+                            s_rsh[0] = (uint32_t)(nb - 1 - (tid * kPer + jj));
+                            s_rsh[1] = cum;
+                            s_rsh[2] = cnt[jj];
                         }
+                        cum += cnt[jj];
                     }
                 }
                 __syncthreads();
                 remaining -= s_rsh[1];
                 prefix |= s_rsh[0] << shift;
-                pmask |= 255u << shift;
+                pmask |= (uint32_t)(nb - 1) << shift;
                 if (remaining == s_rsh[2]) break;  // every key with this prefix is taken
             }
             tau = prefix;

@@ -72,16 +72,17 @@ def test_concentrated_selection_moves_blocks_between_ctas(cuda_device):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
 
 
-@pytest.mark.parametrize("ctx,topk,max_topk", [
-    ([333, 257, 1999], [5, 0, 10**6], 80),     # candidates resolved in shared memory
-    ([65536], [300], 300),                      # 4096 tied candidates: read from the workspace
-], ids=["smem", "workspace"])
-def test_exact_ties_go_to_lower_block_ids(cuda_device, ctx, topk, max_topk):
+@pytest.mark.parametrize("ctx,topk,max_topk,d", [
+    ([333, 257, 1999], [5, 0, 10**6], 80, 64),  # candidate lists in shared memory
+    ([65536], [300], 300, 64),                   # 4096 tied candidates
+    ([131072], [500], 500, 128),                 # 8192 tied candidates: past the lists' room
+], ids=["small", "4096-tied", "8192-tied"])
+def test_exact_ties_go_to_lower_block_ids(cuda_device, ctx, topk, max_topk, d):
     """All keys equal: every score ties, so the lowest block ids win; top-k 0
     keeps the current block only; top-k above max_topk is clamped and
     reported."""
     B = len(ctx)
-    p = inputs.make_decode_problem(9, B, 8, 1, 64, 16, ctx, paged=True, needles=0,
+    p = inputs.make_decode_problem(9, B, 8, 1, d, 16, ctx, paged=True, needles=0,
                                    topk=[1] * B)
     p.k_cache[:] = 0.5
     p.k_new[:] = 0.5
