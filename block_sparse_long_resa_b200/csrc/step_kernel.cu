@@ -35,9 +35,10 @@
 //     row, 32 channels) slice of the unit's G partials; the others leave.
 //
 // The append (K/V of the decode token at position L-1 and the fold of its key
-// into the current block's descriptor) is done by one warp of CTA 0 of each
-// unit during the scoring phase: only the current block reads it, and that
-// block is never scored and is decoded after the barrier.
+// into the current block's descriptor) is done by one warp of CTA G-1 of each
+// unit during the scoring phase: only the current block reads it, that block
+// is never scored, and it is the last work item, which CTA G-1 itself
+// decodes, so the CTA's own barriers order the append before the read.
 #include "attn_common.cuh"
 
 namespace resa {
@@ -199,15 +200,19 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     uint32_t *ukeys_g = a.ukeys + (size_t)u * a.key_stride;
 
     // ---- prologue: inputs of the call only (before the dependency wait) ----
+    #pragma unroll 1
     for (int i = tid; i < nmine; i += kThreadsAll) pages[i] = a.page_table[prow + p0 + i];
     {
         const uint16_t *qh = a.q + ((size_t)b * hkv * g + (size_t)h * g) * D;
+        #pragma unroll 1
         for (int j = tid; j < D; j += kThreadsAll) {
             float s = 0.f;
+            #pragma unroll 1
             for (int r = 0; r < g; ++r) s += bf16_bits_to_f32(qh[(size_t)r * D + j]);
             qbar_s[j] = s / (float)g;
         }
     }
+    #pragma unroll 1
     for (int i = tid; i < kHash; i += kThreadsAll) {
         hkey[i] = kHashEmpty;
         hcnt[i] = 0;
@@ -237,7 +242,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     // it) and, for the appending warp, the decode token's K / V chunks.
     const int cur_page = seq_ok ? a.page_table[prow + M] : -1;
     constexpr int CPR = D / 8;  // 16-byte chunks per K / V row
-    const bool appender = x == 0 && warp == kWarpsAll - 1 && seq_ok;
+    const bool appender = x == G - 1 && warp == kWarpsAll - 1 && seq_ok;
     uint4 app_k = make_uint4(0, 0, 0, 0), app_v = app_k;
     if (appender && lane < CPR) {
         app_k = a.k_new[((size_t)b * hkv + h) * CPR + lane];
@@ -288,7 +293,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             }
             cp_async_commit();
         };
-#pragma unroll
+#pragma unroll 1
         for (int it = 0; it < kScoreSlots - 1; ++it) issue(it);
         const int j = lane >> 2, s = lane & 3, sw = (j & 1) << 2;
         float qv[RC][8];
@@ -366,10 +371,12 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         // per-CTA histogram of the keys' top 16 bits, then one global atomic
         // per distinct digit
         int lo = 0x7fffffff, hi = -1;
+        #pragma unroll 1
         for (int i = tid; i < nmine; i += kThreadsAll) {
             const uint32_t digit = keys[i] >> 16;
             uint32_t slot = (digit * 0x9E3779B1u) >> 22;  // 10 bits
             bool placed = false;
+            #pragma unroll 1
             for (int probe = 0; probe < 64; ++probe) {
                 const uint32_t old = atomicCAS(&hkey[slot], kHashEmpty, digit);
                 if (old == kHashEmpty || old == digit) {
@@ -386,6 +393,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             }
         }
         __syncthreads();
+        #pragma unroll 1
         for (int i = tid; i < kHash; i += kThreadsAll) {
             const uint32_t k = hkey[i];
             if (k != kHashEmpty) {
@@ -417,7 +425,9 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     if (mode == kModeAll || mode == kModeMid) {
         const int32_t *prow_al = a.page_table + (prow - pshift);
         const int nfull = (M + pshift) / 4;
+        #pragma unroll 1
         for (int c = tid; c < nfull; c += kThreadsAll) cp_async16(upages_s + 4 * c, prow_al + 4 * c);
+        #pragma unroll 1
         for (int e = 4 * nfull + tid; e < M + pshift; e += kThreadsAll) cp_async4(upages_s + e, prow_al + e);
     }
     cp_async_commit();
@@ -436,6 +446,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     // in one round trip: the unit's keys (into the idle K/V rings) and the
     // histogram around this CTA's own top digit
     if (mode == kModeMid) {
+        #pragma unroll 1
         for (int c = tid; c < (M + 3) / 4; c += kThreadsAll) cp_async16(ukeys_s + 4 * c, ukeys_g + 4 * c);
         cp_async_commit();
     }
@@ -466,11 +477,13 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             top = dhi - tid * chunk;
             bot = max(dlo, top - chunk + 1);
             loc = 0;
+            #pragma unroll 1
             for (int d = top; d >= bot; --d) loc += __ldcg(&hb[d]);
         }
         above_me = cta_scan(loc, s_scan, total);  // keys in the bins above this thread's
         if (above_me < (uint32_t)keff && (uint32_t)keff <= above_me + loc) {
             uint32_t cum = above_me;
+            #pragma unroll 1
             for (int d = top; d >= bot; --d) {
                 const uint32_t c = covered ? wc : __ldcg(&hb[d]);
                 if (cum + c >= (uint32_t)keff) {
@@ -521,6 +534,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         const uint32_t lt_mask = (1u << lane) - 1u;
         uint32_t *seg = cand_s + warp * cap;
         int nseg = 0;
+        #pragma unroll 1
         for (int g0 = warp; g0 < ngroups; g0 += 4 * kWarpsAll) {
             uint32_t kk[4], bd[4], bc[4];
 #pragma unroll
@@ -569,6 +583,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         // overflowed, candidates are found by scanning the keys instead
         auto for_each_cand = [&](auto fn) {
             if (fits) {
+                #pragma unroll 1
                 for (int f = tid; f < NC; f += kThreadsAll) {
                     int w = 0, st0 = 0;
 #pragma unroll
@@ -580,6 +595,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                     fn(cand_s[w * cap + (f - st0)]);
                 }
             } else {
+                #pragma unroll 1
                 for (int i = tid; i < M; i += kThreadsAll) {
                     const uint32_t k = ukeys_s[i];
                     if ((k >> 16) == d1) fn(composite(k, i));
@@ -598,10 +614,12 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             uint32_t *rh = cand_s + kWarpsAll * cap;  // [2048]
             uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)rem;
             int shift = 32;
+            #pragma unroll 1
             for (int pass = 0; pass < 4; ++pass) {
                 const int width = pass == 0 ? 11 : pass == 3 ? 5 : 8;
                 shift -= width;
                 const int nb = 1 << width;
+                #pragma unroll 1
                 for (int i = tid; i < nb; i += kThreadsAll) rh[i] = 0;
                 __syncthreads();
                 for_each_cand([&](uint32_t c) {
@@ -672,6 +690,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                 if (gpre[mid] + gcnt[mid] > s0) hi = mid;
                 else lo = mid + 1;
             }
+            #pragma unroll 1
             for (int q = lo + warp; q < ngroups && gpre[q] < e_sel; q += kWarpsAll) {
                 const int i = q * 32 + lane;
                 const uint32_t k = i < M ? ukeys_s[i] : 0u;
@@ -687,6 +706,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
     } else if (mode == kModeAll) {
         // every complete block is selected: items are block ids themselves
+        #pragma unroll 1
         for (int j = tid; j < min(s1, M) - s0; j += kThreadsAll) {
             res_item[j] = item_of_page(page_of(s0 + j), a.num_pages, kBlock);
             own_item[j] = (uint32_t)(s0 + j);
@@ -722,7 +742,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             }
             cp_async_commit();
         };
-#pragma unroll
+#pragma unroll 1
         for (int t = 0; t < kKvStages - 1; ++t) issue(t);
         for (int t = 0; warp + kDW * t < n_items; ++t) {
             issue(t + kKvStages - 1);
@@ -768,6 +788,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         // count, errors, and (a single CTA per unit) the histogram cleanup ----
         const int ct = tid - kDW * 32;
         int32_t *list = a.block_idx + (size_t)u * (a.max_topk + 1);
+        #pragma unroll 1
         for (int j = ct; j < n_items; j += kCtlThreads) list[s0 + j] = (int32_t)own_item[j];
         if (x == 0 && ct == 0) {
             a.block_cnt[u] = seq_ok ? keff + 1 : 0;
@@ -776,6 +797,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
         if (G == 1 && need_hist) {
             uint32_t *hb = a.hist + (size_t)u * kHistBins;
+            #pragma unroll 1
             for (int d = s_v[kVDlo] + ct; d <= s_v[kVDhi]; d += kCtlThreads) hb[d] = 0;
             if (ct == 0) {
                 a.hist_range[2 * u] = 0;
@@ -794,6 +816,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         float *po = a.part_o + (size_t)cta * kStepMaxGroup * D;
         float *pl = a.part_lse + (size_t)cta * kMaxGroup;
         const int hq = hkv * g;
+        #pragma unroll 1
         for (int e = tid; e < g * D; e += kThreadsAll) {
             const int r = e / D, c = e % D;
             float mstar = -INFINITY;
@@ -844,6 +867,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         // every CTA of the unit read the histogram before this barrier: leave
         // it clear for the next call
         uint32_t *hb = a.hist + (size_t)u * kHistBins;
+        #pragma unroll 1
         for (int d = s_v[kVDlo] + tid; d <= s_v[kVDhi]; d += kThreadsAll) hb[d] = 0;
         if (tid == 0) {
             a.hist_range[2 * u] = 0;
@@ -855,6 +879,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     constexpr int kPW = (kNumSms + kWarpsAll - 1) / kWarpsAll;  // partials per warp
     constexpr int kPL = (kNumSms + 31) / 32;                     // log-sum-exps per lane
     float *red = reinterpret_cast<float *>(ring);                // [kWarpsAll][33]
+    #pragma unroll 1
     for (int item = x; item < n_slices; item += G) {
         const int r = item / C32, cc = item % C32;
         // every load of the item in flight at once: this warp's partials
