@@ -1,9 +1,10 @@
 """The fused decode step (one cooperative launch per step) against the CPU
-oracle, on the cases that reach its own code paths: the residual pool that
-moves definite blocks between CTAs, exact score ties resolved by block index
-(in shared memory and, past its capacity, from the workspace), top-k 0 and
-top-k >= M in one launch, and back-to-back calls that must leave the
-workspace clean (histogram and barriers) and give identical results.
+oracle, on the cases that reach its own code paths: a selection concentrated
+in a few CTAs' ranges that the balanced slices of the ordered selection
+spread over all CTAs, exact score ties resolved by block index (candidate
+lists in shared memory and, past their room, the fallback scan of the keys),
+top-k 0 and top-k >= M in one launch, and back-to-back calls that must leave
+the workspace clean (histogram and barriers) and give identical results.
 
 Bars as in test_gpu_parity: block sets exact (up to fp32 near-ties of the
 k-th score), outputs within 2e-3 absolute, log-sum-exp within 1e-3.
@@ -46,8 +47,8 @@ def test_fused_path_is_taken(cuda_device):
 
 def test_concentrated_selection_moves_blocks_between_ctas(cuda_device):
     """Blocks 0..299 of the sequence get keys pushed along the pooled query,
-    so the top 205 all lie in the first CTAs' ranges: their definite blocks
-    beyond the fair share go to the residual pool of the other CTAs."""
+    so the top 205 all lie in the first CTAs' ranges: the contiguous slices of
+    the ordered selection hand them to every CTA of the unit."""
     p = inputs.make_decode_problem(61, 1, 28, 4, 128, 16, [32768], needles=0)
     hq, hkv, g = 28, 4, 7
     qbar = p.q.float().view(1, hkv, g, 128).mean(2)[0]          # [Hkv][d]
