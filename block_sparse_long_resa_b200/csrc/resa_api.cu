@@ -322,8 +322,7 @@ resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cac
         buf.hist_range = at<uint32_t>(ws, w.hist_range);
         buf.bars = at<unsigned long long>(ws, w.step_bars);
         buf.ukeys = at<uint32_t>(ws, w.step_keys);
-        buf.part_o = at<float>(ws, w.dec_o);
-        buf.part_lse = at<float>(ws, w.dec_lse);
+        buf.part = at<unsigned long long>(ws, w.step_part);
         buf.err = at<uint32_t>(ws, w.err);
         return cuda_status(launch_decode_step_fused(s, G, cache->k, cache->v, cache->desc,
                                                     cache->page_table, cache->seq_len, q, k_new,

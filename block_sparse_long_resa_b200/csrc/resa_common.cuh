@@ -120,8 +120,9 @@ struct WsLayout {
     size_t sel_cnt;      // i32 [B][Hkv]
     size_t dec_o;        // f32 [partials][kMaxGroup][d]: per split, or per warp when spread
     size_t dec_lse;      // f32 [partials][kMaxGroup] lse, or float2 (row max, row sum) when spread
-    size_t step_bars;    // u64 [B][Hkv][2] unit barriers of the fused step (zero between calls)
+    size_t step_bars;    // u64 [B][Hkv][4] unit counter (zero between calls) and generation of the fused step
     size_t step_keys;    // u32 [B][Hkv][step_key_stride(max_pages)] block score keys of the fused step
+    size_t step_part;    // u64 [kNumSms][kStepMaxGroup][d + 1] tagged per-CTA partials of the fused step
     size_t rect_o;       // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta][d]
     size_t rect_lse;     // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta]
     size_t total;
@@ -157,8 +158,9 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     const size_t parts = decode_partials((int)units, w.dec_splits);
     w.dec_o = take(parts * kMaxGroup * d * 4);
     w.dec_lse = take(parts * kMaxGroup * 2 * 4);  // (lse) or (row max, row sum) pairs
-    w.step_bars = take(units * 2 * 8);
+    w.step_bars = take(units * 4 * 8);
     w.step_keys = take(units * (size_t)step_key_stride(max_pages) * 4);
+    w.step_part = take((size_t)kNumSms * kStepMaxGroup * (d + 1) * 8);
     size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerCta;
     w.rect_o = take(rect_rows * d * 4);
     w.rect_lse = take(rect_rows * 4);
@@ -464,9 +466,9 @@ cudaError_t launch_sparse_decode(const Shape &s, const void *k, const void *v,
 struct StepBuffers {
     int32_t *block_idx, *block_cnt;  // selection output [B][Hkv][max_topk+1], [B][Hkv]
     uint32_t *hist, *hist_range;
-    unsigned long long *bars;
+    unsigned long long *bars;   // [B][Hkv][4]
     uint32_t *ukeys;
-    float *part_o, *part_lse;
+    unsigned long long *part;   // [kNumSms][kStepMaxGroup][d + 1]
     uint32_t *err;
 };
 cudaError_t launch_decode_step_fused(const Shape &s, int G, void *k, void *v, void *desc,

@@ -89,29 +89,36 @@ struct StepArgs {
     int32_t *block_idx, *block_cnt;
     float *out, *lse;
     uint32_t *hist, *hist_range;
-    unsigned long long *bars;  // [units][2] unit barriers
+    unsigned long long *bars;  // [units][4]: scored count, -, -, generation
     uint32_t *ukeys;           // [units][key_stride] every block's key
-    float *part_o, *part_lse;
+    unsigned long long *part;  // [units * G][kStepMaxGroup][D + 1] tagged partial (o, then lse)
     uint32_t *err;
     int hkv, g, max_pages, num_pages, max_topk, key_stride;
     float scale_log2;
 };
 
-// ---------------------------------------------------------------------------
-// Unit barrier: one 64-bit word per barrier holds (generation << 32) |
-// arrivals; the last arriver's single add returns the count to zero and bumps
-// the generation.  The caller fences its writes before arriving.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t unit_bar_arrive(unsigned long long *bar, uint32_t n) {
-    const unsigned long long old = atomicAdd(bar, 1ull);
-    if ((uint32_t)old == n - 1) atomicAdd(bar, (1ull << 32) - n);
-    return (uint32_t)(old >> 32);
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
 }
-__device__ __forceinline__ bool unit_bar_wait(const unsigned long long *bar, uint32_t gen) {
+// Partials are written as 64-bit words (tag << 32 | value) tagged with the
+// call's generation, so readers poll the words themselves (no fence, no
+// barrier): a word with another tag is from an earlier call.
+__device__ __forceinline__ unsigned long long tagged(uint32_t tag, uint32_t v) {
+    return ((unsigned long long)tag << 32) | v;
+}
+__device__ __forceinline__ uint32_t tag_of(unsigned long long w) { return (uint32_t)(w >> 32); }
+
+// Unit counter: each CTA adds one (no return value needed); waiters poll
+// until all G arrived.  CTA 0 sets it back to zero once every CTA's partial
+// is visible, i.e. after every CTA has passed it.  The caller fences its
+// writes before arriving.
+__device__ __forceinline__ bool unit_wait_count(const unsigned long long *ctr, uint32_t n) {
     for (uint32_t polls = 0;; ++polls) {
         unsigned long long v;
-        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(bar) : "memory");
-        if ((uint32_t)(v >> 32) != gen) return true;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
+        if (v >= (unsigned long long)n) return true;
         if (polls > (1u << 22)) return false;  // each poll is an L2 round trip
     }
 }
@@ -151,7 +158,7 @@ __device__ __forceinline__ uint32_t composite(uint32_t k, int i) {
 
 // Indices of the small shared values.
 enum {
-    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVOk3, kVLo, kVHi, kVAB, kVCount
+    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVLo, kVHi, kVAB, kVGen, kVCount
 };
 
 template <int D>
@@ -219,7 +226,6 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     if (tid == 0) {
         s_v[kVOk] = 1;
-        s_v[kVOk3] = 1;
         s_v[kVLo] = 0x7fffffff;
         s_v[kVHi] = -1;
         s_v[kVD1] = 0;
@@ -250,6 +256,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     __syncthreads();
     pdl_wait();  // descriptors and K/V may be written by the preceding kernels
+    unsigned long long *ubar = a.bars + 4 * (size_t)u;
+    const uint32_t gen = tid == 0 ? (uint32_t)ld_relaxed_u64(&ubar[3]) : 0u;  // used after scoring
 
     // ---- 1. scoring (+ the append, whose descriptor loads are issued first) ----
     uint4 app_mn = make_uint4(0, 0, 0, 0), app_mx = app_mn;
@@ -365,6 +373,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             }
         }
     }
+    if (tid == 0) s_v[kVGen] = (int)gen;
     __syncthreads();
     const bool need_hist = mode == kModeMid;
     if (need_hist) {
@@ -412,7 +421,6 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             atomicMax(&a.hist_range[2 * u + 1], (uint32_t)(s_v[kVHi] + 1));
         }
     }
-    __threadfence();
     __syncthreads();
 
     // ---- 2. the unit's page ids (an input: copied while the unit's CTAs
@@ -433,15 +441,15 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     cp_async_commit();
     if (G > 1 && need_hist) {
         if (tid == 0) {
-            const uint32_t gen = unit_bar_arrive(&a.bars[2 * u], G);
-            s_v[kVOk] = unit_bar_wait(&a.bars[2 * u], gen) ? 1 : 0;
+            __threadfence();  // the CTA's key row and histogram atomics, ordered by the barrier above
+            atomicAdd(&ubar[0], 1ull);
+            s_v[kVOk] = unit_wait_count(&ubar[0], G) ? 1 : 0;
         }
         __syncthreads();
         if (!s_v[kVOk]) {
             if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
             return;
         }
-        __threadfence();
     }
     // in one round trip: the unit's keys (into the idle K/V rings) and the
     // histogram around this CTA's own top digit
@@ -807,16 +815,17 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     __syncthreads();  // warp states are in shared memory
 
-    // ---- 4. merge the warps, then the unit's CTAs ----
+    // ---- 4. merge the warps into this CTA's partial (tagged words) ----
     const float kLn2 = 0.6931471805599453f;
+    const uint32_t tag = (uint32_t)s_v[kVGen] + 1u;
+    constexpr int PS = D + 1;  // partial row: D outputs, then the log2-sum-exp
     {
         const float *mw = reinterpret_cast<const float *>(ring);
         const float *lw = mw + kDW * kMaxGroup;
         const float *ow = lw + kDW * kMaxGroup;
-        float *po = a.part_o + (size_t)cta * kStepMaxGroup * D;
-        float *pl = a.part_lse + (size_t)cta * kMaxGroup;
+        unsigned long long *pp = a.part + (size_t)cta * kStepMaxGroup * PS;
         const int hq = hkv * g;
-        #pragma unroll 1
+#pragma unroll 1
         for (int e = tid; e < g * D; e += kThreadsAll) {
             const int r = e / D, c = e % D;
             float mstar = -INFINITY;
@@ -838,75 +847,64 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                 a.out[orow * D + c] = on;
                 if (a.lse && c == 0) a.lse[orow] = lse2 * kLn2;
             } else {
-                po[(size_t)r * D + c] = on;
-                if (c == 0) pl[r] = lse2;
+                pp[(size_t)r * PS + c] = tagged(tag, __float_as_uint(on));
+                if (c == 0) pp[(size_t)r * PS + D] = tagged(tag, __float_as_uint(lse2));
             }
         }
     }
     if (G == 1) return;
-    // The unit's G partials are merged by slices: item (row r, 32 channels)
-    // goes to CTA item % G, after a second unit barrier.  CTAs without an item
-    // arrive and leave.
+    // Each (query row, 32 channels) slice of the output goes to CTA
+    // slice % G, which polls the G partials' words until they carry this
+    // call's tag.  CTAs without a slice leave.
     constexpr int C32 = D / 32;
     const int n_slices = g * C32;
-    const bool merger = x < n_slices;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t gen = unit_bar_arrive(&a.bars[2 * u + 1], G);
-        s_v[kVOk3] = merger ? (unit_bar_wait(&a.bars[2 * u + 1], gen) ? 1 : 0) : 1;
-    }
-    __syncthreads();
-    if (!merger) return;
-    if (!s_v[kVOk3]) {
-        if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
-        return;
-    }
-    __threadfence();
-    if (x == 0 && need_hist) {
-        // every CTA of the unit read the histogram before this barrier: leave
-        // it clear for the next call
-        uint32_t *hb = a.hist + (size_t)u * kHistBins;
-        #pragma unroll 1
-        for (int d = s_v[kVDlo] + tid; d <= s_v[kVDhi]; d += kThreadsAll) hb[d] = 0;
-        if (tid == 0) {
-            a.hist_range[2 * u] = 0;
-            a.hist_range[2 * u + 1] = 0;
-        }
-    }
-    const float *ul = a.part_lse + (size_t)u * G * kMaxGroup;
-    const float *uo = a.part_o + (size_t)u * G * kStepMaxGroup * D;
+    if (x >= n_slices) return;
+    __syncthreads();  // the ring's warp states are read; it holds the reduction below
+    const unsigned long long *up = a.part + (size_t)u * G * kStepMaxGroup * PS;
     constexpr int kPW = (kNumSms + kWarpsAll - 1) / kWarpsAll;  // partials per warp
-    constexpr int kPL = (kNumSms + 31) / 32;                     // log-sum-exps per lane
     float *red = reinterpret_cast<float *>(ring);                // [kWarpsAll][33]
-    #pragma unroll 1
+    float *lse_s = red + kWarpsAll * 33;                         // [G] partials' log2-sum-exp
+    bool all_ok = true;
+#pragma unroll 1
     for (int item = x; item < n_slices; item += G) {
         const int r = item / C32, cc = item % C32;
-        // every load of the item in flight at once: this warp's partials
-        // (warp, warp + 12, ...) and every partial's log2-sum-exp
-        float v[kPW], lv[kPW], la[kPL];
+        // this warp's partials (warp, warp + 12, ...) at lane's channel; one
+        // thread per partial for its log2-sum-exp
+        unsigned long long wv[kPW];
+        bool ok = false;
+#pragma unroll 1
+        for (uint32_t polls = 0; polls < (1u << 20) && !ok; ++polls) {
+            bool good = true;
 #pragma unroll
-        for (int k = 0; k < kPW; ++k) {
-            const int sp = warp + kWarpsAll * k;
-            v[k] = sp < G ? __ldcg(&uo[((size_t)sp * kStepMaxGroup + r) * D + cc * 32 + lane]) : 0.f;
-            lv[k] = sp < G ? __ldcg(&ul[sp * kMaxGroup + r]) : -INFINITY;
+            for (int k = 0; k < kPW; ++k) {
+                const int sp = warp + kWarpsAll * k;
+                wv[k] = sp < G ? ld_relaxed_u64(up + ((size_t)sp * kStepMaxGroup + r) * PS + cc * 32 + lane)
+                               : tagged(tag, 0u);
+                good = good && tag_of(wv[k]) == tag;
+            }
+            if (tid < G) {
+                const unsigned long long wl = ld_relaxed_u64(up + ((size_t)tid * kStepMaxGroup + r) * PS + D);
+                good = good && tag_of(wl) == tag;
+                lse_s[tid] = __uint_as_float((uint32_t)wl);
+            }
+            ok = __syncthreads_and(good) != 0;
         }
+        all_ok = all_ok && ok;
         float mstar = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < kPL; ++k) {
-            const int sp = lane + 32 * k;
-            la[k] = sp < G ? __ldcg(&ul[sp * kMaxGroup + r]) : -INFINITY;
-            mstar = fmaxf(mstar, la[k]);
-        }
+#pragma unroll 1
+        for (int sp = lane; sp < G; sp += 32) mstar = fmaxf(mstar, lse_s[sp]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
         float lsum = 0.f, acc = 0.f;
         if (mstar != -INFINITY) {
 #pragma unroll
             for (int k = 0; k < kPW; ++k) {
-                const float wk = exp2f(lv[k] - mstar);
-                lsum += wk;
-                acc += wk * v[k];
+                const int sp = warp + kWarpsAll * k;
+                if (sp < G) {
+                    const float wk = exp2f(lse_s[sp] - mstar);
+                    lsum += wk;
+                    acc += wk * __uint_as_float((uint32_t)wv[k]);
+                }
             }
         }
         red[warp * 33 + lane] = acc;
@@ -925,6 +923,28 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                 a.lse[orow] = (lt > 0.f ? mstar + log2f(lt) : -INFINITY) * kLn2;
         }
         __syncthreads();
+    }
+    if (!all_ok) {
+        if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
+        return;
+    }
+    if (x == 0) {
+        // Every CTA's partial is visible, so every CTA has passed the counter
+        // and read the histogram: reset them for the next call and advance
+        // the generation.
+        if (tid == 0) {
+            ubar[0] = 0;
+            ubar[3] = (unsigned long long)tag;
+        }
+        if (need_hist) {
+            uint32_t *hb = a.hist + (size_t)u * kHistBins;
+#pragma unroll 1
+            for (int d = s_v[kVDlo] + tid; d <= s_v[kVDhi]; d += kThreadsAll) hb[d] = 0;
+            if (tid == 0) {
+                a.hist_range[2 * u] = 0;
+                a.hist_range[2 * u + 1] = 0;
+            }
+        }
     }
 }
 
@@ -953,8 +973,7 @@ cudaError_t launch_decode_step_fused(const Shape &s, int G, void *k, void *v, vo
     a.hist_range = buf.hist_range;
     a.bars = buf.bars;
     a.ukeys = buf.ukeys;
-    a.part_o = buf.part_o;
-    a.part_lse = buf.part_lse;
+    a.part = buf.part;
     a.err = buf.err;
     a.hkv = s.hkv;
     a.g = s.g;
