@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     __shared__ uint32_t s_rsh[3];
     __shared__ int s_v[kVCount];
     __shared__ int s_seg[kWarpsAll];
+    __shared__ float s_sc[kDW][kStepMaxGroup], s_rinv[kStepMaxGroup], s_rlse[kStepMaxGroup];
 
     pdl_launch_next();
     const int x = blockIdx.x, G = gridDim.x, u = blockIdx.y;
@@ -825,30 +826,38 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         const float *ow = lw + kDW * kMaxGroup;
         unsigned long long *pp = a.part + (size_t)cta * kStepMaxGroup * PS;
         const int hq = hkv * g;
-#pragma unroll 1
-        for (int e = tid; e < g * D; e += kThreadsAll) {
-            const int r = e / D, c = e % D;
+        // per row: the warps' scale factors exp2(m_w - m*), 1 / l and the
+        // log2-sum-exp, once
+        if (tid < g) {
+            const int r = tid;
             float mstar = -INFINITY;
 #pragma unroll
             for (int w = 0; w < kDW; ++w) mstar = fmaxf(mstar, mw[w * kMaxGroup + r]);
-            float lsum = 0.f, o = 0.f;
-            if (mstar != -INFINITY) {
+            float lsum = 0.f;
 #pragma unroll
-                for (int w = 0; w < kDW; ++w) {
-                    const float sc = exp2f(mw[w * kMaxGroup + r] - mstar);
-                    lsum += lw[w * kMaxGroup + r] * sc;
-                    o += ow[((size_t)w * kMaxGroup + r) * D + c] * sc;
-                }
+            for (int w = 0; w < kDW; ++w) {
+                const float sc = mstar != -INFINITY ? exp2f(mw[w * kMaxGroup + r] - mstar) : 0.f;
+                s_sc[w][r] = sc;
+                lsum += lw[w * kMaxGroup + r] * sc;
             }
-            const float lse2 = lsum > 0.f ? mstar + log2f(lsum) : -INFINITY;
-            const float on = lsum > 0.f ? o / lsum : 0.f;
+            s_rinv[r] = lsum > 0.f ? 1.f / lsum : 0.f;
+            s_rlse[r] = lsum > 0.f ? mstar + log2f(lsum) : -INFINITY;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int e = tid; e < g * D; e += kThreadsAll) {
+            const int r = e / D, c = e % D;
+            float o = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDW; ++w) o += ow[((size_t)w * kMaxGroup + r) * D + c] * s_sc[w][r];
+            const float on = o * s_rinv[r];
             if (G == 1) {
                 const size_t orow = (size_t)b * hq + (size_t)h * g + r;
                 a.out[orow * D + c] = on;
-                if (a.lse && c == 0) a.lse[orow] = lse2 * kLn2;
+                if (a.lse && c == 0) a.lse[orow] = s_rlse[r] * kLn2;
             } else {
                 pp[(size_t)r * PS + c] = tagged(tag, __float_as_uint(on));
-                if (c == 0) pp[(size_t)r * PS + D] = tagged(tag, __float_as_uint(lse2));
+                if (c == 0) pp[(size_t)r * PS + D] = tagged(tag, __float_as_uint(s_rlse[r]));
             }
         }
     }
