@@ -9,8 +9,11 @@
 // blocks, streamed as tiles of 64 keys (four blocks).
 //
 // Warp roles (384 threads, one CTA per SM):
-//   warp 0      TMA producer: per block and channel half, 2-D tensor loads of
-//               K and V (16 x 64, 128-byte swizzled) into a two-stage ring;
+//   warp 0      TMA producer: when a tile's four blocks sit on four
+//               consecutive pages, one 4-D tensor load per channel half of K
+//               and of V (64 channels x 16 tokens x 1 head x 4 pages, 8 KB,
+//               128-byte swizzled); otherwise one 2-D load (16 x 64) per
+//               block and half.  Both write the same shared-memory image;
 //   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into a
 //               double-buffered TMEM tile (kind::f16, bf16 inputs), then
 //               O += P V (kind::f16, fp16 inputs), commits on mbarriers;
@@ -81,6 +84,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap k1map,
                       const __grid_constant__ CUtensorMap v0map,
                       const __grid_constant__ CUtensorMap v1map,
+                      const __grid_constant__ CUtensorMap k0run,
+                      const __grid_constant__ CUtensorMap k1run,
+                      const __grid_constant__ CUtensorMap v0run,
+                      const __grid_constant__ CUtensorMap v1run,
                       const int32_t *__restrict__ page_table, const int32_t *__restrict__ seq_len,
                       int f, const uint16_t *__restrict__ q_chunk, int hkv, int g, int max_pages,
                       int num_pages, float scale_log2, float *__restrict__ part_o,
@@ -156,6 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const uint32_t vmask = __ballot_sync(0xffffffffu, page >= 0);
             const uint32_t bytes = (uint32_t)__popc(vmask) * 2u * LY::kHalves * kBlock * 128u;
+            // four valid blocks on consecutive pages: one 4-page box per half
+            const int page0 = __shfl_sync(0xffffffffu, page, 0);
+            const bool run = __all_sync(0xffffffffu, lane >= kBlocksPerTile ||
+                                                          (page >= 0 && page == page0 + lane));
             if (lane == 0) {
                 stage_vmask[s] = vmask;
                 if (bytes == 0)
@@ -164,7 +175,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&kv_full[s], bytes);
             }
             __syncwarp();
-            if (page >= 0) {
+            if (run) {
+                if (lane == 0) {
+                    uint8_t *kt = kv_s + (size_t)s * 2 * LY::kKV;
+                    uint8_t *vt = kt + LY::kKV;
+                    tc::tma_load_4d(kt, &k0run, 0, 0, h, page0, &kv_full[s]);
+                    tc::tma_load_4d(vt, &v0run, 0, 0, h, page0, &kv_full[s]);
+                    if (LY::kHalves == 2) {
+                        tc::tma_load_4d(kt + LY::kKVHalf, &k1run, 0, 0, h, page0, &kv_full[s]);
+                        tc::tma_load_4d(vt + LY::kKVHalf, &v1run, 0, 0, h, page0, &kv_full[s]);
+                    }
+                }
+            } else if (page >= 0) {
                 const int y = (page * hkv + h) * kBlock;
                 uint8_t *kt = kv_s + (size_t)s * 2 * LY::kKV;
                 uint8_t *vt = kt + LY::kKV;
@@ -530,6 +552,7 @@ cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *pa
     cfg.attrs = attr;
     cfg.numAttrs = splits > 1 ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, rectify_tc_kernel<D>, maps[0], maps[1], maps[2], maps[3],
+                              maps[4], maps[5], maps[6], maps[7],
                               page_table, seq_len, f, (const uint16_t *)q_chunk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out,
                               lse, err);

@@ -43,6 +43,24 @@ bool make_kv_half_map(CUtensorMap *map, void *base, int half, int num_pages, int
     return r == CUDA_SUCCESS;
 }
 
+// The same channel half as a 4-D tensor (channels, tokens, heads, pages):
+// one box is the 16 tokens of one head on four consecutive pages, 128-byte
+// swizzled, laid out in shared memory exactly as four single-block boxes.
+bool make_kv_half_run_map(CUtensorMap *map, void *base, int half, int num_pages, int hkv, int d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    void *b = static_cast<uint8_t *>(base) + (size_t)half * 128;
+    const cuuint64_t dims[4] = {64, (cuuint64_t)kBlock, (cuuint64_t)hkv, (cuuint64_t)num_pages};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)kBlock * d * 2,
+                                   (cuuint64_t)hkv * kBlock * d * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)kBlock, 1, 4};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, b, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 resa_status_t check_config(const resa_config_t *cfg, Shape *s) {
@@ -280,12 +298,15 @@ resa_status_t resa_rectify_attention(const resa_config_t *cfg, const resa_cache_
     RESA_TRY(cuda_status(launch_rectify_writeback(s, cache->k, cache->v, cache->desc,
                                                   cache->page_table, cache->seq_len, f, k_new,
                                                   v_new, err, stream)));
-    CUtensorMap maps[4];
+    // 2-D single-block maps (K half 0, 1, V half 0, 1), then the 4-page maps
+    CUtensorMap maps[8];
     const int halves = s.d / 64;
     for (int hf = 0; hf < 2; ++hf) {
         const int use = hf < halves ? hf : 0;  // d = 64: one half, second map unused
         if (!make_kv_half_map(&maps[hf], cache->k, use, s.num_pages, s.hkv, s.d) ||
-            !make_kv_half_map(&maps[2 + hf], cache->v, use, s.num_pages, s.hkv, s.d))
+            !make_kv_half_map(&maps[2 + hf], cache->v, use, s.num_pages, s.hkv, s.d) ||
+            !make_kv_half_run_map(&maps[4 + hf], cache->k, use, s.num_pages, s.hkv, s.d) ||
+            !make_kv_half_run_map(&maps[6 + hf], cache->v, use, s.num_pages, s.hkv, s.d))
             return RESA_ERR_CUDA;
     }
     return cuda_status(launch_rectify_attention(

@@ -476,7 +476,8 @@ cudaError_t launch_decode_step_fused(const Shape &s, int G, void *k, void *v, vo
                                      const void *q, const void *k_new, const void *v_new,
                                      const int32_t *topk, int max_topk, float *out, float *lse,
                                      const StepBuffers &buf, cudaStream_t st);
-// maps: K half 0, K half 1, V half 0, V half 1 (2-D, 16 x 64 boxes, 128-byte swizzle).
+// maps: K half 0, K half 1, V half 0, V half 1 (2-D, 16 x 64 boxes, 128-byte swizzle),
+// then the same four as 4-D maps whose box is one head on four consecutive pages.
 cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap *maps,
                                      const int32_t *page_table, const int32_t *seq_len, int f,
                                      const void *q_chunk, int groups, int splits, float *part_o,

@@ -292,15 +292,21 @@ def test_all_blocks_equals_dense(cuda_device):
     np.testing.assert_allclose(out.cpu().numpy(), dense, rtol=0, atol=OUT_ATOL)
 
 
-@pytest.mark.parametrize("shape,ctx,f", [
-    ((4, 2, 64), [2049], 32),
-    ((28, 4, 128), [4096, 1000], 32),
-    ((28, 4, 128), [777], 13),
-    ((8, 1, 64), [40, 64, 300], 40),
-], ids=["tiny", "qwen-aligned", "qwen-unaligned", "whole-seq"])
-def test_rectify_matches_oracle(cuda_device, shape, ctx, f):
+@pytest.mark.parametrize("shape,ctx,f,paged", [
+    ((4, 2, 64), [2049], 32, True),
+    ((28, 4, 128), [4096, 1000], 32, True),
+    ((28, 4, 128), [777], 13, True),
+    ((8, 1, 64), [40, 64, 300], 40, True),
+    ((28, 4, 128), [4096, 1000], 32, False),
+    ((4, 2, 64), [2049, 77], 32, False),
+], ids=["tiny", "qwen-aligned", "qwen-unaligned", "whole-seq", "qwen-contiguous",
+        "tiny-contiguous"])
+def test_rectify_matches_oracle(cuda_device, shape, ctx, f, paged):
+    """Random page order takes the per-block tensor loads; the contiguous
+    layout takes the four-page loads wherever a tile's pages are consecutive
+    (and the per-block ones on the ragged last tile)."""
     hq, hkv, d = shape
-    p = inputs.make_decode_problem(20 + f, len(ctx), hq, hkv, d, 16, ctx, paged=True,
+    p = inputs.make_decode_problem(20 + f, len(ctx), hq, hkv, d, 16, ctx, paged=paged,
                                    needles=0, topk=[1] * len(ctx))
     cfg, lc, ws = setup_layer(p, cuda_device, max_chunk=f)
     L = p.ctx_len.clone()
