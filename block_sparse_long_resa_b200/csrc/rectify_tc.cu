@@ -146,20 +146,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = tmem_base_s;
 
     if (warp == 0) {  // ------------------------------------------------ TMA producer
+        // Page ids arrive 32 blocks (8 tiles) at a time, one id a lane, with
+        // the next window's load already in flight; they are checked when used.
+        constexpr int kWin = 32 / kBlocksPerTile;  // tiles per window
+        auto load_win = [&](int w) -> int {
+            const int blk = blk0 + w * 32 + lane;
+            return blk < blk1 ? page_table[(size_t)b * max_pages + blk] : -1;
+        };
+        int win_cur = ntiles > 0 ? load_win(0) : -1;
+        int win_next = ntiles > kWin ? load_win(1) : -1;
         bool ok = true;
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % kStages;
             if (i >= kStages) ok = mbar_wait_bounded(&kv_empty[s], ((i / kStages) - 1) & 1);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
+            if (i > 0 && i % kWin == 0) {
+                win_cur = win_next;
+                win_next = i + kWin < ntiles ? load_win(i / kWin + 1) : -1;
+            }
             const int blk = blk0 + i * kBlocksPerTile + lane;
-            int page = -1;
+            int page = __shfl_sync(0xffffffffu, win_cur, ((i % kWin) * kBlocksPerTile + lane) & 31);
             if (lane < kBlocksPerTile && blk < blk1) {
-                page = page_table[(size_t)b * max_pages + blk];
                 if (page < 0 || page >= num_pages) {
                     set_error(err, RESA_DEVERR_PAGE);
                     page = -1;
                 }
+            } else {
+                page = -1;
             }
             const uint32_t vmask = __ballot_sync(0xffffffffu, page >= 0);
             const uint32_t bytes = (uint32_t)__popc(vmask) * 2u * LY::kHalves * kBlock * 128u;
