@@ -66,6 +66,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown-reps", type=int, default=5)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the decode step over top-k fractions and the rectification over "
+                         "chunk lengths f, and compare the per-token cost with Eq. 6 (prints one "
+                         "JSON line, not the benchmark line)")
     return ap.parse_args(argv)
 
 
@@ -676,10 +680,110 @@ def kernel_breakdown(w, stream, device, reps):
     return res
 
 
+SWEEP_FRACS = (1 / 64, 1 / 32, 1 / 16, 1 / 10, 1 / 8, 1 / 4, 1 / 2, 1.0)
+SWEEP_CHUNKS = (8, 16, 32, 64)
+
+
+def run_sweep(args):
+    """Per-token cost of a ReSA cycle over (selected fraction s, rectification
+    period f) on the workload's layers: t_token = ((f-1) t_step(s) + t_rect(f)) / f,
+    next to the pages' memory model (ReSA summary §3.3, Eq. 6): bytes per token
+    relative to dense decoding = 1/b (block descriptors) + s (selected K/V)
+    + 1/f (one dense pass over the cache every f tokens)."""
+    import torch
+    from block_sparse_long_resa_b200 import resa as R
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = WORKLOADS[args.workload]
+    w = GpuWorkload(wl, 1, args.seed, device)
+    stream = torch.cuda.Stream(device)
+    n, B = w.layers, w.B
+    row = w.f - 2  # a decode step of cycle 0
+    # the cycle's earlier steps first, so that the blocks they complete carry
+    # their incrementally built descriptors, as in a real decode loop
+    for st in range(row):
+        for layer in range(n):
+            R.resa_decode_step(w.cfg, w.cache(layer, st), w.q[0, st, layer], w.kn[0, st, layer],
+                               w.vn[0, st, layer], w.topk_ptr(st), w.max_topk, w.out[layer], None,
+                               w.idx[layer], w.cnt[layer], w.ws)
+    torch.cuda.synchronize(device)
+    Ls = w.sched.decode_L(0, w.f - 2)
+    M = [(L - 1) // 16 for L in Ls]
+    rounds = max(1, -(-28 // n))
+
+    def timed(enqueue, calls, reps=5):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(rounds):
+                    enqueue()
+            g.replay()
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        return 1e3 * e0.elapsed_time(e1) / (reps * calls * rounds)
+
+    steps = []
+    for frac in SWEEP_FRACS:
+        k = [min(m, max(16, int(frac * m + 0.5))) for m in M]
+        kmax = max(k)
+        tk = torch.zeros(w.sched.Bpad, dtype=torch.int32, device=device)
+        tk[:B] = torch.tensor(k, dtype=torch.int32)
+        idx = [torch.empty(B, w.hkv, kmax + 1, dtype=torch.int32, device=device) for _ in range(n)]
+        cnt = [torch.empty(B, w.hkv, dtype=torch.int32, device=device) for _ in range(n)]
+        us = timed(lambda: [R.resa_decode_step(
+            w.cfg, w.cache(l, row), w.q[0, row, l], w.kn[0, row, l], w.vn[0, row, l], tk, kmax,
+            w.out[l], None, idx[l], cnt[l], w.ws) for l in range(n)], n)
+        steps.append({"s": frac, "topk": k[0] if B == 1 else k, "us_per_layer": us,
+                      "launches_per_step": R.resa_decode_step_launches(w.cfg, B, w.max_pages,
+                                                                       w.num_pages)})
+        del idx, cnt
+    t_dense = steps[-1]["us_per_layer"]
+    fmax = max(SWEEP_CHUNKS)
+    ws = torch.empty(R.resa_workspace_size(w.cfg, B, w.max_pages, fmax), dtype=torch.uint8,
+                     device=device)
+    R.resa_workspace_init(ws)
+    g = torch.Generator(device=device)
+    g.manual_seed(args.seed + 99)
+    rects = []
+    for f in SWEEP_CHUNKS:
+        qc = torch.randn(n, B, f, w.hq, w.d, generator=g, device=device).to(torch.bfloat16)
+        kc = torch.randn(n, B, f, w.hkv, w.d, generator=g, device=device).to(torch.bfloat16)
+        vc = torch.randn(n, B, f, w.hkv, w.d, generator=g, device=device).to(torch.bfloat16)
+        out = torch.empty(B, f, w.hq, w.d, device=device)
+        us = timed(lambda: [R.resa_rectify_attention(
+            w.cfg, w.cache(l, w.f - 1), f, qc[l], kc[l], vc[l], out, None, ws)
+            for l in range(n)], n)
+        rects.append({"f": f, "us_per_layer": us})
+        del qc, kc, vc, out
+    code = R.resa_check_device_status(w.ws, raise_on_error=False) | \
+        R.resa_check_device_status(ws, raise_on_error=False)
+    table = []
+    for st in steps[:-1]:
+        for rc in rects:
+            f = rc["f"]
+            t_tok = ((f - 1) * st["us_per_layer"] + rc["us_per_layer"]) / f
+            table.append({"s": st["s"], "f": f, "us_per_token_layer": t_tok,
+                          "measured_vs_dense": t_tok / t_dense,
+                          "eq6_bytes_vs_dense": 1 / 16 + st["s"] + 1 / f})
+    print(json.dumps({"sweep": args.workload, "layers": n, "context": Ls,
+                      "dense_step_us_per_layer": t_dense, "decode_steps": steps,
+                      "rectification": rects, "per_token": table,
+                      "device_error_word": code}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_resa(args)
 
 

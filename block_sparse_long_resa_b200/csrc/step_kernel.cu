@@ -158,7 +158,7 @@ __device__ __forceinline__ uint32_t composite(uint32_t k, int i) {
 
 // Indices of the small shared values.
 enum {
-    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVLo, kVHi, kVAB, kVGen, kVCount
+    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVLo, kVHi, kVAB, kVGen, kVCTop, kVCBot, kVCount
 };
 
 template <int D>
@@ -463,50 +463,73 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     uint32_t d1 = 0;
     int above = 0;
     if (need_hist) {
-        // a window of kThreadsAll bins below (this CTA's top digit + 128) and
-        // the touched range; the whole range is read only when the window
-        // does not hold it
+        // The boundary digit: the first read whose bins reach the unit's top
+        // digit and hold at least keff keys decides it, each read one round
+        // trip: (1) the kThreadsAll bins below this CTA's top digit + 128, read
+        // together with the touched range; (2) the kThreadsAll bins below the
+        // unit's top digit; (3) the whole touched range in contiguous chunks
+        // (a thread's loads all in flight), then the chunk that holds the
+        // boundary, one bin a thread.
         const uint32_t *hb = a.hist + (size_t)u * kHistBins;
-        const int wtop = min(kHistBins - 1, s_v[kVHi] + 128);
-        const int wbot = max(0, wtop - (kThreadsAll - 1));
+        const int wtop1 = min(kHistBins - 1, s_v[kVHi] + 128);
         const uint32_t emin = __ldcg(&a.hist_range[2 * u]), emax = __ldcg(&a.hist_range[2 * u + 1]);
-        const int wd = wtop - tid;
-        const uint32_t wc = wd >= wbot ? __ldcg(&hb[wd]) : 0u;
+        const int wd1 = wtop1 - tid;
+        const uint32_t wc1 = wd1 >= 0 ? __ldcg(&hb[wd1]) : 0u;
         const int dlo = kHistBins - (int)emin, dhi = (int)emax - 1;
-        const bool covered = dlo >= wbot && dhi <= wtop;  // uniform over the CTA
-        uint32_t total, above_me, loc;
-        int top, bot;
-        if (covered) {
-            loc = wc;
-            top = wd;
-            bot = wd;
-        } else {
-            const int nb = dhi >= dlo ? dhi - dlo + 1 : 0;
-            const int chunk = (nb + kThreadsAll - 1) / kThreadsAll;
-            top = dhi - tid * chunk;
-            bot = max(dlo, top - chunk + 1);
-            loc = 0;
-            #pragma unroll 1
-            for (int d = top; d >= bot; --d) loc += __ldcg(&hb[d]);
-        }
-        above_me = cta_scan(loc, s_scan, total);  // keys in the bins above this thread's
-        if (above_me < (uint32_t)keff && (uint32_t)keff <= above_me + loc) {
-            uint32_t cum = above_me;
-            #pragma unroll 1
-            for (int d = top; d >= bot; --d) {
-                const uint32_t c = covered ? wc : __ldcg(&hb[d]);
-                if (cum + c >= (uint32_t)keff) {
-                    s_v[kVD1] = d;
-                    s_v[kVAB] = (int)cum;  // keys above the boundary digit
-                    break;
-                }
-                cum += c;
-            }
-        }
         if (tid == 0) {
             s_v[kVDlo] = dlo;
             s_v[kVDhi] = dhi;
-            s_v[kVHistOk] = total == (uint32_t)M ? 1 : 0;
+            s_v[kVCTop] = dhi;
+            s_v[kVCBot] = dhi + 1;
+        }
+        // a descending scan over kThreadsAll bins (thread t: bin wtop - t)
+        auto window = [&](int wtop, uint32_t c) -> bool {
+            uint32_t tot;
+            const uint32_t before = cta_scan(c, s_scan, tot);
+            if (c > 0 && before < (uint32_t)keff && (uint32_t)keff <= before + c) {
+                s_v[kVD1] = wtop - tid;
+                s_v[kVAB] = (int)before;  // keys above the boundary digit
+            }
+            if (tid == 0 && tot > (uint32_t)M) s_v[kVHistOk] = 0;
+            return tot >= (uint32_t)keff;
+        };
+        bool found = dhi <= wtop1 && window(wtop1, wc1);  // uniform over the CTA
+        if (!found) {
+            const int wd2 = dhi - tid;
+            found = window(dhi, wd2 >= 0 ? __ldcg(&hb[wd2]) : 0u);
+        }
+        if (!found) {
+            const int nb = dhi >= dlo ? dhi - dlo + 1 : 0;
+            const int chunk = (nb + kThreadsAll - 1) / kThreadsAll;  // <= kThreadsAll bins
+            const int top = dhi - tid * chunk, bot = max(dlo, top - chunk + 1);
+            uint32_t loc = 0;
+#pragma unroll 1
+            for (int d0 = top; d0 >= bot; d0 -= 16) {
+                uint32_t c16[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) c16[e] = d0 - e >= bot ? __ldcg(&hb[d0 - e]) : 0u;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) loc += c16[e];
+            }
+            uint32_t total;
+            const uint32_t before = cta_scan(loc, s_scan, total);
+            if (loc > 0 && before < (uint32_t)keff && (uint32_t)keff <= before + loc) {
+                s_v[kVCTop] = top;
+                s_v[kVCBot] = bot;
+                s_v[kVAB] = (int)before;
+            }
+            if (tid == 0) s_v[kVHistOk] = total == (uint32_t)M ? 1 : 0;
+            __syncthreads();
+            const int ctop = s_v[kVCTop], cbot = s_v[kVCBot];
+            const uint32_t cbefore = (uint32_t)s_v[kVAB];
+            const int d = ctop - tid;
+            const uint32_t c = d >= cbot ? __ldcg(&hb[d]) : 0u;
+            uint32_t tot2;
+            const uint32_t b2 = cta_scan(c, s_scan, tot2);
+            if (c > 0 && cbefore + b2 < (uint32_t)keff && (uint32_t)keff <= cbefore + b2 + c) {
+                s_v[kVD1] = d;
+                s_v[kVAB] = (int)(cbefore + b2);
+            }
         }
     }
     cp_async_wait<0>();

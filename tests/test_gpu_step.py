@@ -73,6 +73,37 @@ def test_concentrated_selection_moves_blocks_between_ctas(cuda_device):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
 
 
+@pytest.mark.parametrize("outlier", [0.0, 60.0], ids=["zero-blocks", "zero-blocks+top-outlier"])
+def test_wide_score_range(cuda_device, outlier):
+    """Blocks of all-zero keys score 0, thousands of histogram bins below the
+    rest; with a block pushed far along the pooled query the unit's top digit
+    also lies far above the bulk.  The boundary search then needs its second
+    window or the chunked read of the whole touched range."""
+    p = inputs.make_decode_problem(71, 1, 28, 4, 128, 16, [65536], needles=0)
+    for blk in (3, 500, 2047, 3000):
+        p.k_cache[int(p.page_table[0, blk])] = 0
+    if outlier:
+        qbar = p.q.float().view(1, 4, 7, 128).mean(2)[0]
+        u = qbar / qbar.norm(dim=-1, keepdim=True)
+        page = int(p.page_table[0, 1234])
+        p.k_cache[page] = (p.k_cache[page].float() + outlier * u[:, None, :]).to(torch.bfloat16)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    k = int(p.topk[0])
+    out, lse, idx, cnt = run_step(p, lc, cfg, ws, cuda_device, p.topk, k, L)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    r = o.decode_step(p.q, p.k_new, p.v_new, p.topk, L, k)
+    gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    same = check_block_sets(gidx, gcnt, r["block_idx"], r["block_cnt"], r["scores"], p.topk, L, 16)
+    ref, ref_lse = (r["out"], r["lse"]) if same else o.sparse_attention(p.q, gidx, gcnt, L)
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+    if outlier:
+        assert (gidx[0, :, :k] == 1234).any(axis=1).all()
+
+
 @pytest.mark.parametrize("ctx,topk,max_topk,d", [
     ([333, 257, 1999], [5, 0, 10**6], 80, 64),  # candidate lists in shared memory
     ([65536], [300], 300, 64),                   # 4096 tied candidates
