@@ -73,12 +73,14 @@ def test_concentrated_selection_moves_blocks_between_ctas(cuda_device):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
 
 
-@pytest.mark.parametrize("outlier", [0.0, 60.0], ids=["zero-blocks", "zero-blocks+top-outlier"])
+@pytest.mark.parametrize("outlier", [0.0, 60.0, 300.0],
+                         ids=["zero-blocks", "top-outlier-2-octaves", "top-outlier-4-octaves"])
 def test_wide_score_range(cuda_device, outlier):
     """Blocks of all-zero keys score 0, thousands of histogram bins below the
-    rest; with a block pushed far along the pooled query the unit's top digit
-    also lies far above the bulk.  The boundary search then needs its second
-    window or the chunked read of the whole touched range."""
+    rest (the first window still holds the boundary).  A block pushed along
+    the pooled query puts the unit's top digit about two octaves (the window
+    below it holds the boundary) or four octaves (more than a window: the
+    chunked read of the whole touched range) above the bulk."""
     p = inputs.make_decode_problem(71, 1, 28, 4, 128, 16, [65536], needles=0)
     for blk in (3, 500, 2047, 3000):
         p.k_cache[int(p.page_table[0, blk])] = 0
