@@ -14,25 +14,26 @@
 //     the fp32 scores go to shared memory and to the unit's key row in the
 //     workspace; their top 16 bits feed the unit's histogram (aggregated per
 //     CTA in a shared-memory hash table, then one atomic per distinct digit).
-//  2. Unit barrier.  In one round trip every CTA reads the histogram bins
-//     around its own top digit and the unit's whole key row (into the idle
-//     K/V ring).  The boundary digit d1 holding the k-th largest key splits
-//     the blocks into definite (above d1) and candidates (at d1); a radix
-//     select over the candidates' composite keys (low 16 key bits, then the
-//     complement of the block id: larger = higher score or, on equal scores,
-//     lower block id) gives the exact threshold.  Every CTA holds every key,
-//     so every CTA computes the same canonical work layout without another
-//     exchange: CTA x' keeps its own selected blocks (definite, then
-//     qualifying candidates, each in block order) up to the fair share
-//     F = ceil((k + 1) / G); the rest is the pool (CTA order, then the current
-//     block), and CTA x takes the slice of the pool that fills its share.
-//  3. The eight decode warps attend to their F blocks with per-warp 3-stage
-//     K/V rings of 16-byte cp.async copies and swapped m16n8k16 MMAs
-//     (attn_common.cuh); the other four warps write the block list (ascending)
-//     and the count.
-//  4. The CTA merges its warps into a partial (o / l, log2-sum-exp); after a
-//     second unit barrier each of the first g * d/32 CTAs merges one (query
-//     row, 32 channels) slice of the unit's G partials; the others leave.
+//  2. Unit counter (one add, then a bounded poll).  In one round trip every
+//     CTA reads the histogram bins around its own top digit and the unit's
+//     whole key row (into the idle K/V ring).  The boundary digit d1 holding
+//     the k-th largest key splits the blocks into definite (above d1) and
+//     candidates (at d1); one pass over the keys counts the definite blocks of
+//     each 32-block group and collects the candidates, and a radix select over
+//     the candidates' composite keys (low 16 key bits, then the complement of
+//     the block id: larger = higher score or, on equal scores, lower block id)
+//     gives the exact threshold.  Every CTA holds every key, so every CTA
+//     computes the same ordered work list without another exchange: the
+//     selected blocks in ascending order, then the current block; CTA x takes
+//     the contiguous slice [x W / G, (x + 1) W / G) of its W items.
+//  3. The eight decode warps attend to the slice with per-warp 3-stage K/V
+//     rings of 16-byte cp.async copies and swapped m16n8k16 MMAs
+//     (attn_common.cuh); the other four warps write the slice's part of the
+//     block list (ascending) and the count.
+//  4. The CTA merges its warps into a partial (o / l, log2-sum-exp) written as
+//     generation-tagged 64-bit words; each of the first g * d/32 CTAs polls
+//     the words of one (query row, 32 channels) slice of the unit's G partials
+//     until every tag is current and merges them; the others leave.
 //
 // The append (K/V of the decode token at position L-1 and the fold of its key
 // into the current block's descriptor) is done by one warp of CTA G-1 of each
@@ -158,7 +159,7 @@ __device__ __forceinline__ uint32_t composite(uint32_t k, int i) {
 
 // Indices of the small shared values.
 enum {
-    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVLo, kVHi, kVAB, kVGen, kVCTop, kVCBot, kVCount
+    kVD1 = 0, kVDlo, kVDhi, kVHistOk, kVOk, kVLo, kVHi, kVAB, kVGen, kVCTop, kVCBot, kVG0, kVCount
 };
 
 template <int D>
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         s_v[kVHi] = -1;
         s_v[kVD1] = 0;
         s_v[kVHistOk] = 1;
+        s_v[kVG0] = (M + 31) >> 5;  // no group (the selection loop then reads nothing)
     }
     // Q^T fragments for the decode warps: head lane/4 (zero beyond g),
     // channels 2*(lane%4)+{0,1} (+8) of each 16-channel slice.
@@ -377,7 +379,17 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     if (tid == 0) s_v[kVGen] = (int)gen;
     __syncthreads();
     const bool need_hist = mode == kModeMid;
+    // The rings after scoring: the unit's keys, its page ids (block i at
+    // upages_s[i + pshift]), the warps' candidate segments, the radix bins.
+    uint32_t *upages_s = ukeys_s + ((M + 3) & ~3);
+    const int pshift = (int)(prow & 3);
+    const int cap = kCandPerWarp;
+    uint32_t *cand_s = upages_s + ((M + pshift + 3) & ~3);       // [kWarpsAll][cap]
+    uint32_t *rh = cand_s + kWarpsAll * cap;                     // [2048]
     if (need_hist) {
+        // the first radix digit's bins are counted during the pass
+        #pragma unroll 1
+        for (int i = tid; i < 2048; i += kThreadsAll) rh[i] = 0;
         // per-CTA histogram of the keys' top 16 bits, then one global atomic
         // per distinct digit
         int lo = 0x7fffffff, hi = -1;
@@ -426,11 +438,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
 
     // ---- 2. the unit's page ids (an input: copied while the unit's CTAs
     // meet), unit barrier, then the unit's keys and histogram ----
-    // page id of block i at upages_s[i + pshift]: the row is copied from the
-    // 16-byte boundary at or below its start, the tail (inside the row) with
-    // 4-byte copies
-    uint32_t *upages_s = ukeys_s + ((M + 3) & ~3);
-    const int pshift = (int)(prow & 3);
+    // the page-id row is copied from the 16-byte boundary at or below its
+    // start, the tail (inside the row) with 4-byte copies
     if (mode == kModeAll || mode == kModeMid) {
         const int32_t *prow_al = a.page_table + (prow - pshift);
         const int nfull = (M + pshift) / 4;
@@ -557,42 +566,65 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     uint32_t tau = 0xffffffffu;
     int rem = 0;
     if (mode == kModeMid) {
-        // One pass over the unit's keys, a 32-block group per warp step (one
-        // key a lane, four groups in flight): the definite count of each group
-        // and the candidates' composite keys, appended to the warp's segment.
-        const int KW = (ngroups + kWarpsAll - 1) / kWarpsAll * 32;  // keys one warp sees at most
-        uint32_t *cand_s = upages_s + ((M + pshift + 3) & ~3);      // [kWarpsAll][min(KW, cap)]
-        const int cap = min(KW, kCandPerWarp);
-        const uint32_t lt_mask = (1u << lane) - 1u;
+        // One pass over the unit's keys, a 32-block group per lane: the
+        // group's definite count and a mask of its candidates from the
+        // lane's 32 keys (eight 16-byte loads, their order rotated by lane so
+        // that each quarter-warp's loads cover all banks once), then the
+        // candidates' composite keys appended to the warp's segment (offsets
+        // by a warp scan) and counted in the bins of the first radix digit.
+        // Per key only full-rate integer operations: a key's digit is above
+        // d1 iff the key is above hi1, equal to d1 iff key - lo1 < 2^16.
+        // (A ballot-per-key pass was bound by the quarter-rate vote and
+        // population-count units.)
+        const uint32_t lo1 = d1 << 16, hi1 = lo1 | 0xffffu;
         uint32_t *seg = cand_s + warp * cap;
         int nseg = 0;
         #pragma unroll 1
-        for (int g0 = warp; g0 < ngroups; g0 += 4 * kWarpsAll) {
-            uint32_t kk[4], bd[4], bc[4];
+        for (int q0 = warp * 32; q0 < ngroups; q0 += kThreadsAll) {
+            const int q = q0 + lane;
+            const int lim = M - q * 32;  // keys of group q: min(32, lim)
+            const uint32_t *gk = ukeys_s + (size_t)q * 32;
+            int nd = 0;
+            uint32_t cm = 0;  // bit 4j + e: key 4 ((j + lane) & 7) + e of the group
+            if (lim >= 32) {
 #pragma unroll
-            for (int u4 = 0; u4 < 4; ++u4) {
-                const int i = (g0 + kWarpsAll * u4) * 32 + lane;
-                kk[u4] = i < M ? ukeys_s[i] : 0u;
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 k4 = *reinterpret_cast<const uint4 *>(gk + 4 * ((j + lane) & 7));
+                    const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        nd += kk[e] > hi1 ? 1 : 0;
+                        cm |= kk[e] - lo1 < 0x10000u ? (1u << (4 * j + e)) : 0u;
+                    }
+                }
+            } else if (lim > 0) {  // the unit's last, ragged group
+                #pragma unroll 1
+                for (int t = 0; t < lim; ++t) {
+                    const uint32_t k = gk[t];
+                    nd += k > hi1 ? 1 : 0;
+                    const int j = ((t >> 2) - lane) & 7;
+                    cm |= k - lo1 < 0x10000u ? (1u << (4 * j + (t & 3))) : 0u;
+                }
             }
+            if (lim > 0) gcnt[q] = nd;
+            const int nc = __popc(cm);
+            int incl = nc;
 #pragma unroll
-            for (int u4 = 0; u4 < 4; ++u4) {
-                const int i = (g0 + kWarpsAll * u4) * 32 + lane;
-                const uint32_t dg = kk[u4] >> 16;
-                bd[u4] = __ballot_sync(0xffffffffu, i < M && dg > d1);
-                bc[u4] = __ballot_sync(0xffffffffu, i < M && dg == d1);
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
             }
-            // lane u4 < 4 stores group u4's definite count
-            uint32_t mine = bd[0];
-#pragma unroll
-            for (int u4 = 1; u4 < 4; ++u4) mine = lane == u4 ? bd[u4] : mine;
-            const int gme = g0 + kWarpsAll * lane;
-            if (lane < 4 && gme < ngroups) gcnt[gme] = __popc(mine);
-#pragma unroll
-            for (int u4 = 0; u4 < 4; ++u4) {
-                const int i = (g0 + kWarpsAll * u4) * 32 + lane;
-                const int r = nseg + __popc(bc[u4] & lt_mask);
-                if (((bc[u4] >> lane) & 1u) && r < cap) seg[r] = composite(kk[u4], i);
-                nseg += __popc(bc[u4]);
+            int r = nseg + incl - nc;
+            nseg += __shfl_sync(0xffffffffu, incl, 31);
+            #pragma unroll 1
+            while (cm != 0u) {
+                const int bit = __ffs(cm) - 1;
+                cm &= cm - 1u;
+                const int i = q * 32 + 4 * (((bit >> 2) + lane) & 7) + (bit & 3);
+                const uint32_t cmp = composite(ukeys_s[i], i);
+                atomicAdd(&rh[cmp >> 21], 1u);
+                if (r < cap) seg[r] = cmp;
+                ++r;
             }
         }
         if (lane == 0) s_seg[warp] = nseg;
@@ -640,10 +672,10 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             rem = max(0, min(rem, NC));
         }
         if (rem > 0) {
-            // digits of 11, 8, 8 and 5 bits, most significant first; bins in
-            // the rings after the candidates; the digit holding the remaining-th
-            // largest candidate is found by one CTA-wide scan in descending order
-            uint32_t *rh = cand_s + kWarpsAll * cap;  // [2048]
+            // digits of 11, 8, 8 and 5 bits, most significant first (the
+            // first one's bins were filled by the pass); the digit holding the
+            // remaining-th largest candidate is found by one CTA-wide scan in
+            // descending order
             uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)rem;
             int shift = 32;
             #pragma unroll 1
@@ -651,13 +683,15 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                 const int width = pass == 0 ? 11 : pass == 3 ? 5 : 8;
                 shift -= width;
                 const int nb = 1 << width;
-                #pragma unroll 1
-                for (int i = tid; i < nb; i += kThreadsAll) rh[i] = 0;
-                __syncthreads();
-                for_each_cand([&](uint32_t c) {
-                    if ((c & pmask) == prefix) atomicAdd(&rh[(c >> shift) & (uint32_t)(nb - 1)], 1u);
-                });
-                __syncthreads();
+                if (pass > 0) {
+                    #pragma unroll 1
+                    for (int i = tid; i < nb; i += kThreadsAll) rh[i] = 0;
+                    __syncthreads();
+                    for_each_cand([&](uint32_t c) {
+                        if ((c & pmask) == prefix) atomicAdd(&rh[(c >> shift) & (uint32_t)(nb - 1)], 1u);
+                    });
+                    __syncthreads();
+                }
                 constexpr int kPer = (2048 + kThreadsAll - 1) / kThreadsAll;
                 uint32_t cnt[kPer], sum = 0;
 #pragma unroll
@@ -692,7 +726,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             });
         }
         __syncthreads();
-        // exclusive prefix of the selected count over the groups
+        // exclusive prefix of the selected count over the groups; the group
+        // that holds item s0 (selected, so of nonzero count) is noted
         {
             constexpr int RG = (kMaxGroups + kThreadsAll - 1) / kThreadsAll;
             const int q0 = tid * RG;
@@ -707,7 +742,10 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             uint32_t run = cta_scan(sum, s_scan, tot);
 #pragma unroll
             for (int r = 0; r < RG; ++r) {
-                if (q0 + r < ngroups) gpre[q0 + r] = (int)run;
+                if (q0 + r < ngroups) {
+                    gpre[q0 + r] = (int)run;
+                    if (run <= (uint32_t)s0 && (uint32_t)s0 < run + (uint32_t)v[r]) s_v[kVG0] = q0 + r;
+                }
                 run += v[r];
             }
         }
@@ -716,12 +754,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         // gpre[q] < e and gpre[q] + gcnt[q] > s0, one warp per group
         const int e_sel = min(s1, keff);
         if (s0 < e_sel) {
-            int lo = 0, hi = ngroups - 1;  // first group ending past s0
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (gpre[mid] + gcnt[mid] > s0) hi = mid;
-                else lo = mid + 1;
-            }
+            const uint32_t lt_mask = (1u << lane) - 1u;
+            const int lo = s_v[kVG0];  // s0 < keff: exactly one group holds item s0
             #pragma unroll 1
             for (int q = lo + warp; q < ngroups && gpre[q] < e_sel; q += kWarpsAll) {
                 const int i = q * 32 + lane;
