@@ -566,12 +566,13 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     uint32_t tau = 0xffffffffu;
     int rem = 0;
     if (mode == kModeMid) {
-        // One pass over the unit's keys, a 32-block group per lane: the
-        // group's definite count and a mask of its candidates from the
-        // lane's 32 keys (eight 16-byte loads, their order rotated by lane so
-        // that each quarter-warp's loads cover all banks once), then the
-        // candidates' composite keys appended to the warp's segment (offsets
-        // by a warp scan) and counted in the bins of the first radix digit.
+        // One pass over the unit's keys, half a 32-block group per lane: the
+        // half's definite count (two lanes' counts make the group's) and a
+        // mask of its candidates from the lane's 16 keys (four 16-byte loads,
+        // their order rotated by lane pair so that each quarter-warp's loads
+        // cover all banks once), then the candidates' composite keys appended
+        // to the warp's segment (offsets by a warp scan) and counted in the
+        // bins of the first radix digit.
         // Per key only full-rate integer operations: a key's digit is above
         // d1 iff the key is above hi1, equal to d1 iff key - lo1 < 2^16.
         // (A ballot-per-key pass was bound by the quarter-rate vote and
@@ -580,33 +581,40 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         uint32_t *seg = cand_s + warp * cap;
         int nseg = 0;
         #pragma unroll 1
-        for (int q0 = warp * 32; q0 < ngroups; q0 += kThreadsAll) {
-            const int q = q0 + lane;
-            const int lim = M - q * 32;  // keys of group q: min(32, lim)
-            const uint32_t *gk = ukeys_s + (size_t)q * 32;
+        for (int h0 = warp * 32; h0 < 2 * ngroups; h0 += kThreadsAll) {
+            const int hg = h0 + lane;          // half-group: keys [16 hg, 16 hg + 16)
+            const int q = hg >> 1;
+            const int lim = M - hg * 16;       // keys of the half: min(16, lim)
+            const uint32_t *gk = ukeys_s + (size_t)hg * 16;
+            const int rot = lane >> 1;
             int nd = 0;
-            uint32_t cm = 0;  // bit 4j + e: key 4 ((j + lane) & 7) + e of the group
-            if (lim >= 32) {
+            uint32_t cm = 0;  // bit 4j + e: key 4 ((j + rot) & 3) + e of the half
+            if (lim >= 16) {
+                int nde[4] = {0, 0, 0, 0};
+                uint32_t cme[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 k4 = *reinterpret_cast<const uint4 *>(gk + 4 * ((j + lane) & 7));
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 k4 = *reinterpret_cast<const uint4 *>(gk + 4 * ((j + rot) & 3));
                     const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        nd += kk[e] > hi1 ? 1 : 0;
-                        cm |= kk[e] - lo1 < 0x10000u ? (1u << (4 * j + e)) : 0u;
+                        nde[e] += kk[e] > hi1 ? 1 : 0;
+                        cme[e] |= kk[e] - lo1 < 0x10000u ? (1u << (4 * j + e)) : 0u;
                     }
                 }
-            } else if (lim > 0) {  // the unit's last, ragged group
+                nd = (nde[0] + nde[1]) + (nde[2] + nde[3]);
+                cm = (cme[0] | cme[1]) | (cme[2] | cme[3]);
+            } else if (lim > 0) {
                 #pragma unroll 1
                 for (int t = 0; t < lim; ++t) {
                     const uint32_t k = gk[t];
                     nd += k > hi1 ? 1 : 0;
-                    const int j = ((t >> 2) - lane) & 7;
+                    const int j = ((t >> 2) - rot) & 3;
                     cm |= k - lo1 < 0x10000u ? (1u << (4 * j + (t & 3))) : 0u;
                 }
             }
-            if (lim > 0) gcnt[q] = nd;
+            const int ng = nd + __shfl_xor_sync(0xffffffffu, nd, 1);
+            if ((lane & 1) == 0 && q < ngroups) gcnt[q] = ng;
             const int nc = __popc(cm);
             int incl = nc;
 #pragma unroll
@@ -620,7 +628,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
             while (cm != 0u) {
                 const int bit = __ffs(cm) - 1;
                 cm &= cm - 1u;
-                const int i = q * 32 + 4 * (((bit >> 2) + lane) & 7) + (bit & 3);
+                const int i = hg * 16 + 4 * (((bit >> 2) + rot) & 3) + (bit & 3);
                 const uint32_t cmp = composite(ukeys_s[i], i);
                 atomicAdd(&rh[cmp >> 21], 1u);
                 if (r < cap) seg[r] = cmp;
