@@ -436,8 +436,14 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     __syncthreads();
 
-    // ---- 2. the unit's page ids (an input: copied while the unit's CTAs
-    // meet), unit barrier, then the unit's keys and histogram ----
+    // ---- 2. unit barrier (the unit's page ids, an input, are copied while
+    // the unit's CTAs meet), then the unit's keys and histogram ----
+    // The arrival's fence comes before the page-id copies are issued, so it
+    // does not wait for them.
+    if (G > 1 && need_hist && tid == 0) {
+        __threadfence();  // the CTA's key row and histogram atomics, ordered by the barrier above
+        atomicAdd(&ubar[0], 1ull);
+    }
     // the page-id row is copied from the 16-byte boundary at or below its
     // start, the tail (inside the row) with 4-byte copies
     if (mode == kModeAll || mode == kModeMid) {
@@ -450,11 +456,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     cp_async_commit();
     if (G > 1 && need_hist) {
-        if (tid == 0) {
-            __threadfence();  // the CTA's key row and histogram atomics, ordered by the barrier above
-            atomicAdd(&ubar[0], 1ull);
-            s_v[kVOk] = unit_wait_count(&ubar[0], G) ? 1 : 0;
-        }
+        if (tid == 0) s_v[kVOk] = unit_wait_count(&ubar[0], G) ? 1 : 0;
         __syncthreads();
         if (!s_v[kVOk]) {
             if (tid == 0) set_error(a.err, RESA_DEVERR_TIMEOUT);
