@@ -894,21 +894,28 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         unsigned long long *pp = a.part + (size_t)cta * kStepMaxGroup * PS;
         const int hq = hkv * g;
         // per row: the warps' scale factors exp2(m_w - m*), 1 / l and the
-        // log2-sum-exp, once
-        if (tid < g) {
-            const int r = tid;
+        // log2-sum-exp, once, by one warp: lane (w4, r) takes decode warps
+        // w4 and w4 + 4 of row r
+        static_assert(kDW == 8 && kStepMaxGroup == 8, "one warp covers 8 rows x 8 decode warps");
+        if (warp == 0) {
+            const int r = lane & 7, w4 = lane >> 3;
             float mstar = -INFINITY;
 #pragma unroll
             for (int w = 0; w < kDW; ++w) mstar = fmaxf(mstar, mw[w * kMaxGroup + r]);
             float lsum = 0.f;
 #pragma unroll
-            for (int w = 0; w < kDW; ++w) {
+            for (int k = 0; k < 2; ++k) {
+                const int w = w4 + 4 * k;
                 const float sc = mstar != -INFINITY ? exp2f(mw[w * kMaxGroup + r] - mstar) : 0.f;
                 s_sc[w][r] = sc;
                 lsum += lw[w * kMaxGroup + r] * sc;
             }
-            s_rinv[r] = lsum > 0.f ? 1.f / lsum : 0.f;
-            s_rlse[r] = lsum > 0.f ? mstar + log2f(lsum) : -INFINITY;
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+            if (w4 == 0) {
+                s_rinv[r] = lsum > 0.f ? 1.f / lsum : 0.f;
+                s_rlse[r] = lsum > 0.f ? mstar + log2f(lsum) : -INFINITY;
+            }
         }
         __syncthreads();
 #pragma unroll 1
@@ -963,8 +970,9 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
                 good = good && tag_of(wl) == tag;
                 lse_s[tid] = __uint_as_float((uint32_t)wl);
             }
-            ok = __syncthreads_and(good) != 0;
+            ok = __all_sync(0xffffffffu, good);  // each warp polls its own words
         }
+        ok = __syncthreads_and(ok) != 0;  // lse_s is complete
         all_ok = all_ok && ok;
         float mstar = -INFINITY;
 #pragma unroll 1
