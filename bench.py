@@ -584,7 +584,7 @@ def run_resa(args):
                  [x for x in L_state])
         cpu = cpu_baseline(wl, args.seed, state)
 
-    per_token_us = ms / K / wl["f"] if world == 1 else ms_local / K / wl["f"]
+    per_token_us = 1e3 * (ms if world == 1 else ms_local) / K / wl["f"]  # one sequence's token latency
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
