@@ -71,6 +71,9 @@ constexpr int step_unit_keys(int d) {
 // Row stride (in keys) of a unit's key row in the workspace: 16-byte rows.
 inline int step_key_stride(int max_pages) { return (max_pages + 3) & ~3; }
 constexpr int kStepMaxGroup = 8;  // one n8 MMA tile of query heads (register budget)
+// Words per unit of the fused step's counter block: one 128-byte line each, so
+// the units' counters, polled by all their CTAs, do not share a line.
+constexpr int kStepBarWords = 16;
 // CTAs per unit of the fused step, or 0 when the shape needs the unfused path.
 inline int step_ctas_per_unit(int units, int g, int d, int max_pages, int sms) {
     if (g > kStepMaxGroup || max_pages > kStepMaxPages || units <= 0) return 0;
@@ -120,7 +123,7 @@ struct WsLayout {
     size_t sel_cnt;      // i32 [B][Hkv]
     size_t dec_o;        // f32 [partials][kMaxGroup][d]: per split, or per warp when spread
     size_t dec_lse;      // f32 [partials][kMaxGroup] lse, or float2 (row max, row sum) when spread
-    size_t step_bars;    // u64 [B][Hkv][4] unit counter (zero between calls) and generation of the fused step
+    size_t step_bars;    // u64 [B][Hkv][kStepBarWords] unit counter (zero between calls) and generation of the fused step
     size_t step_keys;    // u32 [B][Hkv][step_key_stride(max_pages)] block score keys of the fused step
     size_t step_part;    // u64 [kNumSms][kStepMaxGroup][d + 1] tagged per-CTA partials of the fused step
     size_t rect_o;       // f32 [B][Hkv][row_groups][rect_splits][kRectRowsPerCta][d]
@@ -158,7 +161,7 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     const size_t parts = decode_partials((int)units, w.dec_splits);
     w.dec_o = take(parts * kMaxGroup * d * 4);
     w.dec_lse = take(parts * kMaxGroup * 2 * 4);  // (lse) or (row max, row sum) pairs
-    w.step_bars = take(units * 4 * 8);
+    w.step_bars = take(units * kStepBarWords * 8);
     w.step_keys = take(units * (size_t)step_key_stride(max_pages) * 4);
     w.step_part = take((size_t)kNumSms * kStepMaxGroup * (d + 1) * 8);
     size_t rect_rows = units * w.row_tiles * w.rect_splits * kRectRowsPerCta;
@@ -466,7 +469,7 @@ cudaError_t launch_sparse_decode(const Shape &s, const void *k, const void *v,
 struct StepBuffers {
     int32_t *block_idx, *block_cnt;  // selection output [B][Hkv][max_topk+1], [B][Hkv]
     uint32_t *hist, *hist_range;
-    unsigned long long *bars;   // [B][Hkv][4]
+    unsigned long long *bars;   // [B][Hkv][kStepBarWords]
     uint32_t *ukeys;
     unsigned long long *part;   // [kNumSms][kStepMaxGroup][d + 1]
     uint32_t *err;

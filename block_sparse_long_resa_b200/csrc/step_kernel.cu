@@ -90,7 +90,7 @@ struct StepArgs {
     int32_t *block_idx, *block_cnt;
     float *out, *lse;
     uint32_t *hist, *hist_range;
-    unsigned long long *bars;  // [units][4]: scored count, -, -, generation
+    unsigned long long *bars;  // [units][kStepBarWords]: scored count, -, -, generation, padding
     uint32_t *ukeys;           // [units][key_stride] every block's key
     unsigned long long *part;  // [units * G][kStepMaxGroup][D + 1] tagged partial (o, then lse)
     uint32_t *err;
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     }
     __syncthreads();
     pdl_wait();  // descriptors and K/V may be written by the preceding kernels
-    unsigned long long *ubar = a.bars + 4 * (size_t)u;
+    unsigned long long *ubar = a.bars + kStepBarWords * (size_t)u;
     const uint32_t gen = tid == 0 ? (uint32_t)ld_relaxed_u64(&ubar[3]) : 0u;  // used after scoring
 
     // ---- 1. scoring (+ the append, whose descriptor loads are issued first) ----
