@@ -35,7 +35,9 @@
  *   set bits of an error word in the workspace and the offending item is
  *   skipped or clamped (never a trap); read and clear the word with
  *   resa_check_device_status.  Device waits are bounded; a wait that gives up
- *   sets RESA_DEVERR_TIMEOUT.
+ *   sets RESA_DEVERR_TIMEOUT.  The outputs of a call that timed out are
+ *   undefined, and its workspace may hold words of that call: zero it again
+ *   with resa_workspace_init before the next call.
  * Supported shapes.  head_dim in {64, 128}; block_size 16; group size
  *   g = Hq / Hkv in 1 .. 16; Hkv <= 8.  Other shapes return
  *   RESA_ERR_UNSUPPORTED.
@@ -179,8 +181,9 @@ RESA_API resa_status_t resa_rectify_attention(const resa_config_t *cfg, const re
  * G = 148 / (batch * Hkv) CTAs per (sequence, kv head) scores at most 1024
  * blocks) the whole step is one cooperative launch: the CTAs of a (sequence,
  * kv head) score their share of the descriptors, agree on the selection
- * through two bounded barriers in the workspace and split the selected
- * blocks evenly; other shapes run as three launches (append fused with the
+ * through one bounded counter in the workspace, split the selected blocks
+ * evenly and hand their partial results over as words tagged with the
+ * call's generation; other shapes run as three launches (append fused with the
  * scores, selection, sparse decode).  resa_decode_step_launches tells which.
  * Both give the same selection; outputs agree to fp32 rounding. */
 RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cache,
