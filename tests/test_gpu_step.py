@@ -145,7 +145,8 @@ def test_exact_ties_go_to_lower_block_ids(cuda_device, ctx, topk, max_topk, d):
 def test_mixed_modes_and_repeat_calls_are_identical(cuda_device):
     """One launch with top-k 0, top-k = M and ordinary top-k, called three
     times on the same state: the append is idempotent, the histogram and the
-    unit barriers must be left clean, and the results repeat bit for bit."""
+    unit counters must be left clean (and the generation advanced), and the
+    results repeat bit for bit."""
     p = inputs.make_decode_problem(12, 4, 28, 4, 128, 16, [4000, 700, 16, 12000], paged=True,
                                    topk=[0, 10**5, 3, 300])
     cfg, lc, ws = setup_layer(p, cuda_device)
