@@ -209,8 +209,9 @@ class GpuWorkload:
         self.qc = torch.randn(cycles, nl, B, f, hq, d, generator=g, device=device).to(torch.bfloat16)
         self.kc = torch.randn(cycles, nl, B, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
         self.vc = torch.randn(cycles, nl, B, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
-        # outputs
-        self.out = torch.empty(nl, B, hq, d, device=device)
+        # outputs: one slot per (decode step of the cycle, layer), so that every
+        # step's result survives the cycle and can be read back
+        self.out = torch.empty(f - 1, nl, B, hq, d, device=device)
         self.rout = torch.empty(nl, B, f, hq, d, device=device)
         # separate allocations keep every layer's selection buffers 16-byte aligned
         self.idx = [torch.empty(B, hkv, self.max_topk + 1, dtype=torch.int32, device=device)
@@ -234,7 +235,7 @@ class GpuWorkload:
             for layer in range(self.layers):
                 R.resa_decode_step(self.cfg, self.cache(layer, row), self.q[c, s, layer],
                                    self.kn[c, s, layer], self.vn[c, s, layer], self.topk_ptr(row),
-                                   self.max_topk, self.out[layer], None, self.idx[layer],
+                                   self.max_topk, self.out[s, layer], None, self.idx[layer],
                                    self.cnt[layer], self.ws)
         row = c * f + f - 1
         for layer in range(self.layers):
@@ -416,12 +417,23 @@ class OracleSample:
 
 
 def cpu_baseline(wl, seed, layer_state, samples=2):
+    """The oracle on the host cores (all threads, then one thread) on a bounded
+    sample of the workload; the median sample is extrapolated to a cycle."""
     from oracle import oracle as O
     s = OracleSample(wl, seed, layer_state)
+    cores = O.num_threads()
     cyc = [s.run()[0] for _ in range(samples)]
     t = statistics.median(cyc)
-    return {"value": wl["f"] * wl["batch"] / t, "unit": "tokens/s", "cores": O.num_threads(),
-            "kind": "oracle", "sample": s.describe(), "s_per_cycle_extrapolated": t}
+    O.set_num_threads(1)
+    try:
+        t1 = s.run()[0]
+    finally:
+        O.set_num_threads(cores)
+    tok = wl["f"] * wl["batch"]
+    return {"value": tok / t, "unit": "tokens/s", "cores": cores, "samples": samples,
+            "kind": "oracle", "sample": s.describe(), "s_per_cycle_extrapolated": t,
+            "threads_1": {"value": tok / t1, "unit": "tokens/s", "cores": 1, "samples": 1,
+                          "s_per_cycle_extrapolated": t1}}
 
 
 # ---------------------------------------------------------------------------
@@ -534,7 +546,10 @@ def run_resa(args):
         torch.cuda.synchronize(device)
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / K}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / K,
+               "copies": "per cycle: q/k/v of every decode step and the rectification chunk "
+                         "in; every decode step's output (f-1 per layer) and the rectified "
+                         "rows out"}
 
     code = w.R.resa_check_device_status(w.ws, raise_on_error=False)
 
@@ -649,8 +664,8 @@ def kernel_breakdown(w, stream, device, reps):
     n = w.layers
     res = {}
     res["sparse_decode_us"] = timed(lambda: [R.resa_sparse_decode(
-        w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.idx[l], w.cnt[l], w.max_topk, w.out[l],
-        None, w.ws) for l in range(n)], n)
+        w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.idx[l], w.cnt[l], w.max_topk,
+        w.out[w.f - 2, l], None, w.ws) for l in range(n)], n)
     scratch_idx = [torch.empty_like(t) for t in w.idx]
     scratch_cnt = [torch.empty_like(t) for t in w.cnt]
     res["select_blocks_us"] = timed(lambda: [R.resa_select_blocks(
@@ -661,7 +676,7 @@ def kernel_breakdown(w, stream, device, reps):
         for l in range(n)], n)
     res["decode_step_us"] = timed(lambda: [R.resa_decode_step(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
-        w.topk_ptr(row), w.max_topk, w.out[l], None, w.idx[l], w.cnt[l], w.ws)
+        w.topk_ptr(row), w.max_topk, w.out[w.f - 2, l], None, w.idx[l], w.cnt[l], w.ws)
         for l in range(n)], n)
     # dense decode for comparison: the same step with top-k = every block (Eq. 1 path)
     Ls = w.sched.decode_L(c, w.f - 2)
@@ -671,7 +686,7 @@ def kernel_breakdown(w, stream, device, reps):
                  for _ in range(n)]
     res["dense_decode_step_us"] = timed(lambda: [R.resa_decode_step(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
-        topk_all, all_k, w.out[l], None, dense_idx[l], scratch_cnt[l], w.ws)
+        topk_all, all_k, w.out[w.f - 2, l], None, dense_idx[l], scratch_cnt[l], w.ws)
         for l in range(n)], n)
     del dense_idx
     res["rectify_us"] = timed(lambda: [R.resa_rectify_attention(
@@ -704,8 +719,8 @@ def run_sweep(args):
     for st in range(row):
         for layer in range(n):
             R.resa_decode_step(w.cfg, w.cache(layer, st), w.q[0, st, layer], w.kn[0, st, layer],
-                               w.vn[0, st, layer], w.topk_ptr(st), w.max_topk, w.out[layer], None,
-                               w.idx[layer], w.cnt[layer], w.ws)
+                               w.vn[0, st, layer], w.topk_ptr(st), w.max_topk, w.out[st, layer],
+                               None, w.idx[layer], w.cnt[layer], w.ws)
     torch.cuda.synchronize(device)
     Ls = w.sched.decode_L(0, w.f - 2)
     M = [(L - 1) // 16 for L in Ls]
@@ -738,7 +753,7 @@ def run_sweep(args):
         cnt = [torch.empty(B, w.hkv, dtype=torch.int32, device=device) for _ in range(n)]
         us = timed(lambda: [R.resa_decode_step(
             w.cfg, w.cache(l, row), w.q[0, row, l], w.kn[0, row, l], w.vn[0, row, l], tk, kmax,
-            w.out[l], None, idx[l], cnt[l], w.ws) for l in range(n)], n)
+            w.out[row, l], None, idx[l], cnt[l], w.ws) for l in range(n)], n)
         steps.append({"s": frac, "topk": k[0] if B == 1 else k, "us_per_layer": us,
                       "launches_per_step": R.resa_decode_step_launches(w.cfg, B, w.max_pages,
                                                                        w.num_pages)})

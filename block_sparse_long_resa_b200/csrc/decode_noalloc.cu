@@ -19,7 +19,7 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB per device
 constexpr int kScratchMaxUnits = 4096;             // batch * Hkv
-constexpr size_t kScratchHeader = 256;  // error word; grid barrier at kDecBarrierOffset
+constexpr size_t kScratchHeader = 256;  // grid barrier at kDecBarrierOffset
 
 // Shared by every call on a device; it keeps the previous call's contents.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
@@ -56,8 +56,8 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
                                                     const int32_t *block_idx,
                                                     const int32_t *block_cnt, int32_t max_topk,
                                                     float *out, float *lse_opt,
-                                                    uint32_t *dev_error_opt, cudaStream_t stream) {
-    if (!cfg || !cache || !q || !block_idx || !block_cnt || !out) return RESA_ERR_NULL;
+                                                    uint32_t *dev_error, cudaStream_t stream) {
+    if (!cfg || !cache || !q || !block_idx || !block_cnt || !out || !dev_error) return RESA_ERR_NULL;
     if (!cache->k || !cache->v || !cache->page_table || !cache->seq_len) return RESA_ERR_NULL;
     if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 ||
         cfg->num_q_heads % cfg->num_kv_heads != 0)
@@ -71,8 +71,12 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     if ((long long)cache->max_pages * kBlock > 0x7fffffffLL ||
         (long long)cache->num_pages * hkv * kBlock > 0x7fffffffLL || max_topk < 0)
         return RESA_ERR_RANGE;
+    // The split merge holds the weights of at most kMaxDecodeSplits splits:
+    // the same bound resa_sparse_decode enforces (max_topk + 1 <= 1024 * 512).
+    if ((long long)max_topk + 1 > (long long)kMaxDecodeSplits * kMaxBlocksPerSplit)
+        return RESA_ERR_RANGE;
     if (!al16(cache->k) || !al16(cache->v) || !al16(cache->page_table) || !al16(cache->seq_len) ||
-        !al16(q) || !al16(out))
+        !al16(q) || !al16(out) || (reinterpret_cast<uintptr_t>(dev_error) & 3u) != 0)
         return RESA_ERR_UNSUPPORTED;
 
     // Size the scratch use and refuse what does not fit.
@@ -80,6 +84,7 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     if (units > kScratchMaxUnits) return RESA_ERR_SHAPE;
     const int d = cfg->head_dim;
     const int splits = decode_splits_for(units, max_topk + 1);
+    if (splits > kMaxDecodeSplits) return RESA_ERR_RANGE;
     const size_t tickets_bytes = align_up((size_t)units * 4, 256);
     // Per-warp partials for a grid-wide merge when they fit the array, else
     // per-split partials and the last-CTA merge.
@@ -97,12 +102,12 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     const resa_status_t st = scratch_address(&base);
     if (st != RESA_OK) return st;
     uint8_t *scratch = static_cast<uint8_t *>(base);
-    uint32_t *err = reinterpret_cast<uint32_t *>(scratch);
     uint32_t *tickets = reinterpret_cast<uint32_t *>(scratch + kScratchHeader);
     float *part_lse = reinterpret_cast<float *>(scratch + kScratchHeader + tickets_bytes);
     float *part_o = reinterpret_cast<float *>(scratch + kScratchHeader + tickets_bytes + lse_bytes);
-    // The array keeps the previous call's contents: the error word and the
-    // split tickets must start at zero.
+    // The array keeps the previous call's contents: the grid barrier word and
+    // the split tickets must start at zero.  Device errors go to the caller's
+    // word, never to the array, so the next call cannot wipe them unread.
     if (cudaMemsetAsync(scratch, 0, kScratchHeader + tickets_bytes, stream) != cudaSuccess)
         return RESA_ERR_CUDA;
 
@@ -120,7 +125,6 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
         s, cache->k, cache->v, cache->page_table, cache->seq_len, q, block_idx, block_cnt, max_topk,
         splits, part_o, part_lse, tickets,
         spread_fits ? reinterpret_cast<uint32_t *>(scratch + kDecBarrierOffset) : nullptr, out,
-        lse_opt,
-        dev_error_opt ? dev_error_opt : err, stream);
+        lse_opt, dev_error, stream);
     return e == cudaSuccess ? RESA_OK : RESA_ERR_CUDA;
 }

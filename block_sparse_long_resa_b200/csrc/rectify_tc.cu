@@ -17,13 +17,20 @@
 //   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into a
 //               double-buffered TMEM tile (kind::f16, bf16 inputs), then
 //               O += P V (kind::f16, fp16 inputs), commits on mbarriers;
-//   warps 2-3   convert the V tile bf16 -> fp16 in place (exact for
-//               |v| < 65504), zero blocks that were not loaded;
+//   warps 2-3   convert the V tile bf16 -> fp16 in place, scaled by a
+//               power of two 2^-e chosen per tile from its largest |v| so
+//               that every finite bf16 value lands in fp16's normal range
+//               (e = 0, no scaling, when the largest |v| is in [2^-8, 2^16));
+//               zero blocks that were not loaded;
 //   warps 4-11  softmax, one thread per query row (TMEM lane): tcgen05.ld of
 //               the S row, causal mask (skipped for interior tiles), base-2
 //               online softmax with lazy O rescaling (only when the row
 //               maximum grows by more than 8), P written to shared memory as
-//               fp16 in the canonical K-major swizzled layout.
+//               fp16 in the canonical K-major swizzled layout.  With E the
+//               largest tile exponent seen so far, a tile's P is multiplied
+//               by 2^(e - E) and O is rescaled whenever E grows, so the TMEM
+//               accumulator holds 2^-E times the true sum; the epilogue
+//               multiplies by 2^E.
 // Three K/V stages are in flight (released per stage by the P.V commit); the
 // P tile is single-buffered, written once the previous P.V has completed.
 // P is fp16 (11-bit mantissa), so the P.V product keeps the weights' precision
@@ -46,6 +53,24 @@ constexpr int kThreads = 32 * (kWarpSm0 + kNumSm);
 constexpr int kSmThreads = 32 * kNumSm;
 constexpr int kConvThreads = 32 * kNumConv;
 constexpr float kRescaleSlack = 8.0f;   // log2 units of growth tolerated before rescaling O
+constexpr int kNoExp = -1000;           // no V tile exponent seen yet
+
+// Power-of-two exponent e of a V tile whose largest magnitude has the bf16
+// bit pattern `mag` (sign cleared): the tile is stored as V * 2^-e in fp16.
+// 0 when the largest |v| lies in [2^-8, 2^16) (bf16 values there are exact
+// fp16 values, and smaller ones of the tile lose at most 2^-17 of the largest);
+// otherwise the largest |v| * 2^-e falls in [2^14, 2^15).  Zero tiles and
+// non-finite values keep e = 0.
+__device__ __forceinline__ int v_tile_exponent(uint32_t mag) {
+    if (mag == 0u || mag >= 0x7f80u) return 0;
+    const int ex = (int)(mag >> 7) - 127;  // floor(log2|v|) for normal bf16
+    if (ex >= -8 && ex <= 15) return 0;
+    return min(113, max(-100, ex - 14));
+}
+// 2^k as a float for k in [-126, 127]; 0 below.
+__device__ __forceinline__ float exp2i(int k) {
+    return k < -126 ? 0.f : __int_as_float((127 + k) << 23);
+}
 
 template <int D>
 struct TcLayout {
@@ -77,6 +102,10 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
     const __half2 h = __floats2half2_rn(bf_lo(x), bf_hi(x));
     return *reinterpret_cast<const uint32_t *>(&h);
 }
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t x, float scale) {
+    const __half2 h = __floats2half2_rn(bf_lo(x) * scale, bf_hi(x) * scale);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -98,9 +127,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     __shared__ uint64_t q_ready, kv_full[kStages], v_ready[kStages], kv_empty[kStages], s_full[2],
-        p_full, pv_done;
+        p_full, pv_done, conv_seen[kStages];
     __shared__ uint32_t tmem_base_s;
     __shared__ uint32_t stage_vmask[kStages];
+    __shared__ int stage_vexp[kStages];            // V tile exponent of each stage
+    __shared__ uint32_t conv_max[kStages][kNumConv];  // converter warps' largest |v| bits
 
     const int group = blockIdx.x, split = blockIdx.y, unit = blockIdx.z;
     const int G = gridDim.x, S = gridDim.y;
@@ -133,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&kv_full[s], 1);
             mbar_init(&v_ready[s], kConvThreads);
             mbar_init(&kv_empty[s], 1);
+            mbar_init(&conv_seen[s], kNumConv);
         }
         for (int s = 0; s < 2; ++s) mbar_init(&s_full[s], 1);
         mbar_init(&p_full, kSmThreads);
@@ -271,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < kWarpSm0) {  // ---------------------------------- V converters
         const int ct = threadIdx.x - 64;
+        const int cw = warp - 2;
         bool ok = true;
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % kStages;
@@ -280,19 +313,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4 *vt = reinterpret_cast<uint4 *>(kv_s + (size_t)s * 2 * LY::kKV + LY::kKV);
             constexpr int kChunks = LY::kKV / 16;           // 16-byte chunks of the tile
             constexpr int kChunksPerBlock = kBlock * 128 / 16;  // per half
-            for (int c = ct; c < kChunks; c += kConvThreads) {
+            constexpr int kPer = kChunks / kConvThreads;
+            static_assert(kChunks % kConvThreads == 0, "equal converter shares");
+            // the thread's chunks into registers (blocks not loaded become
+            // zero) and the largest magnitude among them, two halves a word
+            uint4 x[kPer];
+            uint32_t m2 = 0u;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int c = ct + k * kConvThreads;
                 const int blk_in_tile = (c % (LY::kKVHalf / 16)) / kChunksPerBlock;
-                uint4 x = vt[c];
-                if ((vmask >> blk_in_tile) & 1u) {
-                    x.x = bf16x2_to_f16x2(x.x);
-                    x.y = bf16x2_to_f16x2(x.y);
-                    x.z = bf16x2_to_f16x2(x.z);
-                    x.w = bf16x2_to_f16x2(x.w);
-                } else {
-                    x = make_uint4(0u, 0u, 0u, 0u);
-                }
-                vt[c] = x;
+                x[k] = ((vmask >> blk_in_tile) & 1u) ? vt[c] : make_uint4(0u, 0u, 0u, 0u);
+                m2 = __vmaxu2(m2, x[k].x & 0x7fff7fffu);
+                m2 = __vmaxu2(m2, x[k].y & 0x7fff7fffu);
+                m2 = __vmaxu2(m2, x[k].z & 0x7fff7fffu);
+                m2 = __vmaxu2(m2, x[k].w & 0x7fff7fffu);
             }
+            uint32_t mag = max(m2 & 0xffffu, m2 >> 16);
+            mag = __reduce_max_sync(0xffffffffu, mag);
+            if ((threadIdx.x & 31) == 0) {
+                conv_max[s][cw] = mag;
+                mbar_arrive(&conv_seen[s]);
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&conv_seen[s], (i / kStages) & 1));
+            if (!ok) break;
+            mag = max(conv_max[s][0], conv_max[s][1]);
+            const int e = v_tile_exponent(mag);
+            if (e == 0) {
+#pragma unroll
+                for (int k = 0; k < kPer; ++k) {
+                    uint4 y = x[k];
+                    y.x = bf16x2_to_f16x2(y.x);
+                    y.y = bf16x2_to_f16x2(y.y);
+                    y.z = bf16x2_to_f16x2(y.z);
+                    y.w = bf16x2_to_f16x2(y.w);
+                    vt[ct + k * kConvThreads] = y;
+                }
+            } else {
+                const float sc = exp2i(-e);
+#pragma unroll
+                for (int k = 0; k < kPer; ++k) {
+                    uint4 y = x[k];
+                    y.x = bf16x2_to_f16x2_scaled(y.x, sc);
+                    y.y = bf16x2_to_f16x2_scaled(y.y, sc);
+                    y.z = bf16x2_to_f16x2_scaled(y.z, sc);
+                    y.w = bf16x2_to_f16x2_scaled(y.w, sc);
+                    vt[ct + k * kConvThreads] = y;
+                }
+            }
+            if (ct == 0) stage_vexp[s] = e;
             fence_proxy_async_smem();
             mbar_arrive(&v_ready[s]);
         }
@@ -322,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&q_ready);
         }
         float m_use = -INFINITY, l = 0.f;
+        int e_run = kNoExp;  // largest V tile exponent so far (E)
         bool ok = true;
         // Keys every valid row of this CTA may see: tiles entirely below this
         // limit (and fully loaded) need no mask.
@@ -329,10 +399,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tend = blk1 * kBlock;
         for (int i = 0; i < ntiles; ++i) {
             const int buf = i & 1;
-            ok = mbar_wait_bounded(&s_full[buf], (i / 2) & 1);
+            ok = mbar_wait_bounded(&s_full[buf], (i / 2) & 1) &&
+                 mbar_wait_bounded(&v_ready[i % kStages], (i / kStages) & 1);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc::fence_after_sync();
+            // the tile's V exponent (the same for every thread of the CTA)
+            const int e_t = stage_vexp[i % kStages];
+            const bool e_grow = e_run != kNoExp && e_t > e_run;
+            const float alpha_e = e_grow ? exp2i(e_run - e_t) : 1.f;
+            e_run = e_run == kNoExp ? e_t : max(e_run, e_t);
+            const float pfac = exp2i(e_t - e_run);  // 1 unless this tile is smaller
             uint32_t sv[2][32];
             const uint32_t scol = tmem + lane_base + 2 * D + (2 * buf + mt) * kKeys;
             tc::tmem_ld32(scol, sv[0]);
@@ -374,6 +451,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m_use == -INFINITY) {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pw[e] = 0u;
+            } else if (pfac != 1.f) {
+                const float nm = -m_use;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = ex2(fmaf(x[2 * e], scale_log2, nm));
+                    const float p1 = ex2(fmaf(x[2 * e + 1], scale_log2, nm));
+                    psum += p0 + p1;
+                    pw[e] = f16x2(p0 * pfac, p1 * pfac);
+                }
             } else {
                 const float nm = -m_use;
 #pragma unroll
@@ -391,7 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc::fence_after_sync();
-                if (rescale) {
+                if (rescale || e_grow) {
+                    const float alpha_o = (rescale ? alpha : 1.f) * alpha_e;
 #pragma unroll
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         uint32_t ov[32];
@@ -400,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+                            ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha_o);
                         tc::tmem_st32(ocol, ov);
                     }
                     tc::tmem_wait_st();
@@ -428,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (l > 0.f) {
             lse2 = m_use + log2f(l);
-            inv = 1.f / l;
+            // O holds 2^-E times the weighted sum: undo the V scaling here
+            inv = (1.f / l) * exp2i(e_run == kNoExp ? 0 : e_run);
         }
         const float kLn2 = 0.6931471805599453f;
         const int r_pos = rho / g, jh = rho % g;

@@ -203,6 +203,44 @@ def make_rectify_chunk(seed: int, batch: int, f: int, num_q_heads: int, num_kv_h
     return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
 
 
+WIDE_KINDS = ("large", "huge", "tiny", "tiles")
+
+
+def wide_range_values(seed: int, v: torch.Tensor, kind: str, tokens_axis: int = -2) -> torch.Tensor:
+    """bf16 values of ``v``'s shape spanning bf16's range, for the value-range
+    parity cases (seeded; the input's own values are only used for their signs
+    and shapes):
+
+    - ``large``: N(0, 1), with about 1 token in 16 scaled by 1e5;
+    - ``huge``: as ``large``, plus about 1 token in 64 set to +-(1.0 .. 3.3)e38
+      (near the largest finite bf16, 3.39e38);
+    - ``tiny``: N(0, 1) * 1e-6 everywhere;
+    - ``tiles``: runs of 64 consecutive tokens drawn as N(0,1) * 1e-6,
+      N(0,1) * 1e5 or N(0,1), so that whole tiles differ in magnitude.
+    ``tokens_axis`` is the axis along which tokens are counted.
+    """
+    assert kind in WIDE_KINDS, kind
+    g = _gen(seed * 2_654_435 + 97, "cpu")
+    x = torch.randn(v.shape, generator=g)
+    ax = tokens_axis % x.dim()
+    ntok = x.shape[ax]
+    view = [1] * x.dim()
+    view[ax] = ntok
+    if kind == "tiny":
+        return (x * 1e-6).to(torch.bfloat16).to(v.device)
+    if kind == "tiles":
+        run = torch.randint(0, 3, ((ntok + 63) // 64,), generator=g)
+        scale = torch.tensor([1e-6, 1e5, 1.0])[run].repeat_interleave(64)[:ntok]
+        return (x * scale.view(view)).to(torch.bfloat16).to(v.device)
+    big = (torch.rand(ntok, generator=g) < 1 / 16).to(torch.float32)
+    x = x * (1.0 + (1e5 - 1.0) * big).view(view)
+    if kind == "huge":
+        hot = (torch.rand(x.shape, generator=g) < 1 / 64)
+        mag = 1.0e38 + 2.3e38 * torch.rand(x.shape, generator=g)
+        x = torch.where(hot, torch.sign(x) * mag, x)
+    return x.to(torch.bfloat16).to(v.device)
+
+
 def continuous_batch_lengths(seed: int, batch: int, lo: int, hi: int) -> List[int]:
     """Context lengths uniform in [lo, hi] for the continuous-batching workload."""
     g = _gen(seed + 4242, "cpu")

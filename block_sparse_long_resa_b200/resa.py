@@ -190,9 +190,11 @@ def resa_decode_step(cfg, cache, q, k_new, v_new, topk, max_topk: int, out, lse,
 
 
 def resa_sparse_decode_noalloc(cfg, cache, q, block_idx, block_cnt, max_topk: int, out, lse,
-                               dev_error=None, stream=None):
+                               dev_error, stream=None):
     """resa_sparse_decode without a workspace, for callers that cannot allocate
-    device memory (scratch lives in a fixed device array inside the library)."""
+    device memory (scratch lives in a fixed device array inside the library).
+    dev_error: a device uint32 word (e.g. an int32 tensor element) that
+    receives the device error bits; required."""
     _check(lib().resa_sparse_decode_noalloc(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q),
                                             _ptr(block_idx), _ptr(block_cnt), max_topk, _ptr(out),
                                             _ptr(lse), _ptr(dev_error), _stream(stream)),

@@ -15,6 +15,13 @@
  *   (never synchronised), except resa_check_device_status.
  * Precision.  q, K, V and descriptors are bf16; scores, softmax statistics
  *   and accumulation are fp32; attention outputs are fp32.
+ * Value range.  resa_rectify_attention accepts every finite bf16 value: it
+ *   stages each 64-key V tile in fp16 scaled by a power of two chosen from
+ *   the tile's largest |v|, and undoes the scaling in fp32.  The decode entry
+ *   points keep V in bf16 and sum up to ~2^17 weighted values per warp in
+ *   fp32 before normalising, so they need |v| <= 1e33 (far beyond any model's
+ *   activations; larger values may overflow to inf).  Non-finite inputs give
+ *   non-finite outputs.
  * Cache layout (one attention layer):
  *   k, v        [num_pages][Hkv][block_size][head_dim]  bf16
  *   desc        [num_pages][Hkv][2][head_dim]           bf16, row 0 = element-wise
@@ -205,7 +212,9 @@ RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cac
  *     allocated or freed.
  *   - Limit: batch * Hkv <= 4096 and batch * Hkv * splits * 16 * (d + 2) * 4
  *     bytes of partials must fit the array (about 16 MiB); larger calls
- *     return RESA_ERR_SHAPE.  Splits are chosen as in resa_sparse_decode.
+ *     return RESA_ERR_SHAPE.  Splits are chosen as in resa_sparse_decode, and
+ *     as there max_topk + 1 above 1024 * 512 blocks returns RESA_ERR_RANGE
+ *     before anything is launched.
  *   - The first call on each device looks up the array's device address
  *     (a runtime query, done once per device with that device current); make
  *     that first call before any stream capture.
@@ -213,15 +222,17 @@ RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cac
  *     call's contents; the call clears the parts that must start at zero.
  *     Calls that overlap on the GPU (different streams, or host threads
  *     without ordering) race on the array: serialise them.
- *   - dev_error_opt (nullable, device uint32, zeroed by the caller) receives
- *     the device error bits that resa_check_device_status reports for the
- *     workspace path. */
+ *   - dev_error (required, device uint32, 4-byte aligned, zeroed by the
+ *     caller before first use) receives, OR-ed in, the device error bits
+ *     that resa_check_device_status reports for the workspace path; the call
+ *     never clears it.  NULL returns RESA_ERR_NULL: the scratch array is
+ *     reset by every call, so it cannot hold errors until someone reads them. */
 RESA_API resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
                                                   const resa_cache_t *cache, const void *q,
                                                   const int32_t *block_idx,
                                                   const int32_t *block_cnt, int32_t max_topk,
                                                   float *out, float *lse_opt,
-                                                  uint32_t *dev_error_opt, cudaStream_t stream);
+                                                  uint32_t *dev_error, cudaStream_t stream);
 
 /* Number of kernels each entry point launches per call (for launch
  * accounting): 1 for append and build, 2 for select, 1 for sparse decode,

@@ -63,11 +63,18 @@ def lib():
                 fn.argtypes = args
                 fn.restype = None
             _lib.oracle_num_threads.restype = ctypes.c_int
+            _lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+            _lib.oracle_set_num_threads.restype = None
         return _lib
 
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops (results do not depend on it)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def _ptr(a: Optional[np.ndarray]):

@@ -346,3 +346,15 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* Thread count of the parallel loops above (timing harness control only; the
+ * results do not depend on it: every output element is computed by one thread
+ * in the same order). */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

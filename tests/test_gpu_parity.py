@@ -476,3 +476,92 @@ def test_full_size_continuous_batching(cuda_device):
                             cpu(p.topk), cpu(L), 16)
     ref = r["out"] if same else o.sparse_attention(cpu(p.q), gidx, gcnt, cpu(L))[0]
     np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+
+
+# --------------------------------------------------------------------------- value range
+#
+# Tolerance for values far from N(0, 1): the attention output is a convex
+# combination of the values, and its rounding error scales with their size,
+# so the 2e-3 bar (stated for N(0, 1) values) is applied relative to the
+# largest |v| a head's rows attend to: |out - ref| <= 2e-3 * max|v|.
+
+def _wide_values(p, kind, seed):
+    """Replace the cache's values with wide-range ones, drawn along sequence
+    positions of the contiguous layout; slots beyond the context stay zero."""
+    v = p.v_cache
+    P, H, T, D = v.shape
+    tok = v.permute(1, 0, 2, 3).reshape(H, P * T, D)
+    w = inputs.wide_range_values(seed, tok, kind, tokens_axis=1)
+    w = w.reshape(H, P, T, D).permute(1, 0, 2, 3).contiguous()
+    p.v_cache = torch.where(v != 0, w, torch.zeros_like(w))
+
+
+def _row_tol(o, B, hkv, g, L_per_b):
+    """[B][Hq] tolerance: 2e-3 * max|v| over the positions of the row's kv head."""
+    tol = np.zeros((B, hkv * g))
+    for b in range(B):
+        for h in range(hkv):
+            vmax = float(np.abs(o.values(b, h, int(L_per_b[b]))).max())
+            tol[b, h * g:(h + 1) * g] = OUT_ATOL * vmax
+    return tol
+
+
+@pytest.mark.parametrize("kind", inputs.WIDE_KINDS)
+def test_rectify_value_range(cuda_device, kind):
+    """Values from 1e-6 to +-3.3e38, mixed within and across 64-key tiles:
+    the fp16 staging of V is scaled per tile, so no finite bf16 value overflows
+    and tiny ones keep their precision."""
+    hq, hkv, d, f = 28, 4, 128, 32
+    ctx = [1000, 4096]
+    B = len(ctx)
+    p = inputs.make_decode_problem(60, B, hq, hkv, d, 16, ctx, needles=0, topk=[1] * B)
+    _wide_values(p, kind, 61)
+    cfg, lc, ws = setup_layer(p, cuda_device, max_chunk=f)
+    L = p.ctx_len.clone()
+    qc, kc, vc = inputs.make_rectify_chunk(62, B, f, hq, hkv, d)
+    vc = inputs.wide_range_values(63, vc, kind, tokens_axis=1)
+    out = torch.empty(B, f, hq, d, device=cuda_device)
+    lse = torch.empty(B, f, hq, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_rectify_attention(cfg, lc.struct(), f, dev(qc), dev(kc), dev(vc), out, lse, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(L)
+    ref, ref_lse = o.rectify(qc, kc, vc, L, f)
+    np.testing.assert_array_equal(bits_of(lc.v), o.V)
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    tol = _row_tol(o, B, hkv, hq // hkv, L)
+    err = np.abs(got - ref).max(axis=-1)             # [B][f][Hq]
+    assert (err <= tol[:, None, :]).all(), float((err / tol[:, None, :]).max())
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+
+
+@pytest.mark.parametrize("kind", ["large", "tiny", "tiles"])
+def test_decode_step_value_range(cuda_device, kind):
+    """The decode step's bf16 V and hi + lo P keep their precision from 1e-6 to
+    1e5 (the decode paths' range is stated in include/resa.h)."""
+    p = make(QWEN32K)
+    _wide_values(p, kind, 71)
+    if kind == "tiny":
+        p.v_new = (p.v_new.float() * 1e-6).to(torch.bfloat16)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L.to(cuda_device))
+    max_topk = int(p.topk.max())
+    B, Hq, Hkv, d = p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=cuda_device)
+    idx = torch.full((B, Hkv, max_topk + 1), -1, dtype=torch.int32, device=cuda_device)
+    cnt = torch.zeros(B, Hkv, dtype=torch.int32, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_decode_step(cfg, lc.struct(), dev(p.q), dev(p.k_new), dev(p.v_new), dev(p.topk),
+                       max_topk, out, None, idx, cnt, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    o.append(p.k_new, p.v_new, L)
+    gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    ref, _ = o.sparse_attention(p.q, gidx, gcnt, L)
+    tol = _row_tol(o, B, Hkv, Hq // Hkv, L)
+    err = np.abs(out.cpu().numpy() - ref).max(axis=-1)
+    assert (err <= tol).all(), float((err / tol).max())
