@@ -44,6 +44,11 @@ WORKLOADS = {
     "layer256k": dict(layers=1, batch=1, hq=28, hkv=4, d=128, ctx=[262144], f=32, paged=False,
                       text="one layer of the long-context decode workload (28 q / 4 kv, d 128), "
                            "262144-token cache, top-k 10% + current block, ReSA cycle f=32"),
+    "qwen32k": dict(layers=4, batch=1, hq=28, hkv=4, d=128, ctx=[32768], f=32, paged=False,
+                    text="one attention layer of Qwen2.5-7B shape (28 q / 4 kv, d 128), batch 1, "
+                         "32768-token cache, top-k 10% (205) + current block; timed over 4 "
+                         "independent layer caches in turn (268 MB) so that L2 cannot hold "
+                         "the cache, reported per layer"),
     "loop64k": dict(layers=1, batch=4, hq=28, hkv=4, d=128, ctx=[65536] * 4, f=32, paged=False,
                     text="ReSA decode loop: 1 layer (28 q / 4 kv, d 128), batch 4, 65536-token "
                          "cache, top-k 10%, 31 sparse decode steps + 1 rectification of 32"),
@@ -65,6 +70,8 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=1234)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the dense baseline and the further workloads")
     ap.add_argument("--breakdown-reps", type=int, default=5)
     ap.add_argument("--sweep", action="store_true",
                     help="time the decode step over top-k fractions and the rectification over "
@@ -592,6 +599,14 @@ def run_resa(args):
     rect["frac_of_bf16_peak"] = rect["tflops"] / bf16_peak
     rect["frac_of_hbm_peak"] = rect["hbm_gbs"] / hbm_peak
 
+    dense = extra = None
+    if not args.no_extra:
+        dense = dense_baseline(stream, device, args.seed + 500, args.breakdown_reps, hbm_peak)
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            if name != args.workload:
+                extra[name] = workload_block(name, stream, device, args.seed + 700, 3, hbm_peak)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         L_state = w.sched.decode_L(cycles - 1, wl["f"] - 2)
@@ -616,7 +631,9 @@ def run_resa(args):
         "rectify": rect,
         "kernel_breakdown_us": bd,
         "decode_step_path": "fused (1 launch)" if fused else "3 launches",
-        "sparse_vs_dense_step_speedup": bd["dense_decode_step_us"] / bd["decode_step_us"],
+        "sparse_vs_dense_step_speedup": bd["dense_decode_us"] / bd["decode_step_us"],
+        "dense_baseline": dense,
+        "workloads": extra,
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": K * w.launches_per_cycle(),
@@ -678,20 +695,141 @@ def kernel_breakdown(w, stream, device, reps):
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
         w.topk_ptr(row), w.max_topk, w.out[w.f - 2, l], None, w.idx[l], w.cnt[l], w.ws)
         for l in range(n)], n)
-    # dense decode for comparison: the same step with top-k = every block (Eq. 1 path)
-    Ls = w.sched.decode_L(c, w.f - 2)
-    all_k = max((L - 1) // 16 for L in Ls)
-    topk_all = torch.full((w.sched.Bpad,), all_k, dtype=torch.int32, device=device)
-    dense_idx = [torch.empty(w.B, w.hkv, all_k + 1, dtype=torch.int32, device=device)
-                 for _ in range(n)]
-    res["dense_decode_step_us"] = timed(lambda: [R.resa_decode_step(
+    # dense decoding of the same step (append + attention over every position, Eq. 1)
+    res["dense_decode_us"] = timed(lambda: [R.resa_dense_decode(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
-        topk_all, all_k, w.out[w.f - 2, l], None, dense_idx[l], scratch_cnt[l], w.ws)
-        for l in range(n)], n)
-    del dense_idx
+        w.out[w.f - 2, l], None, w.ws) for l in range(n)], n)
     res["rectify_us"] = timed(lambda: [R.resa_rectify_attention(
         w.cfg, w.cache(l, rrow), w.f, w.qc[c, l], w.kc[c, l], w.vc[c, l], w.rout[l], None, w.ws)
         for l in range(n)], n)
+    return res
+
+
+DENSE_CONTEXTS = (16384, 65536, 262144)
+
+
+def dense_baseline(stream, device, seed, reps, hbm_peak):
+    """One decode step of one layer (28 q / 4 kv heads, d 128, batch 1), sparse
+    (top-k 10 % + current block, Eq. 2) against dense decoding over every
+    position (Eq. 1), at the context lengths of the pages' speed-up figures
+    (ReSA summary §5).  Each length rotates over enough independent caches
+    (at least 4x the L2 size) that every call reads its K/V from HBM."""
+    import torch
+    from block_sparse_long_resa_b200 import inputs
+    from block_sparse_long_resa_b200 import resa as R
+    from block_sparse_long_resa_b200.cache import LayerCache, workspace
+    hq, hkv, d = 28, 4, 128
+    cfg = R.make_config(hq, hkv, d, 16)
+    rows = []
+    for L0 in DENSE_CONTEXTS:
+        L = L0 + 1
+        copies = max(2, -(-4 * 126 * 2**20 // (L0 * hkv * d * 4)))
+        caches = []
+        for i in range(copies):
+            p = inputs.make_decode_problem(seed + 31 * i + L0, 1, hq, hkv, d, 16, [L0],
+                                           reserve_tokens=16, device=device, topk=[1])
+            caches.append((LayerCache.from_problem(p, device), p.q.clone(), p.k_new.clone(),
+                           p.v_new.clone()))
+            del p
+        ws = workspace(cfg, 1, caches[0][0].max_pages, 16, device)
+        for lc, *_ in caches:
+            R.resa_build_descriptors(cfg, lc.struct(), None, ws)
+            lc.seq_len.fill_(L)
+        k = topk_rule(L)
+        tk = torch.tensor([k, 0, 0, 0], dtype=torch.int32, device=device)
+        out = torch.empty(1, hq, d, device=device)
+        idx = torch.empty(1, hkv, k + 1, dtype=torch.int32, device=device)
+        cnt = torch.empty(1, hkv, dtype=torch.int32, device=device)
+        calls = 28
+
+        def timed(one):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for j in range(calls):
+                        one(*caches[j % copies])
+                g.replay()
+                torch.cuda.synchronize(device)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize(device)
+            return 1e3 * e0.elapsed_time(e1) / (reps * calls)
+
+        us_s = timed(lambda lc, q, kn, vn: R.resa_decode_step(
+            cfg, lc.struct(), q, kn, vn, tk, k, out, None, idx, cnt, ws))
+        us_d = timed(lambda lc, q, kn, vn: R.resa_dense_decode(
+            cfg, lc.struct(), q, kn, vn, out, None, ws))
+        code = R.resa_check_device_status(ws, raise_on_error=False)
+        M = (L - 1) // 16
+        b_s = hq * d * 2 + M * hkv * 2 * d * 2 + (k + 1) * 16 * hkv * d * 4 + hq * d * 4
+        b_d = hq * d * 2 + L * hkv * d * 4 + hq * d * 4
+        rows.append({"context": L0, "topk": k, "sparse_step_us": us_s, "dense_step_us": us_d,
+                     "dense_over_sparse": us_d / us_s,
+                     "sparse_hbm_frac": b_s / (us_s * 1e-6) / 1e9 / hbm_peak,
+                     "dense_hbm_frac": b_d / (us_d * 1e-6) / 1e9 / hbm_peak,
+                     "cache_copies": copies, "device_error_word": code})
+        del caches, ws
+        torch.cuda.empty_cache()
+    return {"shape": "1 layer, 28 q / 4 kv heads, d 128, batch 1, block 16", "steps": rows,
+            "bytes": "sparse: q + descriptors + selected K/V + output; dense: q + all K/V "
+                     "+ output; fraction of the measured HBM copy bandwidth"}
+
+
+EXTRA_WORKLOADS = ("qwen32k", "cbatch", "loop64k")
+
+
+def workload_block(name, stream, device, seed, reps, hbm_peak):
+    """The cycle graph of a further workload, timed alone: µs per cycle, the
+    decode step's µs and roofline fraction, and the amortised µs per token."""
+    import torch
+    wl = WORKLOADS[name]
+    cycles = 2
+    w = GpuWorkload(wl, cycles, seed, device)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for c in range(cycles):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                w.launch_cycle(c)
+            graphs.append(g)
+        graphs[0].replay()
+        graphs[1].replay()
+        graphs[1].replay()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            graphs[1].replay()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    cyc_us = 1e3 * e0.elapsed_time(e1) / reps
+    bd = kernel_breakdown(w, stream, device, reps)
+    Ls = w.sched.decode_L(cycles - 1, wl["f"] - 2)
+    fused = w.R.resa_decode_step_launches(w.cfg, w.B, w.max_pages, w.num_pages) == 1
+    step_b = w.step_bytes(Ls)
+    gbs = step_b / (bd["decode_step_us"] * 1e-6) / 1e9
+    rb, rflops = w.rectify_bytes_flops(w.sched.rect_L(cycles - 1))
+    code = w.R.resa_check_device_status(w.ws, raise_on_error=False)
+    per_layer_cycle = cyc_us / wl["layers"]
+    res = {"description": wl["text"], "context": Ls if len(Ls) <= 4 else
+           {"min": min(Ls), "max": max(Ls), "sequences": len(Ls)},
+           "decode_step_us": bd["decode_step_us"], "decode_step_launches":
+           1 if fused else w.R.resa_decode_step_launches(w.cfg, w.B, w.max_pages, w.num_pages),
+           "decode_step_gbs": gbs, "decode_step_hbm_frac": gbs / hbm_peak,
+           "dense_decode_us": bd["dense_decode_us"],
+           "rectify_us": bd["rectify_us"],
+           "rectify_tflops": rflops / (bd["rectify_us"] * 1e-6) / 1e12,
+           "cycle_us_per_layer": per_layer_cycle,
+           "amortised_us_per_token_per_layer": per_layer_cycle / wl["f"],
+           "tokens_per_s": wl["batch"] * wl["f"] / (cyc_us * 1e-6),
+           "device_error_word": code}
+    del graphs, w
+    torch.cuda.empty_cache()
     return res
 
 
@@ -758,7 +896,9 @@ def run_sweep(args):
                       "launches_per_step": R.resa_decode_step_launches(w.cfg, B, w.max_pages,
                                                                        w.num_pages)})
         del idx, cnt
-    t_dense = steps[-1]["us_per_layer"]
+    t_dense = timed(lambda: [R.resa_dense_decode(
+        w.cfg, w.cache(l, row), w.q[0, row, l], w.kn[0, row, l], w.vn[0, row, l],
+        w.out[row, l], None, w.ws) for l in range(n)], n)
     fmax = max(SWEEP_CHUNKS)
     ws = torch.empty(R.resa_workspace_size(w.cfg, B, w.max_pages, fmax), dtype=torch.uint8,
                      device=device)
@@ -779,7 +919,7 @@ def run_sweep(args):
     code = R.resa_check_device_status(w.ws, raise_on_error=False) | \
         R.resa_check_device_status(ws, raise_on_error=False)
     table = []
-    for st in steps[:-1]:
+    for st in steps:
         for rc in rects:
             f = rc["f"]
             t_tok = ((f - 1) * st["us_per_layer"] + rc["us_per_layer"]) / f

@@ -162,7 +162,7 @@ __device__ __forceinline__ void merge_warp_partials(const float *__restrict__ pa
 
 template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_decode_kernel(const uint8_t *__restrict__ k_cache, const uint8_t *__restrict__ v_cache,
+    sparse_decode_kernel(const uint8_t *k_cache, const uint8_t *v_cache,
                          const int32_t *__restrict__ page_table,
                          const int32_t *__restrict__ seq_len, const uint16_t *__restrict__ q,
                          const int32_t *__restrict__ block_idx,
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          int max_pages, int num_pages, float scale_log2, float *__restrict__ part_o,
                          float *__restrict__ part_lse, uint32_t *__restrict__ tickets,
                          uint32_t *__restrict__ grid_bar, float *__restrict__ out,
-                         float *__restrict__ lse_out, uint32_t *err) {
+                         float *__restrict__ lse_out, uint32_t *err, const DecodeAppend app) {
     using SM = DecodeSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array itself so that
@@ -211,21 +211,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     pdl_wait();  // block lists / counts come from the preceding selection
-    int cnt = block_cnt[unit];
     const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
+    const int nblk_seq = seq_ok ? (L + kBlock - 1) / kBlock : 0;
+    // without a block list (dense decoding) every block of the sequence
+    int cnt = block_idx ? block_cnt[unit] : nblk_seq;
     if (!seq_ok) {
         if (threadIdx.x == 0 && split == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
         cnt = 0;
     }
-    cnt = max(0, min(cnt, max_topk + 1));
+    cnt = max(0, min(cnt, block_idx ? max_topk + 1 : max_pages));
     const int per = (cnt + S - 1) / S;
     const int j0 = min(cnt, split * per), j1 = min(cnt, j0 + per);
     const int nslice = min(j1 - j0, kMaxBlocksPerSplit);  // the host sizes S so this holds
-    const int32_t *list = block_idx + unit * (max_topk + 1);
-    const int nblk_seq = seq_ok ? (L + kBlock - 1) / kBlock : 0;
+    const int32_t *list = block_idx ? block_idx + unit * (max_topk + 1) : nullptr;
+
+    if (app.k_new != nullptr && cnt > 0 && j0 <= cnt - 1 && cnt - 1 < j1) {
+        // Dense decoding appends the decode token itself: this CTA decodes the
+        // current block (the last entry), and the barrier after the staging
+        // below orders the append before its copies of that block.
+        constexpr int CPR = D / 8;  // 16-byte chunks per K / V row
+        if (threadIdx.x < CPR) {
+            const int c = threadIdx.x, M = (L - 1) / kBlock, slot = (L - 1) % kBlock;
+            const int page = page_table[(size_t)b * max_pages + M];
+            if (page >= 0 && page < num_pages) {
+                const uint4 kx = app.k_new[unit * CPR + c], vx = app.v_new[unit * CPR + c];
+                const size_t o = (((size_t)page * hkv + h) * kBlock + slot) * CPR + c;
+                reinterpret_cast<uint4 *>(app.k)[o] = kx;
+                reinterpret_cast<uint4 *>(app.v)[o] = vx;
+                uint4 *dmn = reinterpret_cast<uint4 *>(app.desc) + (((size_t)page * hkv + h) * 2) * CPR + c;
+                if (slot == 0) {
+                    dmn[0] = kx;
+                    dmn[CPR] = kx;
+                } else {
+                    Bf16x8 mn = unpack8(dmn[0]), mx = unpack8(dmn[CPR]);
+                    fold8(mn, mx, unpack8(kx));
+                    dmn[0] = pack8(mn);
+                    dmn[CPR] = pack8(mx);
+                }
+            } else if (c == 0) {
+                set_error(err, RESA_DEVERR_PAGE);
+            }
+        }
+    }
 
     for (int i = threadIdx.x; i < nslice; i += kThreads) {
-        const int blk = list[j0 + i];
+        const int blk = list ? list[j0 + i] : j0 + i;
         int page = -1, ntok = 0;
         if (blk >= 0 && blk < nblk_seq) {
             page = page_table[(size_t)b * max_pages + blk];
@@ -527,7 +557,8 @@ cudaError_t launch_dn(const Shape &s, const void *k, const void *v,
                       const int32_t *page_table, const int32_t *seq_len, const void *q,
                       const int32_t *block_idx, const int32_t *block_cnt, int max_topk, int splits,
                       float *part_o, float *part_lse, uint32_t *tickets, uint32_t *grid_bar,
-                      float *out, float *lse, uint32_t *err, cudaStream_t st) {
+                      float *out, float *lse, uint32_t *err, const DecodeAppend &app,
+                      cudaStream_t st) {
     constexpr int smem = DecodeSmem<D>::kBytes;
     static std::atomic<int> done[64];
     cudaError_t e = ensure_smem(sparse_decode_kernel<D, NT>, smem, done);
@@ -556,7 +587,7 @@ cudaError_t launch_dn(const Shape &s, const void *k, const void *v,
                               (const uint8_t *)v, page_table, seq_len,
                               (const uint16_t *)q, block_idx, block_cnt, max_topk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets,
-                              spread ? grid_bar : (uint32_t *)nullptr, out, lse, err);
+                              spread ? grid_bar : (uint32_t *)nullptr, out, lse, err, app);
 }
 
 }  // namespace
@@ -566,10 +597,10 @@ cudaError_t launch_sparse_decode(const Shape &s, const void *k, const void *v,
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
                                  uint32_t *grid_bar, float *out, float *lse, uint32_t *err,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, const DecodeAppend &app) {
 #define RESA_DECODE_ARGS                                                                     \
     s, k, v, page_table, seq_len, q, block_idx, block_cnt, max_topk, splits, part_o,       \
-        part_lse, tickets, grid_bar, out, lse, err, st
+        part_lse, tickets, grid_bar, out, lse, err, app, st
     if (s.d == 128)
         return s.g <= 8 ? launch_dn<128, 1>(RESA_DECODE_ARGS) : launch_dn<128, 2>(RESA_DECODE_ARGS);
     if (s.d == 64)

@@ -357,6 +357,33 @@ resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cache_t *cac
     return decode_impl(s, cache, w, ws, q, idx, cnt, max_topk, out, lse_opt, stream);
 }
 
+resa_status_t resa_dense_decode(const resa_config_t *cfg, const resa_cache_t *cache,
+                                const void *q, const void *k_new, const void *v_new, float *out,
+                                float *lse_opt, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    Shape s{};
+    RESA_TRY(check_config(cfg, &s));
+    RESA_TRY(check_cache(cache, &s, true, true));
+    if (!q || !k_new || !v_new || !out) return RESA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out))
+        return RESA_ERR_UNSUPPORTED;
+    const WsLayout w = layout_of(s, 0);
+    RESA_TRY(check_ws(ws, ws_bytes, w));
+    // every block of the sequence: max_topk + 1 = max_pages entries
+    const int splits = decode_splits_for(s.batch * s.hkv, s.max_pages);
+    if (splits > w.dec_splits || splits > kMaxDecodeSplits) return RESA_ERR_RANGE;
+    DecodeAppend app;
+    app.k = cache->k;
+    app.v = cache->v;
+    app.desc = cache->desc;
+    app.k_new = static_cast<const uint4 *>(k_new);
+    app.v_new = static_cast<const uint4 *>(v_new);
+    return cuda_status(launch_sparse_decode(
+        s, cache->k, cache->v, cache->page_table, cache->seq_len, q, nullptr, nullptr,
+        s.max_pages - 1, splits, at<float>(ws, w.dec_o), at<float>(ws, w.dec_lse),
+        at<uint32_t>(ws, w.dec_ticket), at<uint32_t>(ws, w.err + kDecBarrierOffset), out, lse_opt,
+        at<uint32_t>(ws, w.err), stream, app));
+}
+
 int32_t resa_decode_step_launches(const resa_config_t *cfg, int32_t batch, int32_t max_pages,
                                   int32_t num_pages) {
     Shape s{};
@@ -376,7 +403,7 @@ int32_t resa_kernels_per_call(const char *entry_point) {
     } table[] = {{"resa_build_descriptors", 1}, {"resa_append_token", 1},
                  {"resa_select_blocks", 2},     {"resa_sparse_decode", 1},
                  {"resa_rectify_attention", 2}, {"resa_decode_step", 1},
-                 {"resa_sparse_decode_noalloc", 1}};
+                 {"resa_sparse_decode_noalloc", 1}, {"resa_dense_decode", 1}};
     for (auto &e : table)
         if (strcmp(e.name, entry_point) == 0) return e.n;
     return -1;

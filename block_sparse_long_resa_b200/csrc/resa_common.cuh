@@ -458,12 +458,20 @@ cudaError_t launch_select(const Shape &s, const float *scores, uint32_t *hist,
                           uint32_t *hist_range, const int32_t *seq_len, const int32_t *topk,
                           int max_topk, int32_t *block_idx, int32_t *block_cnt, uint32_t *err,
                           cudaStream_t st);
+// The decode-token append a dense decode does in the same launch (all null:
+// none).  k / v / desc are the caches, k_new / v_new [batch][Hkv][d] bf16.
+struct DecodeAppend {
+    void *k = nullptr, *v = nullptr, *desc = nullptr;
+    const uint4 *k_new = nullptr, *v_new = nullptr;
+};
+// block_idx == nullptr: dense decoding over every block of each sequence
+// (block_cnt unused, max_topk + 1 taken as max_pages).
 cudaError_t launch_sparse_decode(const Shape &s, const void *k, const void *v,
                                  const int32_t *page_table, const int32_t *seq_len, const void *q,
                                  const int32_t *block_idx, const int32_t *block_cnt, int max_topk,
                                  int splits, float *part_o, float *part_lse, uint32_t *tickets,
                                  uint32_t *grid_bar, float *out, float *lse, uint32_t *err,
-                                 cudaStream_t st);
+                                 cudaStream_t st, const DecodeAppend &app = DecodeAppend());
 // Fused decode step: append + scores + selection + sparse attention in one
 // cooperative launch of G CTAs per (sequence, kv head) (step_ctas_per_unit).
 struct StepBuffers {

@@ -62,6 +62,7 @@ _SIGS = {
     "resa_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
                          ctypes.c_int),
     "resa_sparse_decode_noalloc": ([_P, _P, _P, _P, _P, _I, _P, _P, _P, _P], ctypes.c_int),
+    "resa_dense_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "resa_kernels_per_call": ([ctypes.c_char_p], ctypes.c_int32),
     "resa_decode_step_launches": ([_P, _I, _I, _I], ctypes.c_int32),
     "resa_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -187,6 +188,14 @@ def resa_decode_step(cfg, cache, q, k_new, v_new, topk, max_topk: int, out, lse,
                                   _ptr(block_idx), _ptr(block_cnt), _ptr(ws), ws.numel(),
                                   _stream(stream)),
            "resa_decode_step")
+
+
+def resa_dense_decode(cfg, cache, q, k_new, v_new, out, lse, ws, stream=None):
+    """Dense decode: append the decode token and attend to every position."""
+    _check(lib().resa_dense_decode(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(k_new),
+                                   _ptr(v_new), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                   _stream(stream)),
+           "resa_dense_decode")
 
 
 def resa_sparse_decode_noalloc(cfg, cache, q, block_idx, block_cnt, max_topk: int, out, lse,

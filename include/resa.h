@@ -199,6 +199,20 @@ RESA_API resa_status_t resa_decode_step(const resa_config_t *cfg, const resa_cac
                                int32_t *block_idx_opt, int32_t *block_cnt_opt, void *ws,
                                size_t ws_bytes, cudaStream_t stream);
 
+/* Dense decode attention, the baseline the sparse step is measured against
+ * (ReSA summary §5 "Experimental Analysis", dense decoding; Eq. 1): append the
+ * decode token (as resa_append_token) and attend, for every query head, to
+ * every position 0 .. L-1 with logits sm_scale * q.k, split across SMs with a
+ * log-sum-exp combine.  No descriptor is scored and nothing is selected; the
+ * append still keeps the block key cache current for later sparse steps.
+ * q [batch][Hq][d] bf16, k_new / v_new [batch][Hkv][d] bf16; out
+ * [batch][Hq][d] fp32, lse_opt (nullable) [batch][Hq] fp32, natural log.
+ * seq_len must already count the decode token.  One launch. */
+RESA_API resa_status_t resa_dense_decode(const resa_config_t *cfg, const resa_cache_t *cache,
+                                         const void *q, const void *k_new, const void *v_new,
+                                         float *out, float *lse_opt, void *ws, size_t ws_bytes,
+                                         cudaStream_t stream);
+
 /* The group block-sparse decode of resa_sparse_decode for callers that
  * cannot allocate device memory.  The pages describe no such variant: it
  * exists for hosts that give this library only input and output pointers,
@@ -237,7 +251,8 @@ RESA_API resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
 /* Number of kernels each entry point launches per call (for launch
  * accounting): 1 for append and build, 2 for select, 1 for sparse decode,
  * 2 for rectify, 1 for a decode step of the fused shapes (see
- * resa_decode_step_launches for the others), 1 for the no-allocation decode.
+ * resa_decode_step_launches for the others), 1 for the no-allocation decode,
+ * 1 for the dense decode.
  * Unknown names return -1. */
 RESA_API int32_t resa_kernels_per_call(const char *entry_point);
 

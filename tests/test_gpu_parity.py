@@ -292,6 +292,50 @@ def test_all_blocks_equals_dense(cuda_device):
     np.testing.assert_allclose(out.cpu().numpy(), dense, rtol=0, atol=OUT_ATOL)
 
 
+@pytest.mark.parametrize("case", [TINY, QWEN32K, RAGGED, RAGGED64, GQA8],
+                         ids=["tiny", "qwen32k", "ragged", "ragged64", "gqa8"])
+def test_dense_decode_matches_oracle(cuda_device, case):
+    """The dense baseline: append, then attention over every position."""
+    p = make(case)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L.to(cuda_device))
+    B, Hq, d = p.batch, p.num_q_heads, p.head_dim
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=cuda_device)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_dense_decode(cfg, lc.struct(), dev(p.q), dev(p.k_new), dev(p.v_new), out, lse, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    o.append(p.k_new, p.v_new, L)
+    np.testing.assert_array_equal(bits_of(lc.k), o.K)
+    np.testing.assert_array_equal(bits_of(lc.v), o.V)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+    ref, ref_lse = o.dense_attention(p.q, L)
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+
+
+def test_dense_decode_long_single_sequence(cuda_device):
+    """One unit over 100K positions: splits far beyond one wave of CTAs."""
+    p = make(dict(seed=11, batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128,
+                  block_size=16, ctx_lens=[100003], paged=True))
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L.to(cuda_device))
+    out = torch.empty(1, 8, 128, dtype=torch.float32, device=cuda_device)
+    lse = torch.empty(1, 8, dtype=torch.float32, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    R.resa_dense_decode(cfg, lc.struct(), dev(p.q), dev(p.k_new), dev(p.v_new), out, lse, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.append(p.k_new, p.v_new, L)
+    ref, ref_lse = o.dense_attention(p.q, L)
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+
+
 @pytest.mark.parametrize("shape,ctx,f,paged", [
     ((4, 2, 64), [2049], 32, True),
     ((28, 4, 128), [4096, 1000], 32, True),
