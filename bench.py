@@ -606,6 +606,7 @@ def run_resa(args):
         for name in EXTRA_WORKLOADS:
             if name != args.workload:
                 extra[name] = workload_block(name, stream, device, args.seed + 700, 3, hbm_peak)
+        extra["stagger64k"] = stagger_block(stream, device, args.seed + 700, 3, hbm_peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -827,6 +828,128 @@ def workload_block(name, stream, device, seed, reps, hbm_peak):
            "cycle_us_per_layer": per_layer_cycle,
            "amortised_us_per_token_per_layer": per_layer_cycle / wl["f"],
            "tokens_per_s": wl["batch"] * wl["f"] / (cyc_us * 1e-6),
+           "device_error_word": code}
+    del graphs, w
+    torch.cuda.empty_cache()
+    return res
+
+
+STAGGER = dict(base="loop64k", phases=[0, 8, 16, 24],
+               text="the loop64k decode loop with the four sequences' cycles offset by 8 "
+                    "steps: at every 8th step one sequence rectifies its last 32 tokens while "
+                    "the other three decode (row-mapped calls on one cache)")
+
+
+def stagger_block(stream, device, seed, reps, hbm_peak):
+    """Staggered rectification inside the decode batch: per step, one
+    resa_decode_step over the decoding rows and (at every 8th step) one
+    resa_rectify_attention over the rectifying row, both on the same cache
+    through row maps.  Reports the amortised µs per token next to the
+    synchronised schedule of the same workload."""
+    import torch
+    wl = WORKLOADS[STAGGER["base"]]
+    cycles = 2
+    w = GpuWorkload(wl, cycles, seed, device)
+    R = w.R
+    B, f, nl, hq, hkv, d = w.B, w.f, w.layers, w.hq, w.hkv, w.d
+    phase = STAGGER["phases"]
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 5)
+    q = torch.randn(cycles, f, nl, B, hq, d, generator=g, device=device).to(torch.bfloat16)
+    kn = torch.randn(cycles, f, nl, B, hkv, d, generator=g, device=device).to(torch.bfloat16)
+    vn = torch.randn(cycles, f, nl, B, hkv, d, generator=g, device=device).to(torch.bfloat16)
+    qc = torch.randn(cycles, f, nl, 1, f, hq, d, generator=g, device=device).to(torch.bfloat16)
+    kc = torch.randn(cycles, f, nl, 1, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
+    vc = torch.randn(cycles, f, nl, 1, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
+    out = torch.empty(f, nl, B, hq, d, device=device)
+    rout = torch.empty(nl, 1, f, hq, d, device=device)
+    dec_rows, rect_rows, topk = [], [], []
+    for t in range(cycles * f):
+        rect = [b for b in range(B) if (t + phase[b]) % f == f - 1]
+        dec = [b for b in range(B) if b not in rect]
+        assert len(rect) <= 1
+        Ls = [w.sched.ctx[b] + t + 1 for b in range(B)]
+        dec_rows.append(torch.tensor(dec, dtype=torch.int32, device=device))
+        rect_rows.append(torch.tensor(rect, dtype=torch.int32, device=device) if rect else None)
+        tk = torch.zeros((len(dec) + 3) // 4 * 4, dtype=torch.int32)
+        tk[:len(dec)] = torch.tensor([topk_rule(Ls[b]) for b in dec])
+        topk.append(tk.to(device))
+
+    def cache(layer, t, rows):
+        ptr = w.seq_len.data_ptr() + 4 * w.sched.Bpad * t
+        return R.make_cache(w.k[layer], w.v[layer], w.desc[layer], w.page_table, ptr, rows)
+
+    def launch_cycle(c):
+        for s in range(f):
+            t = c * f + s
+            n = int(dec_rows[t].numel())
+            for layer in range(nl):
+                R.resa_decode_step(w.cfg, cache(layer, t, dec_rows[t]), q[c, s, layer, :n],
+                                   kn[c, s, layer, :n], vn[c, s, layer, :n], topk[t], w.max_topk,
+                                   out[s, layer, :n], None, w.idx[layer], w.cnt[layer], w.ws)
+                if rect_rows[t] is not None:
+                    R.resa_rectify_attention(w.cfg, cache(layer, t, rect_rows[t]), f,
+                                             qc[c, s, layer], kc[c, s, layer], vc[c, s, layer],
+                                             rout[layer], None, w.ws)
+
+    graphs = []
+    with torch.cuda.stream(stream):
+        for c in range(cycles):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                launch_cycle(c)
+            graphs.append(gr)
+        graphs[0].replay()
+        graphs[1].replay()
+        graphs[1].replay()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            graphs[1].replay()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    cyc_us = 1e3 * e0.elapsed_time(e1) / reps / nl
+
+    def timed(enqueue, calls=28):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(gr, stream=stream):
+                for _ in range(calls):
+                    enqueue()
+            gr.replay()
+            torch.cuda.synchronize(device)
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(reps):
+                gr.replay()
+            a1.record(stream)
+        torch.cuda.synchronize(device)
+        return 1e3 * a0.elapsed_time(a1) / (reps * calls)
+
+    # the two kinds of call of the last cycle's step where sequence 0 rectifies
+    t_r = 2 * f - 1
+    n = int(dec_rows[t_r].numel())
+    dec_us = timed(lambda: R.resa_decode_step(
+        w.cfg, cache(0, t_r, dec_rows[t_r]), q[1, f - 1, 0, :n], kn[1, f - 1, 0, :n],
+        vn[1, f - 1, 0, :n], topk[t_r], w.max_topk, out[f - 1, 0, :n], None, w.idx[0], w.cnt[0],
+        w.ws))
+    rect_us = timed(lambda: R.resa_rectify_attention(
+        w.cfg, cache(0, t_r, rect_rows[t_r]), f, qc[1, f - 1, 0], kc[1, f - 1, 0],
+        vc[1, f - 1, 0], rout[0], None, w.ws))
+    code = R.resa_check_device_status(w.ws, raise_on_error=False)
+    res = {"description": STAGGER["text"], "phases": phase, "f": f,
+           "decode_step_us_3_sequences": dec_us, "rectify_us_1_sequence": rect_us,
+           "cycle_us_per_layer": cyc_us,
+           "amortised_us_per_token_per_layer": cyc_us / f,
+           "tokens_per_s": B * f / (cyc_us * nl * 1e-6),
+           "launches_per_cycle_per_layer": sum(
+               R.resa_decode_step_launches(w.cfg, int(dec_rows[t].numel()), w.max_pages,
+                                           w.num_pages) +
+               (R.resa_kernels_per_call("resa_rectify_attention") if rect_rows[t] is not None
+                else 0) for t in range(f, 2 * f)),
            "device_error_word": code}
     del graphs, w
     torch.cuda.empty_cache()

@@ -29,9 +29,11 @@ class LayerCache:
                                     dtype=torch.bfloat16, device=dev),
                    page_table=p.page_table.to(dev), seq_len=p.ctx_len.to(dev).clone())
 
-    def struct(self, seq_len=None) -> resa.resa_cache_t:
+    def struct(self, seq_len=None, rows=None) -> resa.resa_cache_t:
+        """The C struct; ``rows`` (int32 device tensor) restricts a call to
+        those rows of the page table, in that order."""
         return resa.make_cache(self.k, self.v, self.desc, self.page_table,
-                               self.seq_len if seq_len is None else seq_len)
+                               self.seq_len if seq_len is None else seq_len, rows)
 
     @property
     def batch(self) -> int:

@@ -170,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                          int max_pages, int num_pages, float scale_log2, float *__restrict__ part_o,
                          float *__restrict__ part_lse, uint32_t *__restrict__ tickets,
                          uint32_t *__restrict__ grid_bar, float *__restrict__ out,
-                         float *__restrict__ lse_out, uint32_t *err, const DecodeAppend app) {
+                         float *__restrict__ lse_out, uint32_t *err, const DecodeAppend app,
+                         const RowMap rm) {
     using SM = DecodeSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array itself so that
@@ -188,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t unit = (size_t)b * hkv + h;
 
     pdl_launch_next();
-    const int L = seq_len[b];
+    const int row = cache_row(rm, b, threadIdx.x == 0 && split == 0 ? err : nullptr);
+    const int L = row_seq_len(seq_len, row);
     if (threadIdx.x == 0) {
         mbar_init(&merge_bar, 1);
         fence_mbar_init();
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int CPR = D / 8;  // 16-byte chunks per K / V row
         if (threadIdx.x < CPR) {
             const int c = threadIdx.x, M = (L - 1) / kBlock, slot = (L - 1) % kBlock;
-            const int page = page_table[(size_t)b * max_pages + M];
+            const int page = page_table[(size_t)row * max_pages + M];
             if (page >= 0 && page < num_pages) {
                 const uint4 kx = app.k_new[unit * CPR + c], vx = app.v_new[unit * CPR + c];
                 const size_t o = (((size_t)page * hkv + h) * kBlock + slot) * CPR + c;
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int blk = list ? list[j0 + i] : j0 + i;
         int page = -1, ntok = 0;
         if (blk >= 0 && blk < nblk_seq) {
-            page = page_table[(size_t)b * max_pages + blk];
+            page = page_table[(size_t)row * max_pages + blk];
             if (page >= 0 && page < num_pages)
                 ntok = min(kBlock, L - blk * kBlock);
             else
@@ -587,7 +589,7 @@ cudaError_t launch_dn(const Shape &s, const void *k, const void *v,
                               (const uint8_t *)v, page_table, seq_len,
                               (const uint16_t *)q, block_idx, block_cnt, max_topk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets,
-                              spread ? grid_bar : (uint32_t *)nullptr, out, lse, err, app);
+                              spread ? grid_bar : (uint32_t *)nullptr, out, lse, err, app, s.rows);
 }
 
 }  // namespace

@@ -68,6 +68,7 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
         return RESA_ERR_UNSUPPORTED;
     if (!(cfg->sm_scale >= 0.f) || isinf(cfg->sm_scale)) return RESA_ERR_RANGE;
     if (cache->batch <= 0 || cache->max_pages <= 0 || cache->num_pages <= 0) return RESA_ERR_SHAPE;
+    if (cache->rows != nullptr && cache->table_rows <= 0) return RESA_ERR_SHAPE;
     if ((long long)cache->max_pages * kBlock > 0x7fffffffLL ||
         (long long)cache->num_pages * hkv * kBlock > 0x7fffffffLL || max_topk < 0)
         return RESA_ERR_RANGE;
@@ -76,7 +77,8 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     if ((long long)max_topk + 1 > (long long)kMaxDecodeSplits * kMaxBlocksPerSplit)
         return RESA_ERR_RANGE;
     if (!al16(cache->k) || !al16(cache->v) || !al16(cache->page_table) || !al16(cache->seq_len) ||
-        !al16(q) || !al16(out) || (reinterpret_cast<uintptr_t>(dev_error) & 3u) != 0)
+        (cache->rows != nullptr && !al16(cache->rows)) || !al16(q) || !al16(out) ||
+        (reinterpret_cast<uintptr_t>(dev_error) & 3u) != 0)
         return RESA_ERR_UNSUPPORTED;
 
     // Size the scratch use and refuse what does not fit.
@@ -121,6 +123,7 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     s.batch = cache->batch;
     s.max_pages = cache->max_pages;
     s.num_pages = cache->num_pages;
+    s.rows = RowMap{cache->rows, cache->rows ? cache->table_rows : cache->batch};
     const cudaError_t e = launch_sparse_decode(
         s, cache->k, cache->v, cache->page_table, cache->seq_len, q, block_idx, block_cnt, max_topk,
         splits, part_o, part_lse, tickets,

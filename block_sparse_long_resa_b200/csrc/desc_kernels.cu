@@ -23,18 +23,19 @@ __global__ void append_kernel(uint4 *__restrict__ K, uint4 *__restrict__ V,
                               uint4 *__restrict__ desc, const int32_t *__restrict__ page_table,
                               const int32_t *__restrict__ seq_len, const uint4 *__restrict__ k_new,
                               const uint4 *__restrict__ v_new, int hkv, int d, int max_pages,
-                              int num_pages, uint32_t *err) {
+                              int num_pages, const RowMap rm, uint32_t *err) {
     const int b = blockIdx.x;
     const int cpr = d / 8;  // 16-byte chunks per row
     const int h = threadIdx.x / cpr, c = threadIdx.x % cpr;
     if (h >= hkv) return;
-    const int L = seq_len[b];
+    const int row = cache_row(rm, b, threadIdx.x == 0 ? err : nullptr);
+    const int L = row_seq_len(seq_len, row);
     if (L < 1 || L > max_pages * kBlock) {
         if (threadIdx.x == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
         return;
     }
     const int pos = L - 1;
-    const int page = page_table[(size_t)b * max_pages + pos / kBlock];
+    const int page = page_table[(size_t)row * max_pages + pos / kBlock];
     if (page < 0 || page >= num_pages) {
         if (threadIdx.x == 0) set_error(err, RESA_DEVERR_PAGE);
         return;
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(kBuildThreads)
     build_desc_kernel(const uint4 *__restrict__ K, uint4 *__restrict__ desc,
                       const int32_t *__restrict__ page_table, const int32_t *__restrict__ seq_len,
                       const int32_t *__restrict__ first_block, int hkv, int d, int max_pages,
-                      int num_pages, uint32_t *err) {
+                      int num_pages, const RowMap rm, uint32_t *err) {
     const int b = blockIdx.y;
     const int cpr = d / 8;
     const int tpp = hkv * cpr;                 // threads per page
@@ -75,7 +76,8 @@ __global__ void __launch_bounds__(kBuildThreads)
     const int sub = threadIdx.x / tpp;
     const int h = (threadIdx.x % tpp) / cpr, c = threadIdx.x % cpr;
     if (sub >= ppp) return;
-    const int L = seq_len[b];
+    const int row = cache_row(rm, b, threadIdx.x == 0 && blockIdx.x == 0 ? err : nullptr);
+    const int L = row_seq_len(seq_len, row);
     if (L < 0 || L > max_pages * kBlock) {
         if (threadIdx.x == 0 && blockIdx.x == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
         return;
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(kBuildThreads)
     const int blk0 = blockIdx.x * kBuildPagesPerCta;
     for (int blk = blk0 + sub; blk < blk0 + kBuildPagesPerCta; blk += ppp) {
         if (blk < first || blk >= nblk) continue;
-        const int page = page_table[(size_t)b * max_pages + blk];
+        const int page = page_table[(size_t)row * max_pages + blk];
         if (page < 0 || page >= num_pages) {
             if (h == 0 && c == 0) set_error(err, RESA_DEVERR_PAGE);
             continue;
@@ -113,12 +115,14 @@ __global__ void rectify_writeback_kernel(uint4 *__restrict__ K, uint4 *__restric
                                          const int32_t *__restrict__ seq_len, int f,
                                          const uint4 *__restrict__ k_new,
                                          const uint4 *__restrict__ v_new, int hkv, int d,
-                                         int max_pages, int num_pages, uint32_t *err) {
+                                         int max_pages, int num_pages, const RowMap rm,
+                                         uint32_t *err) {
     const int b = blockIdx.y;
     const int cpr = d / 8;
     const int h = threadIdx.x / cpr, c = threadIdx.x % cpr;
     if (h >= hkv) return;
-    const int L = seq_len[b];
+    const int row = cache_row(rm, b, threadIdx.x == 0 && blockIdx.x == 0 ? err : nullptr);
+    const int L = row_seq_len(seq_len, row);
     if (L < 1 || L > max_pages * kBlock) {
         if (threadIdx.x == 0 && blockIdx.x == 0) set_error(err, RESA_DEVERR_SEQ_LEN);
         return;
@@ -130,7 +134,7 @@ __global__ void rectify_writeback_kernel(uint4 *__restrict__ K, uint4 *__restric
     const int start = L - f;
     const int blk = start / kBlock + blockIdx.x;
     if (blk > (L - 1) / kBlock) return;
-    const int page = page_table[(size_t)b * max_pages + blk];
+    const int page = page_table[(size_t)row * max_pages + blk];
     if (page < 0 || page >= num_pages) {
         if (threadIdx.x == 0) set_error(err, RESA_DEVERR_PAGE);
         return;
@@ -174,7 +178,7 @@ cudaError_t launch_append(const Shape &s, void *k, void *v, void *desc, const in
                           uint32_t *err, cudaStream_t st) {
     append_kernel<<<s.batch, s.hkv * (s.d / 8), 0, st>>>(
         (uint4 *)k, (uint4 *)v, (uint4 *)desc, page_table, seq_len, (const uint4 *)k_new,
-        (const uint4 *)v_new, s.hkv, s.d, s.max_pages, s.num_pages, err);
+        (const uint4 *)v_new, s.hkv, s.d, s.max_pages, s.num_pages, s.rows, err);
     return cudaGetLastError();
 }
 
@@ -184,7 +188,7 @@ cudaError_t launch_build_descriptors(const Shape &s, const void *k, void *desc,
     dim3 grid((s.max_pages + kBuildPagesPerCta - 1) / kBuildPagesPerCta, s.batch);
     build_desc_kernel<<<grid, kBuildThreads, 0, st>>>((const uint4 *)k, (uint4 *)desc, page_table,
                                                       seq_len, first_block, s.hkv, s.d,
-                                                      s.max_pages, s.num_pages, err);
+                                                      s.max_pages, s.num_pages, s.rows, err);
     return cudaGetLastError();
 }
 
@@ -195,7 +199,7 @@ cudaError_t launch_rectify_writeback(const Shape &s, void *k, void *v, void *des
     dim3 grid(f / kBlock + 2, s.batch);
     rectify_writeback_kernel<<<grid, s.hkv * (s.d / 8), 0, st>>>(
         (uint4 *)k, (uint4 *)v, (uint4 *)desc, page_table, seq_len, f, (const uint4 *)k_new,
-        (const uint4 *)v_new, s.hkv, s.d, s.max_pages, s.num_pages, err);
+        (const uint4 *)v_new, s.hkv, s.d, s.max_pages, s.num_pages, s.rows, err);
     return cudaGetLastError();
 }
 

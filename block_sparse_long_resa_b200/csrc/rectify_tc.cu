@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       int f, const uint16_t *__restrict__ q_chunk, int hkv, int g, int max_pages,
                       int num_pages, float scale_log2, float *__restrict__ part_o,
                       float *__restrict__ part_lse, uint32_t *__restrict__ tickets,
-                      float *__restrict__ out, float *__restrict__ lse_out, uint32_t *err) {
+                      float *__restrict__ out, float *__restrict__ lse_out, const RowMap rm,
+                      uint32_t *err) {
     using LY = TcLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hq = hkv * g;
     const int R = f * g;
 
-    const int L = seq_len[b];
+    const int srow = cache_row(rm, b, threadIdx.x == 0 && group == 0 && split == 0 ? err : nullptr);
+    const int L = row_seq_len(seq_len, srow);
     const bool seq_ok = L >= 1 && L <= max_pages * kBlock && f <= L;
     if (!seq_ok && threadIdx.x == 0 && group == 0 && split == 0)
         set_error(err, (L < 1 || L > max_pages * kBlock) ? RESA_DEVERR_SEQ_LEN : RESA_DEVERR_CHUNK);
@@ -183,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kWin = 32 / kBlocksPerTile;  // tiles per window
         auto load_win = [&](int w) -> int {
             const int blk = blk0 + w * 32 + lane;
-            return blk < blk1 ? page_table[(size_t)b * max_pages + blk] : -1;
+            return blk < blk1 ? page_table[(size_t)srow * max_pages + blk] : -1;
         };
         int win_cur = ntiles > 0 ? load_win(0) : -1;
         int win_next = ntiles > kWin ? load_win(1) : -1;
@@ -657,7 +659,7 @@ cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *pa
                               maps[4], maps[5], maps[6], maps[7],
                               page_table, seq_len, f, (const uint16_t *)q_chunk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out,
-                              lse, err);
+                              lse, s.rows, err);
 }
 
 }  // namespace

@@ -96,9 +96,12 @@ resa_status_t check_cache(const resa_cache_t *c, Shape *s, bool need_v, bool nee
     if (!aligned16(c->k) || (c->v && !aligned16(c->v)) || (c->desc && !aligned16(c->desc)) ||
         !aligned16(c->page_table) || !aligned16(c->seq_len))
         return RESA_ERR_UNSUPPORTED;
+    if (c->rows != nullptr && (c->table_rows <= 0 || !aligned16(c->rows)))
+        return c->table_rows <= 0 ? RESA_ERR_SHAPE : RESA_ERR_UNSUPPORTED;
     s->batch = c->batch;
     s->max_pages = c->max_pages;
     s->num_pages = c->num_pages;
+    s->rows = RowMap{c->rows, c->rows ? c->table_rows : c->batch};
     return RESA_OK;
 }
 

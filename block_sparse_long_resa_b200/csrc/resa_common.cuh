@@ -178,6 +178,30 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
     if (err) atomicOr(err, bit);
 }
 
+// Row map of a call (resa_cache_t.rows / table_rows): the call's i-th
+// sequence reads row rows[i] of page_table and seq_len, or row i without a map.
+struct RowMap {
+    const int32_t *rows;
+    int table_rows;
+};
+
+// The cache row of the call's sequence i; -1 (and RESA_DEVERR_ROW) for a
+// mapped row outside [0, table_rows).
+__device__ __forceinline__ int cache_row(const RowMap &m, int i, uint32_t *err) {
+    if (m.rows == nullptr) return i;
+    const int r = m.rows[i];
+    if (r < 0 || r >= m.table_rows) {
+        set_error(err, RESA_DEVERR_ROW);
+        return -1;
+    }
+    return r;
+}
+
+// seq_len of a cache row; an invalid row reads as an empty sequence.
+__device__ __forceinline__ int row_seq_len(const int32_t *seq_len, int row) {
+    return row >= 0 ? seq_len[row] : 0;
+}
+
 // Bounded grid barrier of a cooperatively launched (co-resident) grid; thread
 // 0 of every CTA calls it after a __threadfence and a __syncthreads.  One
 // 64-bit word holds (generation << 32) | arrivals: each CTA adds 1; the last
@@ -436,6 +460,7 @@ struct Shape {
     int hq, hkv, g, d, bs;
     float sm_scale;
     int batch, max_pages, num_pages;
+    RowMap rows;  // the cache's row map (rows == nullptr: identity)
 };
 
 cudaError_t launch_append(const Shape &s, void *k, void *v, void *desc, const int32_t *page_table,

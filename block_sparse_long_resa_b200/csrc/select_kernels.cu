@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                  float *__restrict__ scores, uint32_t *__restrict__ hist,
                  uint32_t *__restrict__ hist_range, int g, int max_pages, int num_pages,
                  uint4 *__restrict__ K, uint4 *__restrict__ V, const uint4 *__restrict__ k_new,
-                 const uint4 *__restrict__ v_new, uint32_t *err) {
+                 const uint4 *__restrict__ v_new, const RowMap rm, uint32_t *err) {
     using CF = ScoreCfg<D, HKV>;
     constexpr int PAGE_ELEMS = HKV * 2 * D;  // bf16 per descriptor page
     constexpr int PAGE_CHUNKS = CF::kPageBytes / 16;
@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const int b = blockIdx.y, x = blockIdx.x, X = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int hq = HKV * g;
-    const int L = seq_len[b];
+    const int row = cache_row(rm, b, x == 0 && threadIdx.x == 0 ? err : nullptr);
+    const int L = row_seq_len(seq_len, row);
     const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
     const int M = seq_ok ? (L - 1) / kBlock : 0;
     const int per = (M + X - 1) / X;
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const int n_mine = p_end - p_begin > warp ? (p_end - p_begin - warp + kScoreWarps - 1) / kScoreWarps : 0;
         auto batch_ids = [&](int t0) {
             const int t = t0 + lane;
-            return t < n_mine ? page_table[(size_t)b * max_pages + p_begin + warp + kScoreWarps * t] : -1;
+            return t < n_mine ? page_table[(size_t)row * max_pages + p_begin + warp + kScoreWarps * t] : -1;
         };
         int ids = batch_ids(0);
         pdl_wait();  // descriptors may be written by the preceding kernels
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         pdl_wait();
         if (!seq_ok) return;
         const int pos = L - 1;
-        const int page = page_table[(size_t)b * max_pages + pos / kBlock];
+        const int page = page_table[(size_t)row * max_pages + pos / kBlock];
         if (page < 0 || page >= num_pages) {
             if (lane == 0) set_error(err, RESA_DEVERR_PAGE);
             return;
@@ -400,7 +401,8 @@ __global__ void __launch_bounds__(kSelThreads)
     select_kernel(const float *__restrict__ scores, uint32_t *__restrict__ hist,
                   uint32_t *__restrict__ hist_range, const int32_t *__restrict__ seq_len,
                   const int32_t *__restrict__ topk, int max_topk, int32_t *__restrict__ block_idx,
-                  int32_t *__restrict__ block_cnt, int hkv, int max_pages, uint32_t *err) {
+                  int32_t *__restrict__ block_cnt, int hkv, int max_pages, const RowMap rm,
+                  uint32_t *err) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     __shared__ uint32_t keys_s[kSelKeys];
@@ -421,7 +423,7 @@ __global__ void __launch_bounds__(kSelThreads)
     const size_t unit = (size_t)b * hkv + h;
     int32_t *out = block_idx + unit * (max_topk + 1);
     int32_t *cnt = block_cnt + unit;
-    const int L = seq_len[b];
+    const int L = row_seq_len(seq_len, cache_row(rm, b, nullptr));
     const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
     const int M = seq_ok ? (L - 1) / kBlock : 0;
     int k = topk[b];
@@ -703,7 +705,8 @@ cudaError_t launch_score_d(const Shape &s, void *desc, const int32_t *page_table
         return launch_pdl(score_kernel<D, H>, grid, dim3(kScoreThreads), smem, st,            \
                           (uint16_t *)desc, page_table, seq_len, (const uint16_t *)q, scores, \
                           hist, hist_range, s.g, s.max_pages, s.num_pages, (uint4 *)K,        \
-                          (uint4 *)V, (const uint4 *)k_new, (const uint4 *)v_new, err);       \
+                          (uint4 *)V, (const uint4 *)k_new, (const uint4 *)v_new, s.rows,     \
+                          err);                                                               \
     }
     switch (s.hkv) {
         RESA_SCORE_CASE(1)
@@ -750,7 +753,7 @@ cudaError_t launch_select(const Shape &s, const float *scores, uint32_t *hist,
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, select_kernel, scores, hist, hist_range, seq_len, topk,
-                              max_topk, block_idx, block_cnt, s.hkv, s.max_pages, err);
+                              max_topk, block_idx, block_cnt, s.hkv, s.max_pages, s.rows, err);
 }
 
 }  // namespace resa

@@ -94,6 +94,7 @@ struct StepArgs {
     uint32_t *ukeys;           // [units][key_stride] every block's key
     unsigned long long *part;  // [units * G][kStepMaxGroup][D + 1] tagged partial (o, then lse)
     uint32_t *err;
+    RowMap rows;
     int hkv, g, max_pages, num_pages, max_topk, key_stride;
     float scale_log2;
 };
@@ -190,7 +191,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     const int b = u / hkv, h = u % hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int cta = u * G + x;
-    const int L = a.seq_len[b];
+    const int row = cache_row(a.rows, b, x == 0 && tid == 0 ? a.err : nullptr);
+    const int L = row_seq_len(a.seq_len, row);
     const bool seq_ok = L >= 1 && L <= a.max_pages * kBlock;
     const int M = seq_ok ? (L - 1) / kBlock : 0;
     int kq = a.topk[b];
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     const int per = (M + G - 1) / G;
     const int p0 = min(M, x * per);
     const int nmine = min(min(M, p0 + per) - p0, kStepMaxBlocks);  // the host keeps per <= cap
-    const size_t prow = (size_t)b * a.max_pages;
+    const size_t prow = (size_t)max(row, 0) * a.max_pages;  // an invalid row reads as empty
     uint32_t *ukeys_g = a.ukeys + (size_t)u * a.key_stride;
 
     // ---- prologue: inputs of the call only (before the dependency wait) ----
@@ -1059,6 +1061,7 @@ cudaError_t launch_decode_step_fused(const Shape &s, int G, void *k, void *v, vo
     a.ukeys = buf.ukeys;
     a.part = buf.part;
     a.err = buf.err;
+    a.rows = s.rows;
     a.hkv = s.hkv;
     a.g = s.g;
     a.max_pages = s.max_pages;

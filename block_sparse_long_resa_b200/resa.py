@@ -18,8 +18,8 @@ LIB_PATH = os.path.join(HERE, "libresa.so")
 RESA_OK = 0
 STATUS_NAMES = {0: "RESA_OK", 1: "RESA_ERR_NULL", 2: "RESA_ERR_SHAPE", 3: "RESA_ERR_RANGE",
                 4: "RESA_ERR_UNSUPPORTED", 5: "RESA_ERR_CUDA", 6: "RESA_ERR_DEVICE_CHECK"}
-DEVERR_SEQ_LEN, DEVERR_PAGE, DEVERR_BLOCK, DEVERR_TOPK, DEVERR_CHUNK, DEVERR_TIMEOUT = (
-    0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
+DEVERR_SEQ_LEN, DEVERR_PAGE, DEVERR_BLOCK, DEVERR_TOPK, DEVERR_CHUNK, DEVERR_TIMEOUT, DEVERR_ROW = (
+    0x1, 0x2, 0x4, 0x8, 0x10, 0x20, 0x40)
 
 
 class ResaError(RuntimeError):
@@ -40,7 +40,8 @@ class resa_cache_t(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("desc", ctypes.c_void_p),
                 ("page_table", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
                 ("batch", ctypes.c_int32), ("max_pages", ctypes.c_int32),
-                ("num_pages", ctypes.c_int32)]
+                ("num_pages", ctypes.c_int32), ("rows", ctypes.c_void_p),
+                ("table_rows", ctypes.c_int32)]
 
 
 _lib = None
@@ -116,11 +117,19 @@ def make_config(num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: 
     return resa_config_t(num_q_heads, num_kv_heads, head_dim, block_size, sm_scale)
 
 
-def make_cache(k, v, desc, page_table, seq_len) -> resa_cache_t:
+def make_cache(k, v, desc, page_table, seq_len, rows=None) -> resa_cache_t:
     """Cache struct over torch tensors k/v [pages][Hkv][b][d] bf16, desc
-    [pages][Hkv][2][d] bf16, page_table [B][max_pages] int32, seq_len [B] int32."""
+    [pages][Hkv][2][d] bf16, page_table [B][max_pages] int32, seq_len [B] int32.
+
+    With ``rows`` (int32 device tensor [n]) the call covers the n sequences in
+    those rows of page_table / seq_len (the row map of resa_cache_t)."""
+    nrows = int(page_table.shape[0])
+    if rows is None:
+        return resa_cache_t(_ptr(k), _ptr(v), _ptr(desc), _ptr(page_table), _ptr(seq_len),
+                            nrows, int(page_table.shape[1]), int(k.shape[0]), None, 0)
     return resa_cache_t(_ptr(k), _ptr(v), _ptr(desc), _ptr(page_table), _ptr(seq_len),
-                        int(page_table.shape[0]), int(page_table.shape[1]), int(k.shape[0]))
+                        int(rows.numel()), int(page_table.shape[1]), int(k.shape[0]),
+                        _ptr(rows), nrows)
 
 
 # ---------------------------------------------------------------------------

@@ -84,6 +84,7 @@ typedef enum {
 #define RESA_DEVERR_TOPK 0x8u      /* topk[b] > max_topk with more blocks available: clamped */
 #define RESA_DEVERR_CHUNK 0x10u    /* rectification chunk f > seq_len */
 #define RESA_DEVERR_TIMEOUT 0x20u  /* a bounded device wait gave up */
+#define RESA_DEVERR_ROW 0x40u      /* rows[i] outside [0, table_rows): sequence skipped */
 
 typedef struct {
     int32_t num_q_heads;   /* Hq */
@@ -93,15 +94,29 @@ typedef struct {
     float sm_scale;        /* softmax scale; 0 selects 1/sqrt(d) (Eq. 1) */
 } resa_config_t;
 
+/* Row map.  Without one (rows == NULL) the call's sequence i is row i of
+ * page_table and seq_len, which then hold `batch` rows.  With one, the call
+ * covers `batch` sequences drawn from a larger table: sequence i reads row
+ * rows[i] (device int32 [batch]) of page_table and seq_len, which hold
+ * `table_rows` rows, while every per-call array (q, k_new, v_new, topk,
+ * block lists, chunks, outputs) stays indexed by i.  This is how one batch
+ * mixes sequences in different phases of their ReSA cycle (the decoding ones
+ * in one resa_decode_step, the rectifying ones in one resa_rectify_attention,
+ * both on the same cache; ReSA summary §3.4.2-§3.4.3, per-request
+ * rectification in continuous batching).  The rows of one call must be
+ * distinct.  A row outside [0, table_rows) sets RESA_DEVERR_ROW (and
+ * RESA_DEVERR_SEQ_LEN) and the sequence is treated as empty. */
 typedef struct {
     void *k;                    /* [num_pages][Hkv][b][d] bf16, device */
     void *v;                    /* [num_pages][Hkv][b][d] bf16, device */
     void *desc;                 /* [num_pages][Hkv][2][d] bf16, device */
-    const int32_t *page_table;  /* [batch][max_pages], device */
-    const int32_t *seq_len;     /* [batch], device; counts the decode token */
-    int32_t batch;
+    const int32_t *page_table;  /* [rows][max_pages], device */
+    const int32_t *seq_len;     /* [rows], device; counts the decode token */
+    int32_t batch;              /* sequences this call covers */
     int32_t max_pages;          /* row length of page_table = max blocks per sequence */
     int32_t num_pages;          /* physical pages in k / v / desc */
+    const int32_t *rows;        /* row map [batch], device, or NULL (see above) */
+    int32_t table_rows;         /* rows of page_table / seq_len when rows != NULL */
 } resa_cache_t;
 
 /* Bytes of workspace needed for caches of `batch` sequences with up to

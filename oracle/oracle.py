@@ -274,6 +274,18 @@ class OracleCache:
                                                sm_scale)
         return res
 
+    def rows_view(self, rows) -> "OracleCache":
+        """The same cache seen by a call that covers the sequences in rows
+        ``rows`` of the page table, in that order (the row map of resa.h):
+        K, V and the descriptors are shared, so the view's steps update this
+        cache; per-call arrays passed to the view are indexed by position in
+        ``rows``."""
+        v = object.__new__(OracleCache)
+        v.__dict__.update(self.__dict__)
+        v.page_table = np.ascontiguousarray(self.page_table[np.asarray(rows, dtype=np.int64)])
+        v.B = v.page_table.shape[0]
+        return v
+
     # Views used by tests ----------------------------------------------------
     def keys(self, b: int, h: int, L: int) -> np.ndarray:
         """Keys of sequence b, kv head h, positions 0 .. L-1 as float32 [L][d]."""

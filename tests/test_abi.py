@@ -90,6 +90,13 @@ def test_host_validation_without_gpu(lib):
     assert _call_select(cfg, _cache(batch=0)) == 2
     assert _call_select(cfg, _cache(k=0x100008)) == 4                      # misaligned
     assert _call_select(cfg, _cache(), ws_bytes=16) == 2                   # workspace too small
+    assert _call_select(cfg, _cache(rows=0xb00000, table_rows=0)) == 2     # row map, no table
+    assert _call_select(cfg, _cache(rows=0xb00004, table_rows=4)) == 4     # misaligned row map
+    # dense decode: NULL token, misaligned query
+    assert lib.resa_dense_decode(ctypes.byref(cfg), ctypes.byref(_cache()), 0x600000, None,
+                                 0x610000, 0x620000, None, 0xa00000, 1 << 30, None) == 1
+    assert lib.resa_dense_decode(ctypes.byref(cfg), ctypes.byref(_cache()), 0x600008, 0x610000,
+                                 0x610000, 0x620000, None, 0xa00000, 1 << 30, None) == 4
     # rectify: f < 1 and chunk too large
     c = _cache()
     assert lib.resa_rectify_attention(ctypes.byref(cfg), ctypes.byref(c), 0, 1 << 20, 1 << 20,

@@ -398,3 +398,40 @@ def test_rectify_rows_equals_rectify_and_skips_short_sequences():
     for blk in range(3):
         page = fresh.page_table[1, blk]
         np.testing.assert_array_equal(a.K[page], fresh.K[page])
+
+
+def test_rows_view_mixed_step_equals_batch_wide_steps():
+    """A call over mapped rows (some sequences decode while others rectify)
+    gives each sequence what a batch-wide call gives it: sequences are
+    independent, so the view only changes which cache row a call reads."""
+    p = small_problem(seed=16, B=4, d=16, bs=4, ctx=(37, 22, 50, 41), topk=[3, 2, 4, 3])
+    f, max_topk = 8, 4
+    L = p.ctx_len + 1
+    q, kn, vn = p.q, p.k_new, p.v_new
+    qc, kc, vc = inputs.make_rectify_chunk(16, 4, f, 4, 2, 16)
+    dec, rect = [2, 0], [3, 1]
+
+    a = oracle_of(p)
+    a.build_descriptors(p.ctx_len)
+    r = a.rows_view(dec).decode_step(q[dec], kn[dec], vn[dec], p.topk[dec], L[dec], max_topk)
+    ro, rl = a.rows_view(rect).rectify(qc[rect], kc[rect], vc[rect], L[rect], f)
+
+    b_ = oracle_of(p)
+    b_.build_descriptors(p.ctx_len)
+    rb = b_.decode_step(q, kn, vn, p.topk, L, max_topk)
+    c_ = oracle_of(p)
+    c_.build_descriptors(p.ctx_len)
+    co, cl = c_.rectify(qc, kc, vc, L, f)
+
+    np.testing.assert_array_equal(r["block_idx"], rb["block_idx"][dec])
+    np.testing.assert_array_equal(r["out"], rb["out"][dec])
+    np.testing.assert_array_equal(r["lse"], rb["lse"][dec])
+    np.testing.assert_array_equal(ro, co[rect])
+    np.testing.assert_array_equal(rl, cl[rect])
+    for rows, ref in ((dec, b_), (rect, c_)):
+        for row in rows:
+            pages = a.page_table[row][a.page_table[row] >= 0]
+            pages = pages[: (int(L[row]) + 3) // 4]
+            np.testing.assert_array_equal(a.K[pages], ref.K[pages])
+            np.testing.assert_array_equal(a.V[pages], ref.V[pages])
+            np.testing.assert_array_equal(a.desc[pages], ref.desc[pages])
