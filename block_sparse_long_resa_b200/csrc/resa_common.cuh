@@ -178,6 +178,13 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
     if (err) atomicOr(err, bit);
 }
 
+// Warm L2 with [p, p + bytes): a bulk prefetch, no completion to wait for
+// and no shared memory (16-byte aligned address, bytes a multiple of 16).
+// It is only a cache fill, so it is coherent with any concurrent write.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Row map of a call (resa_cache_t.rows / table_rows): the call's i-th
 // sequence reads row rows[i] of page_table and seq_len, or row i without a map.
 struct RowMap {

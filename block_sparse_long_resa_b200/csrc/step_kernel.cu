@@ -558,6 +558,22 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
         d1 = (uint32_t)s_v[kVD1];
         above = s_v[kVAB];
+        if (mode == kModeMid) {
+            // The blocks above the boundary digit are selected whatever the
+            // boundary candidates settle: their K/V is pulled into L2 (each
+            // CTA its own scored range) while the threshold and the slices are
+            // worked out, so HBM streams the selection from here on.
+            const uint32_t hi1 = (d1 << 16) | 0xffffu;
+            #pragma unroll 1
+            for (int i = tid; i < nmine; i += kThreadsAll) {
+                const int pg = pages[i];
+                if (keys[i] > hi1 && pg >= 0 && pg < a.num_pages) {
+                    const size_t t = ((size_t)pg * hkv + h) * SM::kTileBytes;
+                    prefetch_l2(a.k_cache + t, SM::kTileBytes);
+                    prefetch_l2(a.v_cache + t, SM::kTileBytes);
+                }
+            }
+        }
     }
     // Work split: the unit's ordered work list is the selected blocks in
     // ascending order, then the current block (W = keff + 1 items); CTA x
