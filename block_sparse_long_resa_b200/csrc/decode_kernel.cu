@@ -36,7 +36,7 @@ constexpr int kStages = 3;
 
 template <int D>
 struct DecodeSmem {
-    static constexpr int kTileBytes = kBlock * D * 2;  // one K or V tile
+    static constexpr int kTileBytes = kTileRows * D * 2;  // one K or V tile (16 tokens)
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
     static constexpr int kMergeBytes = kWarps * kMaxGroup * (D + 3) * 4;
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          float *__restrict__ part_lse, uint32_t *__restrict__ tickets,
                          uint32_t *__restrict__ grid_bar, float *__restrict__ out,
                          float *__restrict__ lse_out, uint32_t *err, const DecodeAppend app,
-                         const RowMap rm) {
+                         const RowMap rm, int bs) {
     using SM = DecodeSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array itself so that
@@ -213,8 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     pdl_wait();  // block lists / counts come from the preceding selection
-    const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
-    const int nblk_seq = seq_ok ? (L + kBlock - 1) / kBlock : 0;
+    const bool seq_ok = L >= 1 && L <= max_pages * bs;
+    const int nblk_seq = seq_ok ? (L + bs - 1) / bs : 0;
+    // a block is bs / 16 tiles of 16 tokens
+    const int sub_shift = bs == 64 ? 2 : bs == 32 ? 1 : 0;
     // without a block list (dense decoding) every block of the sequence
     int cnt = block_idx ? block_cnt[unit] : nblk_seq;
     if (!seq_ok) {
@@ -233,11 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // below orders the append before its copies of that block.
         constexpr int CPR = D / 8;  // 16-byte chunks per K / V row
         if (threadIdx.x < CPR) {
-            const int c = threadIdx.x, M = (L - 1) / kBlock, slot = (L - 1) % kBlock;
+            const int c = threadIdx.x, M = (L - 1) / bs, slot = (L - 1) % bs;
             const int page = page_table[(size_t)row * max_pages + M];
             if (page >= 0 && page < num_pages) {
                 const uint4 kx = app.k_new[unit * CPR + c], vx = app.v_new[unit * CPR + c];
-                const size_t o = (((size_t)page * hkv + h) * kBlock + slot) * CPR + c;
+                const size_t o = (((size_t)page * hkv + h) * bs + slot) * CPR + c;
                 reinterpret_cast<uint4 *>(app.k)[o] = kx;
                 reinterpret_cast<uint4 *>(app.v)[o] = vx;
                 uint4 *dmn = reinterpret_cast<uint4 *>(app.desc) + (((size_t)page * hkv + h) * 2) * CPR + c;
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (blk >= 0 && blk < nblk_seq) {
             page = page_table[(size_t)row * max_pages + blk];
             if (page >= 0 && page < num_pages)
-                ntok = min(kBlock, L - blk * kBlock);
+                ntok = min(bs, L - blk * bs);
             else
                 set_error(err, RESA_DEVERR_PAGE);
         } else {
@@ -272,19 +274,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    // This warp's blocks: slice entries warp + kWarps * t.  Block t goes to
-    // ring slot t % kStages: its K and V tiles (16 x D bf16 each, contiguous
-    // in the cache) are copied with 16-byte cp.async, lane chunk q to the
-    // 128-byte-swizzled position of (row q / 8, chunk q % 8), one copy group
-    // per block (empty groups keep the count uniform).
-    const int n_mine = warp < nslice ? (nslice - warp + kWarps - 1) / kWarps : 0;
+    // The slice's 16-token tiles (bs / 16 per block, in order): this warp
+    // takes tiles warp + kWarps * t.  Tile t goes to ring slot t % kStages:
+    // its K and V (16 x D bf16 each, contiguous in the cache) are copied with
+    // 16-byte cp.async, lane chunk q to the 128-byte-swizzled position of
+    // (row q / 8, chunk q % 8), one copy group per tile (empty groups keep
+    // the count uniform).
+    const int nsub = nslice << sub_shift;
+    const int n_mine = warp < nsub ? (nsub - warp + kWarps - 1) / kWarps : 0;
     uint8_t *ring = smem + (size_t)warp * kStages * SM::kStageBytes;
     constexpr int kPerLane = SM::kTileBytes / 16 / 32;
+    // (page, valid tokens) of tile e of the slice
+    auto tile_of = [&](int e) -> int2 {
+        const int2 mt = meta[e >> sub_shift];
+        const int j = e & ((1 << sub_shift) - 1);
+        return make_int2(mt.x * (1 << sub_shift) + j, min(kTileRows, mt.y - kTileRows * j));
+    };
     auto issue = [&](int t) {
         if (t < n_mine) {
-            const int2 mt = meta[warp + kWarps * t];
+            const int2 mt = tile_of(warp + kWarps * t);
             if (mt.y > 0) {
-                const size_t tile = ((size_t)mt.x * hkv + h) * SM::kTileBytes;
+                const size_t tile =
+                    (((size_t)(mt.x >> sub_shift) * hkv + h) << sub_shift | (mt.x & ((1 << sub_shift) - 1))) *
+                    SM::kTileBytes;
                 uint8_t *st = ring + (size_t)(t % kStages) * SM::kStageBytes;
 #pragma unroll
                 for (int k = 0; k < kPerLane; ++k) {
@@ -306,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue(t + kStages - 1);  // refills the slot of block t - 1
         cp_async_wait<kStages - 1>();
         __syncwarp();
-        const int ntok = meta[warp + kWarps * t].y;
+        const int ntok = tile_of(warp + kWarps * t).y;
         if (ntok > 0) {
             const uint32_t ks = smem_u32(ring + (size_t)(t % kStages) * SM::kStageBytes);
             attend_block_swapped<D, NT>(st, qb, ks, ks + SM::kTileBytes, ntok, scale_log2, lane);
@@ -589,7 +601,8 @@ cudaError_t launch_dn(const Shape &s, const void *k, const void *v,
                               (const uint8_t *)v, page_table, seq_len,
                               (const uint16_t *)q, block_idx, block_cnt, max_topk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets,
-                              spread ? grid_bar : (uint32_t *)nullptr, out, lse, err, app, s.rows);
+                              spread ? grid_bar : (uint32_t *)nullptr, out, lse, err, app, s.rows,
+                              s.bs);
 }
 
 }  // namespace

@@ -64,13 +64,15 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
         return RESA_ERR_SHAPE;
     const int hkv = cfg->num_kv_heads, g = cfg->num_q_heads / cfg->num_kv_heads;
     if (g > kMaxGroup || !(hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8) ||
-        !(cfg->head_dim == 64 || cfg->head_dim == 128) || cfg->block_size != kBlock)
+        !(cfg->head_dim == 64 || cfg->head_dim == 128) ||
+        !(cfg->block_size == 16 || cfg->block_size == 32 || cfg->block_size == 64))
         return RESA_ERR_UNSUPPORTED;
     if (!(cfg->sm_scale >= 0.f) || isinf(cfg->sm_scale)) return RESA_ERR_RANGE;
     if (cache->batch <= 0 || cache->max_pages <= 0 || cache->num_pages <= 0) return RESA_ERR_SHAPE;
     if (cache->rows != nullptr && cache->table_rows <= 0) return RESA_ERR_SHAPE;
-    if ((long long)cache->max_pages * kBlock > 0x7fffffffLL ||
-        (long long)cache->num_pages * hkv * kBlock > 0x7fffffffLL || max_topk < 0)
+    const int bs = cfg->block_size;
+    if ((long long)cache->max_pages * bs > 0x7fffffffLL ||
+        (long long)cache->num_pages * hkv * bs > 0x7fffffffLL || max_topk < 0)
         return RESA_ERR_RANGE;
     // The split merge holds the weights of at most kMaxDecodeSplits splits:
     // the same bound resa_sparse_decode enforces (max_topk + 1 <= 1024 * 512).
@@ -118,7 +120,7 @@ extern "C" resa_status_t resa_sparse_decode_noalloc(const resa_config_t *cfg,
     s.hkv = hkv;
     s.g = g;
     s.d = d;
-    s.bs = kBlock;
+    s.bs = bs;
     s.sm_scale = cfg->sm_scale > 0.f ? cfg->sm_scale : 1.0f / sqrtf((float)d);
     s.batch = cache->batch;
     s.max_pages = cache->max_pages;

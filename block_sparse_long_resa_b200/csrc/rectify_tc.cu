@@ -44,7 +44,6 @@ namespace {
 
 constexpr int kRows = kRectRowsPerCta;  // 256
 constexpr int kKeys = 64;               // keys per KV tile
-constexpr int kBlocksPerTile = kKeys / kBlock;
 constexpr int kStages = 3;
 constexpr int kNumConv = 2;             // converter warps
 constexpr int kWarpSm0 = 4;             // first softmax warp
@@ -107,7 +106,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t x, float sca
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-template <int D>
+template <int D, int BS>
 __global__ void __launch_bounds__(kThreads, 1)
     rectify_tc_kernel(const __grid_constant__ CUtensorMap k0map,
                       const __grid_constant__ CUtensorMap k1map,
@@ -124,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       float *__restrict__ out, float *__restrict__ lse_out, const RowMap rm,
                       uint32_t *err) {
     using LY = TcLayout<D>;
+    constexpr int kBPT = kKeys / BS;  // blocks per 64-key tile
+    static_assert(kKeys % BS == 0 && kBPT <= 4, "a tile holds whole blocks");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
@@ -143,18 +144,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int srow = cache_row(rm, b, threadIdx.x == 0 && group == 0 && split == 0 ? err : nullptr);
     const int L = row_seq_len(seq_len, srow);
-    const bool seq_ok = L >= 1 && L <= max_pages * kBlock && f <= L;
+    const bool seq_ok = L >= 1 && L <= max_pages * BS && f <= L;
     if (!seq_ok && threadIdx.x == 0 && group == 0 && split == 0)
-        set_error(err, (L < 1 || L > max_pages * kBlock) ? RESA_DEVERR_SEQ_LEN : RESA_DEVERR_CHUNK);
+        set_error(err, (L < 1 || L > max_pages * BS) ? RESA_DEVERR_SEQ_LEN : RESA_DEVERR_CHUNK);
     const int start = L - f;
     const int row0 = group * kRows;
     const int last_row = min(R, row0 + kRows) - 1;
     const int lim_max = (seq_ok && row0 < R) ? start + last_row / g + 1 : 0;
-    const int nblk = (lim_max + kBlock - 1) / kBlock;
+    const int nblk = (lim_max + BS - 1) / BS;
     int per = (nblk + S - 1) / S;
-    per = (per + kBlocksPerTile - 1) / kBlocksPerTile * kBlocksPerTile;
+    per = (per + kBPT - 1) / kBPT * kBPT;
     const int blk0 = min(nblk, split * per), blk1 = min(nblk, blk0 + per);
-    const int ntiles = (blk1 - blk0 + kBlocksPerTile - 1) / kBlocksPerTile;
+    const int ntiles = (blk1 - blk0 + kBPT - 1) / kBPT;
 
     uint8_t *q_s = smem + LY::kQOff;
     uint8_t *kv_s = smem + LY::kKVOff;
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {  // ------------------------------------------------ TMA producer
         // Page ids arrive 32 blocks (8 tiles) at a time, one id a lane, with
         // the next window's load already in flight; they are checked when used.
-        constexpr int kWin = 32 / kBlocksPerTile;  // tiles per window
+        constexpr int kWin = 32 / kBPT;  // tiles per window
         auto load_win = [&](int w) -> int {
             const int blk = blk0 + w * 32 + lane;
             return blk < blk1 ? page_table[(size_t)srow * max_pages + blk] : -1;
@@ -199,9 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 win_cur = win_next;
                 win_next = i + kWin < ntiles ? load_win(i / kWin + 1) : -1;
             }
-            const int blk = blk0 + i * kBlocksPerTile + lane;
-            int page = __shfl_sync(0xffffffffu, win_cur, ((i % kWin) * kBlocksPerTile + lane) & 31);
-            if (lane < kBlocksPerTile && blk < blk1) {
+            const int blk = blk0 + i * kBPT + lane;
+            int page = __shfl_sync(0xffffffffu, win_cur, ((i % kWin) * kBPT + lane) & 31);
+            if (lane < kBPT && blk < blk1) {
                 if (page < 0 || page >= num_pages) {
                     set_error(err, RESA_DEVERR_PAGE);
                     page = -1;
@@ -210,10 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 page = -1;
             }
             const uint32_t vmask = __ballot_sync(0xffffffffu, page >= 0);
-            const uint32_t bytes = (uint32_t)__popc(vmask) * 2u * LY::kHalves * kBlock * 128u;
+            const uint32_t bytes = (uint32_t)__popc(vmask) * 2u * LY::kHalves * BS * 128u;
             // four valid blocks on consecutive pages: one 4-page box per half
             const int page0 = __shfl_sync(0xffffffffu, page, 0);
-            const bool run = __all_sync(0xffffffffu, lane >= kBlocksPerTile ||
+            const bool run = __all_sync(0xffffffffu, lane >= kBPT ||
                                                           (page >= 0 && page == page0 + lane));
             if (lane == 0) {
                 stage_vmask[s] = vmask;
@@ -235,10 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else if (page >= 0) {
-                const int y = (page * hkv + h) * kBlock;
+                const int y = (page * hkv + h) * BS;
                 uint8_t *kt = kv_s + (size_t)s * 2 * LY::kKV;
                 uint8_t *vt = kt + LY::kKV;
-                const int off = lane * kBlock * 128;  // this block's 16 rows in each half
+                const int off = lane * BS * 128;  // this block's BS rows in each half
                 tc::tma_load_2d(kt + off, &k0map, 0, y, &kv_full[s]);
                 tc::tma_load_2d(vt + off, &v0map, 0, y, &kv_full[s]);
                 if (LY::kHalves == 2) {
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t vmask = stage_vmask[s];
             uint4 *vt = reinterpret_cast<uint4 *>(kv_s + (size_t)s * 2 * LY::kKV + LY::kKV);
             constexpr int kChunks = LY::kKV / 16;           // 16-byte chunks of the tile
-            constexpr int kChunksPerBlock = kBlock * 128 / 16;  // per half
+            constexpr int kChunksPerBlock = BS * 128 / 16;  // per half
             constexpr int kPer = kChunks / kConvThreads;
             static_assert(kChunks % kConvThreads == 0, "equal converter shares");
             // the thread's chunks into registers (blocks not loaded become
@@ -398,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Keys every valid row of this CTA may see: tiles entirely below this
         // limit (and fully loaded) need no mask.
         const int lim_cta = seq_ok ? start + row0 / g + 1 : 0;
-        const int tend = blk1 * kBlock;
+        const int tend = blk1 * BS;
         for (int i = 0; i < ntiles; ++i) {
             const int buf = i & 1;
             ok = mbar_wait_bounded(&s_full[buf], (i / 2) & 1) &&
@@ -417,9 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tmem_ld32(scol, sv[0]);
             tc::tmem_ld32(scol + 32, sv[1]);
             tc::tmem_wait_ld();
-            const int t0 = (blk0 + i * kBlocksPerTile) * kBlock;
+            const int t0 = (blk0 + i * kBPT) * BS;
             const uint32_t vmask = stage_vmask[i % kStages];
-            const bool full_tile = vmask == 0xFu && t0 + kKeys <= tend && t0 + kKeys <= lim_cta;
+            const bool full_tile = vmask == (1u << kBPT) - 1u && t0 + kKeys <= tend && t0 + kKeys <= lim_cta;
             float x[64];  // raw logits; -inf where masked
             float mraw = -INFINITY;
             if (full_tile) {
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     const int t = t0 + j;
-                    const bool valid = t < lim && t < tend && ((vmask >> (j / kBlock)) & 1u);
+                    const bool valid = t < lim && t < tend && ((vmask >> (j / BS)) & 1u);
                     x[j] = valid ? __uint_as_float(sv[j >> 5][j & 31]) : -INFINITY;
                     mraw = fmaxf(mraw, x[j]);
                 }
@@ -631,14 +632,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D>
+template <int D, int BS>
 cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *page_table,
                       const int32_t *seq_len, int f, const void *q_chunk, int groups, int splits,
                       float *part_o, float *part_lse, uint32_t *tickets, float *out, float *lse,
                       uint32_t *err, cudaStream_t st) {
     constexpr int smem = TcLayout<D>::kBytes;
     static std::atomic<int> done[64];
-    cudaError_t e = ensure_smem(rectify_tc_kernel<D>, smem, done);
+    cudaError_t e = ensure_smem(rectify_tc_kernel<D, BS>, smem, done);
     if (e != cudaSuccess) return e;
     const float scale_log2 = s.sm_scale * 1.4426950408889634f;
     dim3 grid(groups, splits, s.batch * s.hkv);
@@ -655,7 +656,7 @@ cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *pa
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = splits > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, rectify_tc_kernel<D>, maps[0], maps[1], maps[2], maps[3],
+    return cudaLaunchKernelEx(&cfg, rectify_tc_kernel<D, BS>, maps[0], maps[1], maps[2], maps[3],
                               maps[4], maps[5], maps[6], maps[7],
                               page_table, seq_len, f, (const uint16_t *)q_chunk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out,
@@ -670,12 +671,17 @@ cudaError_t launch_rectify_attention(const Shape &s, const CUtensorMap *maps,
                                      float *part_lse, uint32_t *tickets, float *out, float *lse,
                                      uint32_t *err, cudaStream_t st) {
     if (groups > kMaxRowTiles) return cudaErrorInvalidValue;
-    if (s.d == 128)
-        return launch_tc<128>(s, maps, page_table, seq_len, f, q_chunk, groups, splits, part_o,
-                              part_lse, tickets, out, lse, err, st);
-    if (s.d == 64)
-        return launch_tc<64>(s, maps, page_table, seq_len, f, q_chunk, groups, splits, part_o,
-                             part_lse, tickets, out, lse, err, st);
+#define RESA_RECT_CASE(D, BS)                                                                 \
+    if (s.d == D && s.bs == BS)                                                               \
+        return launch_tc<D, BS>(s, maps, page_table, seq_len, f, q_chunk, groups, splits, part_o, \
+                                part_lse, tickets, out, lse, err, st);
+    RESA_RECT_CASE(128, 16)
+    RESA_RECT_CASE(128, 32)
+    RESA_RECT_CASE(128, 64)
+    RESA_RECT_CASE(64, 16)
+    RESA_RECT_CASE(64, 32)
+    RESA_RECT_CASE(64, 64)
+#undef RESA_RECT_CASE
     return cudaErrorInvalidValue;
 }
 

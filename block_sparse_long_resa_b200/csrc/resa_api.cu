@@ -28,14 +28,15 @@ EncodeTiledFn encode_fn() {
 
 // One channel half (64 columns) of a K or V cache as a 2-D tensor: rows are
 // tokens of every (page, head) block (row stride d*2 bytes); one box is the
-// 16 rows x 64 channels of one block, 128-byte swizzled.
-bool make_kv_half_map(CUtensorMap *map, void *base, int half, int num_pages, int hkv, int d) {
+// bs rows x 64 channels of one block, 128-byte swizzled.
+bool make_kv_half_map(CUtensorMap *map, void *base, int half, int num_pages, int hkv, int d,
+                      int bs) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     void *b = static_cast<uint8_t *>(base) + (size_t)half * 128;
-    const cuuint64_t dims[2] = {64, (cuuint64_t)num_pages * hkv * kBlock};
+    const cuuint64_t dims[2] = {64, (cuuint64_t)num_pages * hkv * bs};
     const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kBlock};
+    const cuuint32_t box[2] = {64, (cuuint32_t)bs};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -44,16 +45,18 @@ bool make_kv_half_map(CUtensorMap *map, void *base, int half, int num_pages, int
 }
 
 // The same channel half as a 4-D tensor (channels, tokens, heads, pages):
-// one box is the 16 tokens of one head on four consecutive pages, 128-byte
-// swizzled, laid out in shared memory exactly as four single-block boxes.
-bool make_kv_half_run_map(CUtensorMap *map, void *base, int half, int num_pages, int hkv, int d) {
+// one box is the bs tokens of one head on the 64 / bs consecutive pages of a
+// 64-key tile, 128-byte swizzled, laid out in shared memory exactly as that
+// many single-block boxes.
+bool make_kv_half_run_map(CUtensorMap *map, void *base, int half, int num_pages, int hkv, int d,
+                          int bs) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     void *b = static_cast<uint8_t *>(base) + (size_t)half * 128;
-    const cuuint64_t dims[4] = {64, (cuuint64_t)kBlock, (cuuint64_t)hkv, (cuuint64_t)num_pages};
-    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)kBlock * d * 2,
-                                   (cuuint64_t)hkv * kBlock * d * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)kBlock, 1, 4};
+    const cuuint64_t dims[4] = {64, (cuuint64_t)bs, (cuuint64_t)hkv, (cuuint64_t)num_pages};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)bs * d * 2,
+                                   (cuuint64_t)hkv * bs * d * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)bs, 1, (cuuint32_t)(64 / bs)};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, b, dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -74,7 +77,8 @@ resa_status_t check_config(const resa_config_t *cfg, Shape *s) {
     const int hkv = cfg->num_kv_heads;
     if (!(hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8)) return RESA_ERR_UNSUPPORTED;
     if (!(cfg->head_dim == 64 || cfg->head_dim == 128)) return RESA_ERR_UNSUPPORTED;
-    if (cfg->block_size != kBlock) return RESA_ERR_UNSUPPORTED;
+    if (!(cfg->block_size == 16 || cfg->block_size == 32 || cfg->block_size == 64))
+        return RESA_ERR_UNSUPPORTED;
     if (!(cfg->sm_scale >= 0.f) || isinf(cfg->sm_scale)) return RESA_ERR_RANGE;
     s->hq = cfg->num_q_heads;
     s->hkv = hkv;
@@ -91,8 +95,8 @@ resa_status_t check_cache(const resa_cache_t *c, Shape *s, bool need_v, bool nee
     if (need_v && !c->v) return RESA_ERR_NULL;
     if (need_desc && !c->desc) return RESA_ERR_NULL;
     if (c->batch <= 0 || c->max_pages <= 0 || c->num_pages <= 0) return RESA_ERR_SHAPE;
-    if ((long long)c->max_pages * kBlock > 0x7fffffffLL) return RESA_ERR_RANGE;
-    if ((long long)c->num_pages * s->hkv * kBlock > 0x7fffffffLL) return RESA_ERR_RANGE;
+    if ((long long)c->max_pages * s->bs > 0x7fffffffLL) return RESA_ERR_RANGE;
+    if ((long long)c->num_pages * s->hkv * s->bs > 0x7fffffffLL) return RESA_ERR_RANGE;
     if (!aligned16(c->k) || (c->v && !aligned16(c->v)) || (c->desc && !aligned16(c->desc)) ||
         !aligned16(c->page_table) || !aligned16(c->seq_len))
         return RESA_ERR_UNSUPPORTED;
@@ -162,6 +166,7 @@ int sm_count() {
 // CTAs per (sequence, kv head) of the fused decode step for this shape, 0 when
 // the step runs as three launches (score + append, select, decode).
 int fused_step_ctas(const Shape &s) {
+    if (s.bs != 16) return 0;                            // 16-token blocks only
     if ((long long)s.num_pages >= (1LL << 27)) return 0;  // packed (page, tokens) work items
     return step_ctas_per_unit(s.batch * s.hkv, s.g, s.d, s.max_pages, sm_count());
 }
@@ -306,10 +311,10 @@ resa_status_t resa_rectify_attention(const resa_config_t *cfg, const resa_cache_
     const int halves = s.d / 64;
     for (int hf = 0; hf < 2; ++hf) {
         const int use = hf < halves ? hf : 0;  // d = 64: one half, second map unused
-        if (!make_kv_half_map(&maps[hf], cache->k, use, s.num_pages, s.hkv, s.d) ||
-            !make_kv_half_map(&maps[2 + hf], cache->v, use, s.num_pages, s.hkv, s.d) ||
-            !make_kv_half_run_map(&maps[4 + hf], cache->k, use, s.num_pages, s.hkv, s.d) ||
-            !make_kv_half_run_map(&maps[6 + hf], cache->v, use, s.num_pages, s.hkv, s.d))
+        if (!make_kv_half_map(&maps[hf], cache->k, use, s.num_pages, s.hkv, s.d, s.bs) ||
+            !make_kv_half_map(&maps[2 + hf], cache->v, use, s.num_pages, s.hkv, s.d, s.bs) ||
+            !make_kv_half_run_map(&maps[4 + hf], cache->k, use, s.num_pages, s.hkv, s.d, s.bs) ||
+            !make_kv_half_run_map(&maps[6 + hf], cache->v, use, s.num_pages, s.hkv, s.d, s.bs))
             return RESA_ERR_CUDA;
     }
     return cuda_status(launch_rectify_attention(

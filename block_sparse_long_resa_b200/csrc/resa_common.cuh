@@ -16,7 +16,8 @@ namespace resa {
 // ---------------------------------------------------------------------------
 // Fixed shape limits
 // ---------------------------------------------------------------------------
-constexpr int kBlock = 16;          // tokens per block / page
+constexpr int kBlock = 16;          // tokens per block / page of the fused decode step
+constexpr int kTileRows = 16;       // tokens per K / V tile (a block holds bs / 16 of them)
 constexpr int kMaxGroup = 16;       // query heads per kv head (one m16 MMA tile)
 constexpr int kMaxKvHeads = 8;
 constexpr int kNumSms = 148;

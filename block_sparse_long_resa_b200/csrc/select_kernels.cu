@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                  float *__restrict__ scores, uint32_t *__restrict__ hist,
                  uint32_t *__restrict__ hist_range, int g, int max_pages, int num_pages,
                  uint4 *__restrict__ K, uint4 *__restrict__ V, const uint4 *__restrict__ k_new,
-                 const uint4 *__restrict__ v_new, const RowMap rm, uint32_t *err) {
+                 const uint4 *__restrict__ v_new, int bs, const RowMap rm, uint32_t *err) {
     using CF = ScoreCfg<D, HKV>;
     constexpr int PAGE_ELEMS = HKV * 2 * D;  // bf16 per descriptor page
     constexpr int PAGE_CHUNKS = CF::kPageBytes / 16;
@@ -81,8 +81,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const int hq = HKV * g;
     const int row = cache_row(rm, b, x == 0 && threadIdx.x == 0 ? err : nullptr);
     const int L = row_seq_len(seq_len, row);
-    const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
-    const int M = seq_ok ? (L - 1) / kBlock : 0;
+    const bool seq_ok = L >= 1 && L <= max_pages * bs;
+    const int M = seq_ok ? (L - 1) / bs : 0;
     const int per = (M + X - 1) / X;
     const int p_begin = min(M, x * per), p_end = min(M, p_begin + per);
 
@@ -271,19 +271,19 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         pdl_wait();
         if (!seq_ok) return;
         const int pos = L - 1;
-        const int page = page_table[(size_t)row * max_pages + pos / kBlock];
+        const int page = page_table[(size_t)row * max_pages + pos / bs];
         if (page < 0 || page >= num_pages) {
             if (lane == 0) set_error(err, RESA_DEVERR_PAGE);
             return;
         }
-        const int slot = pos % kBlock;
+        const int slot = pos % bs;
         constexpr int CPR = D / 8;  // 16-byte chunks per row
         uint4 *dsc = reinterpret_cast<uint4 *>(desc);
         for (int e = lane; e < HKV * CPR; e += 32) {
             const int h = e / CPR, cc = e % CPR;
             const uint4 kx = k_new[((size_t)b * HKV + h) * CPR + cc];
             const uint4 vx = v_new[((size_t)b * HKV + h) * CPR + cc];
-            const size_t o = (((size_t)page * HKV + h) * kBlock + slot) * CPR + cc;
+            const size_t o = (((size_t)page * HKV + h) * bs + slot) * CPR + cc;
             K[o] = kx;
             V[o] = vx;
             uint4 *pmn = &dsc[(((size_t)page * HKV + h) * 2) * CPR + cc];
@@ -401,8 +401,8 @@ __global__ void __launch_bounds__(kSelThreads)
     select_kernel(const float *__restrict__ scores, uint32_t *__restrict__ hist,
                   uint32_t *__restrict__ hist_range, const int32_t *__restrict__ seq_len,
                   const int32_t *__restrict__ topk, int max_topk, int32_t *__restrict__ block_idx,
-                  int32_t *__restrict__ block_cnt, int hkv, int max_pages, const RowMap rm,
-                  uint32_t *err) {
+                  int32_t *__restrict__ block_cnt, int hkv, int max_pages, int bs,
+                  const RowMap rm, uint32_t *err) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     __shared__ uint32_t keys_s[kSelKeys];
@@ -424,8 +424,8 @@ __global__ void __launch_bounds__(kSelThreads)
     int32_t *out = block_idx + unit * (max_topk + 1);
     int32_t *cnt = block_cnt + unit;
     const int L = row_seq_len(seq_len, cache_row(rm, b, nullptr));
-    const bool seq_ok = L >= 1 && L <= max_pages * kBlock;
-    const int M = seq_ok ? (L - 1) / kBlock : 0;
+    const bool seq_ok = L >= 1 && L <= max_pages * bs;
+    const int M = seq_ok ? (L - 1) / bs : 0;
     int k = topk[b];
     k = k < 0 ? 0 : k;
     bool topk_err = false;
@@ -705,7 +705,7 @@ cudaError_t launch_score_d(const Shape &s, void *desc, const int32_t *page_table
         return launch_pdl(score_kernel<D, H>, grid, dim3(kScoreThreads), smem, st,            \
                           (uint16_t *)desc, page_table, seq_len, (const uint16_t *)q, scores, \
                           hist, hist_range, s.g, s.max_pages, s.num_pages, (uint4 *)K,        \
-                          (uint4 *)V, (const uint4 *)k_new, (const uint4 *)v_new, s.rows,     \
+                          (uint4 *)V, (const uint4 *)k_new, (const uint4 *)v_new, s.bs, s.rows, \
                           err);                                                               \
     }
     switch (s.hkv) {
@@ -753,7 +753,8 @@ cudaError_t launch_select(const Shape &s, const float *scores, uint32_t *hist,
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, select_kernel, scores, hist, hist_range, seq_len, topk,
-                              max_topk, block_idx, block_cnt, s.hkv, s.max_pages, s.rows, err);
+                              max_topk, block_idx, block_cnt, s.hkv, s.max_pages, s.bs, s.rows,
+                              err);
 }
 
 }  // namespace resa

@@ -45,9 +45,12 @@
  *   sets RESA_DEVERR_TIMEOUT.  The outputs of a call that timed out are
  *   undefined, and its workspace may hold words of that call: zero it again
  *   with resa_workspace_init before the next call.
- * Supported shapes.  head_dim in {64, 128}; block_size 16; group size
+ * Supported shapes.  head_dim in {64, 128}; block_size in {16, 32, 64}
+ *   (the b of the memory model, ReSA summary §3.4.3, Eq. 6); group size
  *   g = Hq / Hkv in 1 .. 16; Hkv <= 8.  Other shapes return
- *   RESA_ERR_UNSUPPORTED.
+ *   RESA_ERR_UNSUPPORTED.  The one-launch decode step is built for
+ *   block_size 16; other block sizes run it as three launches
+ *   (resa_decode_step_launches).
  */
 #ifndef RESA_H_
 #define RESA_H_

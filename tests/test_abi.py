@@ -84,7 +84,8 @@ def test_host_validation_without_gpu(lib):
     assert _call_select(cfg, _cache(), q=None) == 1                        # NULL q
     assert _call_select(R.make_config(4, 3, 64, 16), _cache()) == 2        # Hq % Hkv
     assert _call_select(R.make_config(4, 2, 96, 16), _cache()) == 4        # head_dim 96
-    assert _call_select(R.make_config(4, 2, 64, 32), _cache()) == 4        # block size 32
+    assert _call_select(R.make_config(4, 2, 64, 8), _cache()) == 4         # block size 8
+    assert _call_select(R.make_config(4, 2, 64, 48), _cache()) == 4        # block size 48
     assert _call_select(R.make_config(68, 2, 64, 16), _cache()) == 4       # group 34 > 16
     assert _call_select(R.make_config(4, 2, 64, 16, -1.0), _cache()) == 3  # negative scale
     assert _call_select(cfg, _cache(batch=0)) == 2
