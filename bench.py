@@ -73,6 +73,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the dense baseline and the further workloads")
     ap.add_argument("--breakdown-reps", type=int, default=5)
+    ap.add_argument("--sweep-block-sizes", default="16,32,64",
+                    help="block sizes b of --sweep (comma-separated)")
     ap.add_argument("--sweep", action="store_true",
                     help="time the decode step over top-k fractions and the rectification over "
                          "chunk lengths f, and compare the per-token cost with Eq. 6 (prints one "
@@ -136,8 +138,8 @@ def workload_lengths(wl, seed):
 class Schedule:
     """Sequence lengths and top-k per global step (decode steps and rectifications)."""
 
-    def __init__(self, ctx, f, cycles):
-        self.ctx, self.f, self.cycles = ctx, f, cycles
+    def __init__(self, ctx, f, cycles, bs=16):
+        self.ctx, self.f, self.cycles, self.bs = ctx, f, cycles, bs
         self.B = len(ctx)
         self.Bpad = (self.B + 3) // 4 * 4  # 16-byte aligned rows
 
@@ -148,14 +150,14 @@ class Schedule:
         return [L0 + (c + 1) * self.f for L0 in self.ctx]
 
     def max_topk(self):
-        return max(topk_rule(L0 + self.cycles * self.f) for L0 in self.ctx)
+        return max(topk_rule(L0 + self.cycles * self.f, self.bs) for L0 in self.ctx)
 
     def total_tokens(self):
         return max(self.ctx) + self.cycles * self.f
 
 
 class GpuWorkload:
-    def __init__(self, wl, cycles, seed, device):
+    def __init__(self, wl, cycles, seed, device, bs=16):
         import torch
         from block_sparse_long_resa_b200 import inputs
         from block_sparse_long_resa_b200 import resa as R
@@ -163,14 +165,15 @@ class GpuWorkload:
         self.R = R
         B, hq, hkv, d, f, nl = wl["batch"], wl["hq"], wl["hkv"], wl["d"], wl["f"], wl["layers"]
         self.B, self.hq, self.hkv, self.d, self.f, self.layers = B, hq, hkv, d, f, nl
+        self.bs = bs
         ctx = workload_lengths(wl, seed)
-        self.sched = Schedule(ctx, f, cycles)
-        self.cfg = R.make_config(hq, hkv, d, 16)
+        self.sched = Schedule(ctx, f, cycles, bs)
+        self.cfg = R.make_config(hq, hkv, d, bs)
         reserve = cycles * f + 16
         # one paged cache per layer (K, V, descriptors); the page table is shared
         self.k, self.v, self.desc, self.k_scale = [], [], [], []
         for layer in range(nl):
-            p = inputs.make_decode_problem(seed + 1000 * layer, B, hq, hkv, d, 16, ctx,
+            p = inputs.make_decode_problem(seed + 1000 * layer, B, hq, hkv, d, bs, ctx,
                                            reserve_tokens=reserve, paged=wl["paged"],
                                            device=device, topk=[1] * B)
             self.k.append(p.k_cache)
@@ -196,7 +199,7 @@ class GpuWorkload:
             for s in range(f - 1):
                 Ls = self.sched.decode_L(c, s)
                 sl[c * f + s, :B] = torch.tensor(Ls)
-                tk[c * f + s, :B] = torch.tensor([topk_rule(x) for x in Ls])
+                tk[c * f + s, :B] = torch.tensor([topk_rule(x, bs) for x in Ls])
             sl[c * f + f - 1, :B] = torch.tensor(self.sched.rect_L(c))
         self.seq_len = sl.to(device)
         self.topk = tk.to(device)
@@ -260,14 +263,15 @@ class GpuWorkload:
     def decode_kernel_bytes(self, Ls):
         """q + K/V of the selected blocks and the current block + fp32 output."""
         B, hq, hkv, d = self.B, self.hq, self.hkv, self.d
-        kv = sum(hkv * (min(topk_rule(L), (L - 1) // 16) + 1) * 16 * d * 2 * 2 for L in Ls)
+        bs = self.bs
+        kv = sum(hkv * (min(topk_rule(L, bs), (L - 1) // bs) + 1) * bs * d * 2 * 2 for L in Ls)
         return B * hq * d * 2 + kv + B * hq * d * 4
 
     def step_bytes(self, Ls):
         """One sparse decode step of one layer: q + descriptors of the complete
         blocks + selected K/V + output (the per-unit figure of the design notes)."""
         hkv, d = self.hkv, self.d
-        desc = sum(((L - 1) // 16) * hkv * 2 * d * 2 for L in Ls)
+        desc = sum(((L - 1) // self.bs) * hkv * 2 * d * 2 for L in Ls)
         return self.decode_kernel_bytes(Ls) + desc
 
     def rectify_bytes_flops(self, Ls):
@@ -598,6 +602,12 @@ def run_resa(args):
             "hbm_gbs": rb / (bd["rectify_us"] * 1e-6) / 1e9}
     rect["frac_of_bf16_peak"] = rect["tflops"] / bf16_peak
     rect["frac_of_hbm_peak"] = rect["hbm_gbs"] / hbm_peak
+    # descriptor build: every key read once, every descriptor written once
+    build_bytes = sum(L * w.hkv * w.d * 2 + -(-L // w.bs) * w.hkv * 2 * w.d * 2
+                      for L in last_dec_L)
+    build = {"us_per_layer": bd["build_descriptors_us"],
+             "hbm_gbs": build_bytes / (bd["build_descriptors_us"] * 1e-6) / 1e9}
+    build["frac_of_hbm_peak"] = build["hbm_gbs"] / hbm_peak
 
     dense = extra = None
     if not args.no_extra:
@@ -630,6 +640,7 @@ def run_resa(args):
         "step_roofline": {"algorithmic_bytes_per_step": cyc_bytes / K, "achieved": step_gbs,
                           "peak": hbm_peak, "unit": "GB/s", "frac": step_gbs / hbm_peak},
         "rectify": rect,
+        "build_descriptors": build,
         "kernel_breakdown_us": bd,
         "decode_step_path": "fused (1 launch)" if fused else "3 launches",
         "sparse_vs_dense_step_speedup": bd["dense_decode_us"] / bd["decode_step_us"],
@@ -700,6 +711,9 @@ def kernel_breakdown(w, stream, device, reps):
     res["dense_decode_us"] = timed(lambda: [R.resa_dense_decode(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
         w.out[w.f - 2, l], None, w.ws) for l in range(n)], n)
+    # full descriptor rebuild of every block (idempotent on the same keys)
+    res["build_descriptors_us"] = timed(lambda: [R.resa_build_descriptors(
+        w.cfg, w.cache(l, row), None, w.ws) for l in range(n)], n)
     res["rectify_us"] = timed(lambda: [R.resa_rectify_attention(
         w.cfg, w.cache(l, rrow), w.f, w.qc[c, l], w.kc[c, l], w.vc[c, l], w.rout[l], None, w.ws)
         for l in range(n)], n)
@@ -960,18 +974,14 @@ SWEEP_FRACS = (1 / 64, 1 / 32, 1 / 16, 1 / 10, 1 / 8, 1 / 4, 1 / 2, 1.0)
 SWEEP_CHUNKS = (8, 16, 32, 64)
 
 
-def run_sweep(args):
-    """Per-token cost of a ReSA cycle over (selected fraction s, rectification
-    period f) on the workload's layers: t_token = ((f-1) t_step(s) + t_rect(f)) / f,
-    next to the pages' memory model (ReSA summary §3.3, Eq. 6): bytes per token
-    relative to dense decoding = 1/b (block descriptors) + s (selected K/V)
-    + 1/f (one dense pass over the cache every f tokens)."""
+def sweep_block_size(args, bs):
+    """Decode step over the selected fractions and rectification over the
+    chunk lengths at one block size b; see run_sweep."""
     import torch
     from block_sparse_long_resa_b200 import resa as R
     device = torch.device("cuda", 0)
-    torch.cuda.set_device(device)
     wl = WORKLOADS[args.workload]
-    w = GpuWorkload(wl, 1, args.seed, device)
+    w = GpuWorkload(wl, 1, args.seed, device, bs=bs)
     stream = torch.cuda.Stream(device)
     n, B = w.layers, w.B
     row = w.f - 2  # a decode step of cycle 0
@@ -984,7 +994,7 @@ def run_sweep(args):
                                None, w.idx[layer], w.cnt[layer], w.ws)
     torch.cuda.synchronize(device)
     Ls = w.sched.decode_L(0, w.f - 2)
-    M = [(L - 1) // 16 for L in Ls]
+    M = [(L - 1) // bs for L in Ls]
     rounds = max(1, -(-28 // n))
 
     def timed(enqueue, calls, reps=5):
@@ -1006,6 +1016,7 @@ def run_sweep(args):
 
     steps = []
     for frac in SWEEP_FRACS:
+        # at least 16 blocks, as the top-k rule of the workloads
         k = [min(m, max(16, int(frac * m + 0.5))) for m in M]
         kmax = max(k)
         tk = torch.zeros(w.sched.Bpad, dtype=torch.int32, device=device)
@@ -1048,11 +1059,27 @@ def run_sweep(args):
             t_tok = ((f - 1) * st["us_per_layer"] + rc["us_per_layer"]) / f
             table.append({"s": st["s"], "f": f, "us_per_token_layer": t_tok,
                           "measured_vs_dense": t_tok / t_dense,
-                          "eq6_bytes_vs_dense": 1 / 16 + st["s"] + 1 / f})
-    print(json.dumps({"sweep": args.workload, "layers": n, "context": Ls,
-                      "dense_step_us_per_layer": t_dense, "decode_steps": steps,
-                      "rectification": rects, "per_token": table,
-                      "device_error_word": code}), flush=True)
+                          "eq6_bytes_vs_dense": 1 / bs + st["s"] + 1 / f})
+    res = {"b": bs, "context": Ls, "dense_step_us_per_layer": t_dense, "decode_steps": steps,
+           "rectification": rects, "per_token": table, "device_error_word": code}
+    del w, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_sweep(args):
+    """Per-token cost of a ReSA cycle over (block size b, selected fraction s,
+    rectification period f) on the workload's layers:
+    t_token = ((f-1) t_step(s) + t_rect(f)) / f, next to the pages' memory
+    model (ReSA summary §3.3, Eq. 6): bytes per token relative to dense
+    decoding = 1/b (block descriptors) + s (selected K/V) + 1/f (one dense
+    pass over the cache every f tokens)."""
+    import torch
+    torch.cuda.set_device(torch.device("cuda", 0))
+    sizes = [int(x) for x in args.sweep_block_sizes.split(",")]
+    out = [sweep_block_size(args, bs) for bs in sizes]
+    print(json.dumps({"sweep": args.workload, "layers": WORKLOADS[args.workload]["layers"],
+                      "block_sizes": out}), flush=True)
     return 0
 
 

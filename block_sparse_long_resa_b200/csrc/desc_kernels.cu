@@ -65,7 +65,7 @@ constexpr int kBuildPagesPerCta = 16;
 
 // grid (ceil(max_pages / kBuildPagesPerCta), batch), block kBuildThreads.
 // Rebuilds blocks [first, ceil(L / b)) of each sequence.
-__global__ void __launch_bounds__(kBuildThreads)
+__global__ void __launch_bounds__(kBuildThreads, 2)  // two CTAs an SM: twice the loads in flight
     build_desc_kernel(const uint4 *__restrict__ K, uint4 *__restrict__ desc,
                       const int32_t *__restrict__ page_table, const int32_t *__restrict__ seq_len,
                       const int32_t *__restrict__ first_block, int hkv, int d, int max_pages,

@@ -25,14 +25,16 @@
 //   warps 4-11  softmax, one thread per query row (TMEM lane): tcgen05.ld of
 //               the S row, causal mask (skipped for interior tiles), base-2
 //               online softmax with lazy O rescaling (only when the row
-//               maximum grows by more than 8), P written to shared memory as
-//               fp16 in the canonical K-major swizzled layout.  With E the
+//               maximum grows by more than 8), P written as fp16 pairs into
+//               tensor memory over the tile's S (tcgen05.st), where the
+//               P.V MMA reads its A operand.  With E the
 //               largest tile exponent seen so far, a tile's P is multiplied
 //               by 2^(e - E) and O is rescaled whenever E grows, so the TMEM
 //               accumulator holds 2^-E times the true sum; the epilogue
 //               multiplies by 2^E.
-// Three K/V stages are in flight (released per stage by the P.V commit); the
-// P tile is single-buffered, written once the previous P.V has completed.
+// Three K/V stages are in flight (released per stage by the P.V commit).  P
+// shares the double-buffered S columns, so writing it waits for nothing; O is
+// rescaled only after the previous P.V has completed.
 // P is fp16 (11-bit mantissa), so the P.V product keeps the weights' precision
 // without a second MMA.  With several splits the grid is launched
 // cooperatively; after a bounded grid barrier every CTA merges an equal share
@@ -78,12 +80,11 @@ struct TcLayout {
     static constexpr int kQHalf = 128 * 128;
     static constexpr int kKV = kKeys * D * 2;      // K or V tile, [half][64 keys][128 B]
     static constexpr int kKVHalf = kKeys * 128;
-    static constexpr int kP = 128 * kKeys * 2;     // P of one M tile, [128 rows][128 B]
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = kQOff + 2 * kQTile;
-    static constexpr int kPOff = kKVOff + kStages * 2 * kKV;
-    static constexpr int kBytes = kPOff + 2 * kP + 1024;  // one P buffer per M tile
-    // TMEM columns: O[mt] at mt*D, S[buf][mt] at 2*D + (2*buf + mt)*64.
+    static constexpr int kBytes = kKVOff + kStages * 2 * kKV + 1024;
+    // TMEM columns: O[mt] at mt*D, S[buf][mt] at 2*D + (2*buf + mt)*64; the
+    // tile's P (fp16 pairs) overwrites the first 32 columns of its S.
     static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -159,7 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     uint8_t *q_s = smem + LY::kQOff;
     uint8_t *kv_s = smem + LY::kKVOff;
-    uint8_t *p_s = smem + LY::kPOff;
 
     if (threadIdx.x == 0) {
         mbar_init(&q_ready, kSmThreads);
@@ -289,12 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t vt = smem_u32(kv_s + (size_t)s * 2 * LY::kKV + LY::kKV);
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
-                    const uint32_t pt = smem_u32(p_s + (size_t)mt * LY::kP);
+                    // P of this tile sits in tensor memory over its S
+                    const uint32_t pt = tmem + 2 * D + (2 * (i & 1) + mt) * kKeys;
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk) {
-                        const uint64_t a = tc::smem_desc(pt + kk * 32, 16, 1024);
                         const uint64_t bd = tc::smem_desc(vt + kk * 16 * 128, LY::kKVHalf, 1024);
-                        tc::mma_f16_ss(tmem + mt * D, a, bd, idesc_pv,
+                        tc::mma_f16_ts(tmem + mt * D, pt + kk * 8, bd, idesc_pv,
                                        (i > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
@@ -474,7 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             l += psum;
-            // The single P tile and O are free once the P.V of tile i-1 completed.
+            // P goes over this tile's S (already read; the P.V that last read
+            // this slot, of tile i-2, came before this tile's S in the MMA
+            // order), asynchronously while O waits for the P.V of tile i-1.
+            const uint32_t pcol = tmem + lane_base + 2 * D + (2 * buf + mt) * kKeys;
+            tc::tmem_st32(pcol, pw);
             if (i > 0) {
                 ok = mbar_wait_bounded(&pv_done, (i - 1) & 1);
                 ok = __all_sync(0xffffffffu, ok);
@@ -493,15 +497,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha_o);
                         tc::tmem_st32(ocol, ov);
                     }
-                    tc::tmem_wait_st();
                 }
             }
-            uint8_t *prow = p_s + (size_t)mt * LY::kP;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(prow + swz128(r, c)) =
-                    make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-            fence_proxy_async_smem();
+            tc::tmem_wait_st();
             tc::fence_before_sync();
             mbar_arrive(&p_full);
         }
