@@ -220,9 +220,10 @@ class GpuWorkload:
         self.kc = torch.randn(cycles, nl, B, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
         self.vc = torch.randn(cycles, nl, B, f, hkv, d, generator=g, device=device).to(torch.bfloat16)
         # outputs: one slot per (decode step of the cycle, layer), so that every
-        # step's result survives the cycle and can be read back
-        self.out = torch.empty(f - 1, nl, B, hq, d, device=device)
-        self.rout = torch.empty(nl, B, f, hq, d, device=device)
+        # step's result survives the cycle and can be read back; two sets, used
+        # by alternate cycles, so that one cycle's read-back overlaps the next
+        self.out = torch.empty(2, f - 1, nl, B, hq, d, device=device)
+        self.rout = torch.empty(2, nl, B, f, hq, d, device=device)
         # separate allocations keep every layer's selection buffers 16-byte aligned
         self.idx = [torch.empty(B, hkv, self.max_topk + 1, dtype=torch.int32, device=device)
                     for _ in range(nl)]
@@ -245,12 +246,12 @@ class GpuWorkload:
             for layer in range(self.layers):
                 R.resa_decode_step(self.cfg, self.cache(layer, row), self.q[c, s, layer],
                                    self.kn[c, s, layer], self.vn[c, s, layer], self.topk_ptr(row),
-                                   self.max_topk, self.out[s, layer], None, self.idx[layer],
+                                   self.max_topk, self.out[c % 2, s, layer], None, self.idx[layer],
                                    self.cnt[layer], self.ws)
         row = c * f + f - 1
         for layer in range(self.layers):
             R.resa_rectify_attention(self.cfg, self.cache(layer, row), f, self.qc[c, layer],
-                                     self.kc[c, layer], self.vc[c, layer], self.rout[layer], None,
+                                     self.kc[c, layer], self.vc[c, layer], self.rout[c % 2, layer], None,
                                      self.ws)
 
     def launches_per_cycle(self):
@@ -542,27 +543,50 @@ def run_resa(args):
         host_out = [torch.empty_like(w.out, device="cpu").pin_memory(),
                     torch.empty_like(w.rout, device="cpu").pin_memory()]
         h2d = sum(t[0].numel() * t.element_size() for t in host_in)
-        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        d2h = sum(t[0].numel() * t.element_size() for t in host_out)
+        # Inputs go up on one copy stream, outputs come back on another, and the
+        # cycles run on the compute stream: cycle c waits for its inputs, and
+        # for the read-back of cycle c - 2 (the output set it reuses).
+        up = torch.cuda.Stream(device)
+        down = torch.cuda.Stream(device)
+        n_t = cycles - W
+        ev_in = [torch.cuda.Event() for _ in range(n_t)]
+        ev_run = [torch.cuda.Event() for _ in range(n_t)]
+        ev_out = [torch.cuda.Event() for _ in range(n_t)]
         barrier(dist, device)
         torch.cuda.synchronize(device)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
+        e0.record(stream)
+        up.wait_stream(stream)
+        down.wait_stream(stream)
+        with torch.cuda.stream(up):
             for i, c in enumerate(range(W, cycles)):
                 for hsrc, ddst in zip(host_in, dev_in):
                     ddst[c].copy_(hsrc[i], non_blocking=True)
+                ev_in[i].record(up)
+        for i, c in enumerate(range(W, cycles)):
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])
+            with torch.cuda.stream(stream):
                 graphs[c].replay()
-                host_out[0].copy_(w.out, non_blocking=True)
-                host_out[1].copy_(w.rout, non_blocking=True)
-            e1.record(stream)
+            ev_run[i].record(stream)
+            down.wait_event(ev_run[i])
+            with torch.cuda.stream(down):
+                host_out[0][c % 2].copy_(w.out[c % 2], non_blocking=True)
+                host_out[1][c % 2].copy_(w.rout[c % 2], non_blocking=True)
+            ev_out[i].record(down)
+        stream.wait_event(ev_out[n_t - 1])
+        e1.record(stream)
         torch.cuda.synchronize(device)
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / K,
                "copies": "per cycle: q/k/v of every decode step and the rectification chunk "
                          "in; every decode step's output (f-1 per layer) and the rectified "
-                         "rows out"}
+                         "rows out; copies in and out run on two copy streams, overlapped "
+                         "with the neighbouring cycles' compute"}
 
     code = w.R.resa_check_device_status(w.ws, raise_on_error=False)
 
@@ -696,7 +720,7 @@ def kernel_breakdown(w, stream, device, reps):
     res = {}
     res["sparse_decode_us"] = timed(lambda: [R.resa_sparse_decode(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.idx[l], w.cnt[l], w.max_topk,
-        w.out[w.f - 2, l], None, w.ws) for l in range(n)], n)
+        w.out[0, w.f - 2, l], None, w.ws) for l in range(n)], n)
     scratch_idx = [torch.empty_like(t) for t in w.idx]
     scratch_cnt = [torch.empty_like(t) for t in w.cnt]
     res["select_blocks_us"] = timed(lambda: [R.resa_select_blocks(
@@ -707,17 +731,17 @@ def kernel_breakdown(w, stream, device, reps):
         for l in range(n)], n)
     res["decode_step_us"] = timed(lambda: [R.resa_decode_step(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
-        w.topk_ptr(row), w.max_topk, w.out[w.f - 2, l], None, w.idx[l], w.cnt[l], w.ws)
+        w.topk_ptr(row), w.max_topk, w.out[0, w.f - 2, l], None, w.idx[l], w.cnt[l], w.ws)
         for l in range(n)], n)
     # dense decoding of the same step (append + attention over every position, Eq. 1)
     res["dense_decode_us"] = timed(lambda: [R.resa_dense_decode(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
-        w.out[w.f - 2, l], None, w.ws) for l in range(n)], n)
+        w.out[0, w.f - 2, l], None, w.ws) for l in range(n)], n)
     # full descriptor rebuild of every block (idempotent on the same keys)
     res["build_descriptors_us"] = timed(lambda: [R.resa_build_descriptors(
         w.cfg, w.cache(l, row), None, w.ws) for l in range(n)], n)
     res["rectify_us"] = timed(lambda: [R.resa_rectify_attention(
-        w.cfg, w.cache(l, rrow), w.f, w.qc[c, l], w.kc[c, l], w.vc[c, l], w.rout[l], None, w.ws)
+        w.cfg, w.cache(l, rrow), w.f, w.qc[c, l], w.kc[c, l], w.vc[c, l], w.rout[0, l], None, w.ws)
         for l in range(n)], n)
     return res
 
@@ -992,7 +1016,7 @@ def sweep_block_size(args, bs):
     for st in range(row):
         for layer in range(n):
             R.resa_decode_step(w.cfg, w.cache(layer, st), w.q[0, st, layer], w.kn[0, st, layer],
-                               w.vn[0, st, layer], w.topk_ptr(st), w.max_topk, w.out[st, layer],
+                               w.vn[0, st, layer], w.topk_ptr(st), w.max_topk, w.out[0, st, layer],
                                None, w.idx[layer], w.cnt[layer], w.ws)
     torch.cuda.synchronize(device)
     Ls = w.sched.decode_L(0, w.f - 2)
@@ -1027,14 +1051,14 @@ def sweep_block_size(args, bs):
         cnt = [torch.empty(B, w.hkv, dtype=torch.int32, device=device) for _ in range(n)]
         us = timed(lambda: [R.resa_decode_step(
             w.cfg, w.cache(l, row), w.q[0, row, l], w.kn[0, row, l], w.vn[0, row, l], tk, kmax,
-            w.out[row, l], None, idx[l], cnt[l], w.ws) for l in range(n)], n)
+            w.out[0, row, l], None, idx[l], cnt[l], w.ws) for l in range(n)], n)
         steps.append({"s": frac, "topk": k[0] if B == 1 else k, "us_per_layer": us,
                       "launches_per_step": R.resa_decode_step_launches(w.cfg, B, w.max_pages,
                                                                        w.num_pages)})
         del idx, cnt
     t_dense = timed(lambda: [R.resa_dense_decode(
         w.cfg, w.cache(l, row), w.q[0, row, l], w.kn[0, row, l], w.vn[0, row, l],
-        w.out[row, l], None, w.ws) for l in range(n)], n)
+        w.out[0, row, l], None, w.ws) for l in range(n)], n)
     fmax = max(SWEEP_CHUNKS)
     ws = torch.empty(R.resa_workspace_size(w.cfg, B, w.max_pages, fmax), dtype=torch.uint8,
                      device=device)
