@@ -461,6 +461,32 @@ def test_full_size_256k_layer(cuda_device):
     np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
 
 
+def test_full_size_dense_decode_256k(cuda_device):
+    """Dense decoding of one 256K layer (28 q / 4 kv heads, d 128) in the
+    launch configuration of the bench's dense baseline; the oracle computes
+    every output."""
+    p = inputs.make_decode_problem(9, 1, 28, 4, 128, 16, [262144], device=cuda_device)
+    cfg = cfg_of(p)
+    lc = LayerCache(k=p.k_cache, v=p.v_cache,
+                    desc=torch.zeros(p.num_pages, 4, 2, 128, dtype=torch.bfloat16,
+                                     device=cuda_device),
+                    page_table=p.page_table, seq_len=p.ctx_len.clone())
+    ws = workspace(cfg, 1, lc.max_pages, 16, cuda_device)
+    R.resa_build_descriptors(cfg, lc.struct(), None, ws)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L)
+    out = torch.empty(1, 28, 128, device=cuda_device)
+    lse = torch.empty(1, 28, device=cuda_device)
+    R.resa_dense_decode(cfg, lc.struct(), p.q, p.k_new, p.v_new, out, lse, ws)
+    assert_no_device_error(ws)
+    cpu = lambda t: t.cpu()
+    o = O.OracleCache(cpu(p.k_cache), cpu(p.v_cache), cpu(p.page_table), 28, 4, 128, 16)
+    o.append(cpu(p.k_new), cpu(p.v_new), cpu(L))
+    ref, ref_lse = o.dense_attention(cpu(p.q), cpu(L))
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+
+
 def test_full_size_rectification_sampled_rows(cuda_device):
     """Rectification at the decode-loop workload's size (batch 4, 65536-token
     cache, f = 32, 28 q / 4 kv heads): every output row computed, sampled rows

@@ -54,12 +54,12 @@ def gpu_mixed_step(cfg, lc, ws, dev, dec, rect, f, q, kn, vn, topk, max_topk, qc
     return res
 
 
-def check_decode(o, res, dec, q, kn, vn, topk, L, max_topk):
+def check_decode(o, res, dec, q, kn, vn, topk, L, max_topk, bs=16):
     out, lse, idx, cnt = res["dec"]
     view = o.rows_view(dec)
     r = view.decode_step(q, kn, vn, topk, L, max_topk)
     gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
-    same = check_block_sets(gidx, gcnt, r["block_idx"], r["block_cnt"], r["scores"], topk, L, 16)
+    same = check_block_sets(gidx, gcnt, r["block_idx"], r["block_cnt"], r["scores"], topk, L, bs)
     ref, ref_lse = (r["out"], r["lse"]) if same else view.sparse_attention(q, gidx, gcnt, L)
     np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
@@ -80,11 +80,15 @@ WIDE = dict(seed=22, batch=24, num_q_heads=HQ, num_kv_heads=HKV, head_dim=D, blo
             paged=True)
 
 
+MIXED64 = dict(MIXED, seed=26, block_size=64)
+
+
 @pytest.mark.parametrize("case,dec,rect", [
     (MIXED, [0, 2, 4, 5], [1, 3]),
     (MIXED, [5, 1, 3], [4, 0, 2]),
     (WIDE, [i for i in range(24) if i % 6 != 2], [2, 8, 14, 20]),
-], ids=["fused", "permuted", "three-launch"])
+    (MIXED64, [3, 0, 5], [2, 1, 4]),
+], ids=["fused", "permuted", "three-launch", "block64"])
 def test_mixed_phase_step(cuda_device, case, dec, rect):
     p = make(case)
     f = 32
@@ -93,7 +97,7 @@ def test_mixed_phase_step(cuda_device, case, dec, rect):
     lc.seq_len.copy_(L.to(cuda_device))
     max_topk = int(p.topk[dec].max())
     qc, kc, vc = inputs.make_rectify_chunk(23, len(rect), f, HQ, HKV, D)
-    if len(dec) * HKV <= 74:
+    if len(dec) * HKV <= 74 and p.block_size == 16:
         assert R.resa_decode_step_launches(cfg, len(dec), lc.max_pages, lc.k.shape[0]) == 1
     else:
         assert R.resa_decode_step_launches(cfg, len(dec), lc.max_pages, lc.k.shape[0]) == 3
@@ -104,7 +108,7 @@ def test_mixed_phase_step(cuda_device, case, dec, rect):
     o = oracle_of(p)
     o.build_descriptors(p.ctx_len)
     check_decode(o, res, dec, p.q[dec], p.k_new[dec], p.v_new[dec], p.topk[dec], L[dec],
-                 max_topk)
+                 max_topk, p.block_size)
     check_rect(o, res, rect, qc, kc, vc, L[rect], f)
     np.testing.assert_array_equal(bits_of(lc.k), o.K)
     np.testing.assert_array_equal(bits_of(lc.v), o.V)
@@ -172,3 +176,28 @@ def test_row_outside_table_is_reported(cuda_device):
     o2.build_descriptors(p.ctx_len)
     o2.rows_view([0]).append(p.k_new[:1], p.v_new[:1], L[:1])
     np.testing.assert_array_equal(bits_of(lc.k), o2.K)
+
+
+def test_dense_decode_on_mapped_rows(cuda_device):
+    """Dense decoding of a subset of the table's rows, in a permuted order."""
+    p = make(MIXED)
+    cfg, lc, ws = setup_layer(p, cuda_device)
+    L = p.ctx_len + 1
+    lc.seq_len.copy_(L.to(cuda_device))
+    dec = [4, 1, 5]
+    out = torch.empty(3, HQ, D, device=cuda_device)
+    lse = torch.empty(3, HQ, device=cuda_device)
+    dev = lambda t: t.to(cuda_device)
+    rows = i32(dec, cuda_device)  # kept alive until the call has run
+    R.resa_dense_decode(cfg, lc.struct(rows=rows), dev(p.q[dec]), dev(p.k_new[dec]),
+                        dev(p.v_new[dec]), out, lse, ws)
+    assert_no_device_error(ws)
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    view = o.rows_view(dec)
+    view.append(p.k_new[dec], p.v_new[dec], L[dec])
+    ref, ref_lse = view.dense_attention(p.q[dec], L[dec])
+    np.testing.assert_array_equal(bits_of(lc.k), o.K)
+    np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)

@@ -49,13 +49,16 @@ def _oracle_out(p, lc, idx, cnt):
     dict(seed=3, B=5, hq=28, hkv=4, d=128, ctx=[1, 15, 16, 300, 5003], topk=[4, 16, 16, 7, 500],
          paged=True),
     dict(seed=4, B=3, hq=8, hkv=1, d=64, ctx=[33, 257, 1111], topk=[100, 3, 60], paged=True),
-], ids=["qwen32k", "ragged", "d64"])
+    dict(seed=6, B=3, hq=28, hkv=4, d=128, ctx=[100, 2000, 7000], topk=[2, 20, 50], paged=True,
+         bs=32),
+], ids=["qwen32k", "ragged", "d64", "block32"])
 def test_noalloc_matches_workspace_path_and_oracle_twice(case):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     dev = torch.device("cuda:0")
-    p = inputs.make_decode_problem(case["seed"], case["B"], case["hq"], case["hkv"], case["d"], 16,
-                                   case["ctx"], paged=case["paged"], topk=case["topk"])
+    p = inputs.make_decode_problem(case["seed"], case["B"], case["hq"], case["hkv"], case["d"],
+                                   case.get("bs", 16), case["ctx"], paged=case["paged"],
+                                   topk=case["topk"])
     cfg, lc, ws, idx, cnt, max_topk = _select(p, dev)
     q = p.q.to(dev)
     shape = (p.batch, p.num_q_heads, p.head_dim)
