@@ -558,22 +558,6 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         }
         d1 = (uint32_t)s_v[kVD1];
         above = s_v[kVAB];
-        if (mode == kModeMid) {
-            // The blocks above the boundary digit are selected whatever the
-            // boundary candidates settle: their K/V is pulled into L2 (each
-            // CTA its own scored range) while the threshold and the slices are
-            // worked out, so HBM streams the selection from here on.
-            const uint32_t hi1 = (d1 << 16) | 0xffffu;
-            #pragma unroll 1
-            for (int i = tid; i < nmine; i += kThreadsAll) {
-                const int pg = pages[i];
-                if (keys[i] > hi1 && pg >= 0 && pg < a.num_pages) {
-                    const size_t t = ((size_t)pg * hkv + h) * SM::kTileBytes;
-                    prefetch_l2(a.k_cache + t, SM::kTileBytes);
-                    prefetch_l2(a.v_cache + t, SM::kTileBytes);
-                }
-            }
-        }
     }
     // Work split: the unit's ordered work list is the selected blocks in
     // ascending order, then the current block (W = keff + 1 items); CTA x
@@ -597,11 +581,28 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
         // d1 iff the key is above hi1, equal to d1 iff key - lo1 < 2^16.
         // (A ballot-per-key pass was bound by the quarter-rate vote and
         // population-count units.)
+        // The last warp meanwhile pulls into L2 the K/V of the blocks above
+        // the boundary digit in the CTA's own scored range: they are selected
+        // whatever the candidates settle, so HBM streams the selection from
+        // here on.  (Bulk prefetches queue on the copy unit; issued by every
+        // warp they would hold up the whole pass.)
         const uint32_t lo1 = d1 << 16, hi1 = lo1 | 0xffffu;
         uint32_t *seg = cand_s + warp * cap;
         int nseg = 0;
+        if (warp == kWarpsAll - 1) {
+            #pragma unroll 1
+            for (int i = lane; i < nmine; i += 32) {
+                const int pg = pages[i];
+                if (keys[i] > hi1 && pg >= 0 && pg < a.num_pages) {
+                    const size_t t = ((size_t)pg * hkv + h) * SM::kTileBytes;
+                    prefetch_l2(a.k_cache + t, SM::kTileBytes);
+                    prefetch_l2(a.v_cache + t, SM::kTileBytes);
+                }
+            }
+        }
+        constexpr int kPassThreads = (kWarpsAll - 1) * 32;
         #pragma unroll 1
-        for (int h0 = warp * 32; h0 < 2 * ngroups; h0 += kThreadsAll) {
+        for (int h0 = warp * 32; warp < kWarpsAll - 1 && h0 < 2 * ngroups; h0 += kPassThreads) {
             const int hg = h0 + lane;          // half-group: keys [16 hg, 16 hg + 16)
             const int q = hg >> 1;
             const int lim = M - hg * 16;       // keys of the half: min(16, lim)
