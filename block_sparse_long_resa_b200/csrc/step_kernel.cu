@@ -443,8 +443,9 @@ __global__ void __launch_bounds__(kThreadsAll, 1) decode_step_kernel(const StepA
     // The arrival's fence comes before the page-id copies are issued, so it
     // does not wait for them.
     if (G > 1 && need_hist && tid == 0) {
-        __threadfence();  // the CTA's key row and histogram atomics, ordered by the barrier above
-        atomicAdd(&ubar[0], 1ull);
+        // release: the CTA's key row and histogram atomics, ordered by the
+        // barrier above, are visible before the count
+        asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(&ubar[0]) : "memory");
     }
     // the page-id row is copied from the 16-byte boundary at or below its
     // start, the tail (inside the row) with 4-byte copies
