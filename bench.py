@@ -868,6 +868,7 @@ def workload_block(name, stream, device, seed, reps, hbm_peak):
            "cycle_us_per_layer": per_layer_cycle,
            "amortised_us_per_token_per_layer": per_layer_cycle / wl["f"],
            "tokens_per_s": wl["batch"] * wl["f"] / (cyc_us * 1e-6),
+           "kernel_breakdown_us": bd,
            "device_error_word": code}
     del graphs, w
     torch.cuda.empty_cache()
