@@ -38,6 +38,7 @@ namespace resa {
 namespace {
 
 constexpr int kScoreWarps = 16;                   // scoring warps per CTA (one CTA per SM)
+constexpr int kScoreChunk = 512;                  // pages a scoring CTA takes at most, batches
 constexpr int kScoreRingBytes = 192 * 1024;       // shared-memory ring budget per CTA
 constexpr int kScoreThreads = 32 * (kScoreWarps + 1);  // + the decode-token append warp
 constexpr int kHashSlots = 2048;  // per-CTA histogram aggregation table
@@ -691,10 +692,14 @@ cudaError_t launch_score_d(const Shape &s, void *desc, const int32_t *page_table
                            const int32_t *seq_len, const void *q, float *scores, uint32_t *hist,
                            uint32_t *hist_range, void *K, void *V, const void *k_new,
                            const void *v_new, uint32_t *err, cudaStream_t st) {
-    // One CTA per SM over all sequences, at least two pages per scoring warp.
+    // At least two pages per scoring warp; at least one CTA per SM over all
+    // sequences, and at least one CTA per kScoreChunk pages of the longest, so
+    // that a long sequence in a large batch is scored by proportionally more
+    // CTAs (the shorter ones' CTAs finish early and free their SMs).
     const int by_work = (s.max_pages + 2 * kScoreWarps - 1) / (2 * kScoreWarps);
     const int by_sm = s.batch < kNumSms ? kNumSms / s.batch : 1;
-    const int X = max(1, min(by_work, by_sm));
+    const int by_len = (s.max_pages + kScoreChunk - 1) / kScoreChunk;
+    const int X = max(1, min(by_work, max(by_sm, by_len)));
     dim3 grid(X, s.batch);
 #define RESA_SCORE_CASE(H)                                                                    \
     case H: {                                                                                 \
