@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       int num_pages, float scale_log2, float *__restrict__ part_o,
                       float *__restrict__ part_lse, uint32_t *__restrict__ tickets,
                       float *__restrict__ out, float *__restrict__ lse_out, const RowMap rm,
-                      uint32_t *err) {
+                      int coop, uint32_t *err) {
     using LY = TcLayout<D>;
     constexpr int kBPT = kKeys / BS;  // blocks per 64-key tile
     static_assert(kKeys % BS == 0 && kBPT <= 4, "a tile holds whole blocks");
@@ -561,27 +561,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tc::tmem_dealloc(tmem, LY::kTmemCols);
     if (S == 1) return;
 
-    // Every CTA of the (cooperatively launched, co-resident) grid has written
-    // its partials: bounded grid barrier, then each CTA merges its share of
-    // all rows.  tickets[0..1] hold the barrier's 64-bit (generation, arrivals) word.
+    // Every split's partials are written.  Within one wave (cooperative
+    // launch) a bounded grid barrier lets every CTA merge an equal share of
+    // all rows; tickets[0..1] hold the barrier's 64-bit (generation,
+    // arrivals) word.  Beyond one wave the last split of each (unit, row
+    // group) to arrive merges that group, counted by a ticket it resets.
     __threadfence();
     __syncthreads();
     __shared__ uint32_t sh_ok;
-    const uint32_t nctas = gridDim.x * gridDim.y * gridDim.z;
-    if (threadIdx.x == 0) sh_ok = grid_barrier_bounded(reinterpret_cast<unsigned long long *>(tickets), nctas) ? 1u : 0u;
-    __syncthreads();
-    if (!sh_ok) {
-        if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);
-        return;
+    int i0, i1, cap_rows;
+    if (coop) {
+        const uint32_t nctas = gridDim.x * gridDim.y * gridDim.z;
+        if (threadIdx.x == 0) sh_ok = grid_barrier_bounded(reinterpret_cast<unsigned long long *>(tickets), nctas) ? 1u : 0u;
+        __syncthreads();
+        if (!sh_ok) {
+            if (threadIdx.x == 0) set_error(err, RESA_DEVERR_TIMEOUT);
+            return;
+        }
+        __threadfence();
+        const int total = (int)gridDim.z * R;
+        const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+        cap_rows = (total + (int)nctas - 1) / (int)nctas;
+        i0 = cta * cap_rows;
+        i1 = min(total, i0 + cap_rows);
+    } else {
+        uint32_t *ticket = tickets + kRectTicketBase + (size_t)unit * kMaxRowTiles + group;
+        if (threadIdx.x == 0) sh_ok = atomicAdd(ticket, 1u) == (uint32_t)(S - 1) ? 1u : 0u;
+        __syncthreads();
+        if (!sh_ok) return;
+        __threadfence();
+        if (threadIdx.x == 0) *ticket = 0u;  // every split of the group has arrived
+        cap_rows = kRows;
+        i0 = unit * R + min(R, row0);
+        i1 = unit * R + min(R, row0 + kRows);
     }
-    __threadfence();
-    const int units = gridDim.z;
-    const int total = units * R;
-    const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-    const int per_cta = (total + nctas - 1) / nctas;
-    const int i0 = cta * per_cta, i1 = min(total, i0 + per_cta);
-    float *wts = reinterpret_cast<float *>(smem);  // [per_cta][S] merge weights
-    float *lse_s = wts + per_cta * S;              // [per_cta]
+    float *wts = reinterpret_cast<float *>(smem);  // [cap_rows][S] merge weights
+    float *lse_s = wts + cap_rows * S;             // [cap_rows]
     auto slot_row = [&](int item, int sp) -> size_t {
         const int u = item / R, rho = item % R;
         return (((size_t)u * G + rho / kRows) * S + sp) * kRows + rho % kRows;
@@ -641,9 +656,10 @@ cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *pa
     if (e != cudaSuccess) return e;
     const float scale_log2 = s.sm_scale * 1.4426950408889634f;
     dim3 grid(groups, splits, s.batch * s.hkv);
-    // With several splits the CTAs meet at a grid barrier before merging, so
-    // they must be co-resident: cooperative launch (one CTA per SM; the split
-    // count keeps the grid within the SM count).
+    // With several splits in one wave the CTAs meet at a grid barrier before
+    // merging, so they must be co-resident: cooperative launch (one CTA per
+    // SM).  A larger grid merges by per-group tickets instead.
+    const int coop = splits > 1 && (long long)groups * splits * s.batch * s.hkv <= kNumSms;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kThreads);
@@ -653,12 +669,12 @@ cudaError_t launch_tc(const Shape &s, const CUtensorMap *maps, const int32_t *pa
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = splits > 1 ? 1 : 0;
+    cfg.numAttrs = coop ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, rectify_tc_kernel<D, BS>, maps[0], maps[1], maps[2], maps[3],
                               maps[4], maps[5], maps[6], maps[7],
                               page_table, seq_len, f, (const uint16_t *)q_chunk, s.hkv, s.g,
                               s.max_pages, s.num_pages, scale_log2, part_o, part_lse, tickets, out,
-                              lse, s.rows, err);
+                              lse, s.rows, coop, err);
 }
 
 }  // namespace

@@ -130,7 +130,7 @@ resa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? RESA_OK : R
     } while (0)
 
 WsLayout layout_of(const Shape &s, int chunk) {
-    return ws_layout(s.hq, s.hkv, s.d, s.batch, s.max_pages, chunk);
+    return ws_layout(s.hq, s.hkv, s.d, s.bs, s.batch, s.max_pages, chunk);
 }
 
 
@@ -195,10 +195,10 @@ size_t resa_workspace_size(const resa_config_t *cfg, int32_t batch, int32_t max_
     Shape s{};
     if (check_config(cfg, &s) != RESA_OK || batch <= 0 || max_pages <= 0 || max_chunk < 0)
         return 0;
-    size_t best = ws_layout(s.hq, s.hkv, s.d, batch, max_pages, 0).total;
+    size_t best = ws_layout(s.hq, s.hkv, s.d, s.bs, batch, max_pages, 0).total;
     for (int f = 1; f <= max_chunk; ++f) {
         if (rect_row_groups(f, s.g) > kMaxRowTiles) break;
-        const size_t t = ws_layout(s.hq, s.hkv, s.d, batch, max_pages, f).total;
+        const size_t t = ws_layout(s.hq, s.hkv, s.d, s.bs, batch, max_pages, f).total;
         best = t > best ? t : best;
     }
     return best;

@@ -94,10 +94,17 @@ inline int rect_row_groups(int chunk, int group) {
     const int rows = chunk * group;
     return (rows + kRectRowsPerCta - 1) / kRectRowsPerCta;
 }
-// One CTA per SM over all (unit, row group) pairs.
-inline int rect_splits_for(int batch, int hkv, int groups) {
+// Key splits of a rectification: one CTA per SM over all (unit, row group)
+// pairs, and at least one split per kRectKeysPerSplit keys of the longest
+// sequence.  A grid within one wave merges its splits after a grid barrier
+// (cooperative launch); a larger one (long sequences in a large batch) lets
+// the last split of each (unit, row group) merge it.
+constexpr int kRectKeysPerSplit = 16384;
+inline int rect_splits_for(int batch, int hkv, int groups, long long max_keys) {
     const int units = batch * hkv * (groups > 0 ? groups : 1);
-    const int s = kNumSms / units;
+    int s = kNumSms / units;
+    const long long by_len = (max_keys + kRectKeysPerSplit - 1) / kRectKeysPerSplit;
+    if (by_len > s) s = (int)(by_len < 64 ? by_len : 64);
     return s < 1 ? 1 : (s > 64 ? 64 : s);
 }
 
@@ -108,6 +115,7 @@ inline int rect_splits_for(int batch, int hkv, int groups) {
 // rectification partials come last.
 // ---------------------------------------------------------------------------
 constexpr int kMaxRowTiles = 64;  // rectification row groups per (sequence, kv head)
+constexpr int kRectTicketBase = 16;  // u32 words before the split tickets (grid barrier word)
 
 // Byte offset, inside the 256-byte error header of the workspace, of the
 // decode kernel's grid barrier word (64-bit: generation, arrivals).
@@ -116,7 +124,7 @@ constexpr size_t kDecBarrierOffset = 32;
 struct WsLayout {
     size_t err;          // uint32 error word
     size_t dec_ticket;   // uint32 [B][Hkv]
-    size_t rect_ticket;  // uint32 [B][Hkv][kMaxRowTiles]
+    size_t rect_ticket;  // grid barrier word, then uint32 [B][Hkv][kMaxRowTiles] split tickets
     size_t hist;         // uint32 [B][Hkv][65536] score-key histogram (kept zero between calls)
     size_t hist_range;   // uint32 [B][Hkv][2] touched-bin range (kept zero between calls)
     size_t scores;       // f32 [B][Hkv][max_pages]
@@ -138,7 +146,7 @@ struct WsLayout {
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Layout for a call that rectifies chunks of `chunk` tokens (0: no rectification).
-inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int chunk) {
+inline WsLayout ws_layout(int hq, int hkv, int d, int bs, int batch, int max_pages, int chunk) {
     WsLayout w{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -149,11 +157,11 @@ inline WsLayout ws_layout(int hq, int hkv, int d, int batch, int max_pages, int 
     int g = hkv > 0 ? hq / hkv : 1;
     w.dec_splits = decode_max_splits(batch, hkv, max_pages);
     w.row_tiles = chunk > 0 ? rect_row_groups(chunk, g) : 0;
-    w.rect_splits = chunk > 0 ? rect_splits_for(batch, hkv, w.row_tiles) : 0;
+    w.rect_splits = chunk > 0 ? rect_splits_for(batch, hkv, w.row_tiles, (long long)max_pages * bs) : 0;
     size_t units = (size_t)batch * hkv;
     w.err = take(256);  // error word at 0, decode grid barrier at kDecBarrierOffset
     w.dec_ticket = take(units * 4);
-    w.rect_ticket = take(units * kMaxRowTiles * 4);
+    w.rect_ticket = take(kRectTicketBase * 4 + units * kMaxRowTiles * 4);
     w.hist = take(units * 65536 * 4);
     w.hist_range = take(units * 2 * 4);
     w.scores = take(units * max_pages * 4);

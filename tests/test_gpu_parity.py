@@ -487,6 +487,34 @@ def test_full_size_dense_decode_256k(cuda_device):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
 
 
+def test_rectification_beyond_one_wave(cuda_device):
+    """A batch whose (sequence, kv head) units and key splits exceed one wave
+    of CTAs (160 units, two splits for the longest sequences): each group's
+    last split merges it.  Sampled rows against the oracle; every touched
+    block's descriptor bit-exact; a second call reuses the reset tickets."""
+    B, f = 40, 32
+    ctx = [2000 + (i * 467) % 18000 for i in range(B)]
+    p = inputs.make_decode_problem(12, B, 4, 4, 128, 16, ctx, paged=True)
+    cfg, lc, ws = setup_layer(p, cuda_device, max_chunk=f)
+    L = p.ctx_len
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    rows = [0, 13, 31]
+    dev = lambda t: t.to(cuda_device)
+    for call in range(2):
+        qc, kc, vc = inputs.make_rectify_chunk(13 + call, B, f, 4, 4, 128)
+        out = torch.empty(B, f, 4, 128, device=cuda_device)
+        lse = torch.empty(B, f, 4, device=cuda_device)
+        R.resa_rectify_attention(cfg, lc.struct(), f, dev(qc), dev(kc), dev(vc), out, lse, ws)
+        assert_no_device_error(ws)
+        res = o.rectify_rows(qc, kc, vc, L, f, rows)
+        np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+        for r in rows:
+            ref, ref_lse = res[r]
+            np.testing.assert_allclose(out[:, r].cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+            np.testing.assert_allclose(lse[:, r].cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+
+
 def test_full_size_rectification_sampled_rows(cuda_device):
     """Rectification at the decode-loop workload's size (batch 4, 65536-token
     cache, f = 32, 28 q / 4 kv heads): every output row computed, sampled rows
