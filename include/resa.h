@@ -191,7 +191,10 @@ RESA_API resa_status_t resa_sparse_decode(const resa_config_t *cfg, const resa_c
  *      (position L-f+r) attends to positions 0 .. L-f+r.
  * out [batch][f][Hq][d] fp32, lse_opt (nullable) [batch][f][Hq] fp32.
  * f must be in 1 .. max_chunk of the workspace; f > L sets RESA_DEVERR_CHUNK
- * and the sequence is skipped. */
+ * and the sequence is skipped.  The keys of each (sequence, kv head) are split
+ * across CTAs (enough to fill the SMs, and at least one split per 16384 keys
+ * of the longest sequence); the splits' partial results live in the workspace
+ * and are merged in the same call.  Two launches. */
 RESA_API resa_status_t resa_rectify_attention(const resa_config_t *cfg, const resa_cache_t *cache,
                                      int32_t f, const void *q_chunk, const void *k_new,
                                      const void *v_new, float *out, float *lse_opt, void *ws,
@@ -202,7 +205,8 @@ RESA_API resa_status_t resa_rectify_attention(const resa_config_t *cfg, const re
  * and attend (as resa_sparse_decode).  seq_len must already count the decode
  * token.  block_idx_opt / block_cnt_opt (nullable) receive the selection in
  * the layout of resa_select_blocks; when NULL it lives in the workspace.
- * When batch * Hkv <= 74, g <= 8 and max_pages <= 65536 (and each of the
+ * When block_size is 16, batch * Hkv <= 74, g <= 8 and max_pages <= 65536
+ * (and each of the
  * G = 148 / (batch * Hkv) CTAs per (sequence, kv head) scores at most 1024
  * blocks) the whole step is one cooperative launch: the CTAs of a (sequence,
  * kv head) score their share of the descriptors, agree on the selection
