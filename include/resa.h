@@ -206,10 +206,9 @@ RESA_API resa_status_t resa_rectify_attention(const resa_config_t *cfg, const re
  * token.  block_idx_opt / block_cnt_opt (nullable) receive the selection in
  * the layout of resa_select_blocks; when NULL it lives in the workspace.
  * When block_size is 16, batch * Hkv <= 74, g <= 8 and max_pages <= 65536
- * (and each of the
- * G = 148 / (batch * Hkv) CTAs per (sequence, kv head) scores at most 1024
- * blocks) the whole step is one cooperative launch: the CTAs of a (sequence,
- * kv head) score their share of the descriptors, agree on the selection
+ * (and each of the G = 148 / (batch * Hkv) CTAs per (sequence, kv head)
+ * scores at most 1024 blocks) the whole step is one cooperative launch: the
+ * CTAs of a (sequence, kv head) score their share of the descriptors, agree on the selection
  * through one bounded counter in the workspace, split the selected blocks
  * evenly and hand their partial results over as words tagged with the
  * call's generation; other shapes run as three launches (append fused with the
