@@ -122,6 +122,14 @@ def barrier(dist=None, device=None):
 # Workload construction
 # ---------------------------------------------------------------------------
 
+def bench_config(name, wl):
+    """The workload description both arms print (the same dict)."""
+    return {"workload": name, "description": wl["text"],
+            "step": f"one ReSA cycle of {wl['f']} tokens through {wl['layers']} layers",
+            "l2": "working set larger than L2 (cache > 126 MB per layer set); no flush",
+            "parallelism": "replicas, one per GPU, no data-path collective"}
+
+
 def topk_rule(L: int, bs: int = 16, n_min: int = 16) -> int:
     """top-k of a decode step: max(n_min, round(M / 10)) capped at M, M = (L-1)//bs."""
     M = (L - 1) // bs
@@ -470,9 +478,8 @@ def run_reference(args):
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16 K/V, fp32 scores, fp64 attention (CPU oracle)",
         "data": "synthetic (seeded N(0,1) q/K/V, LogNormal K channel scale, needle blocks)",
-        "config": {"workload": args.workload, "description": wl["text"],
-                   "step": f"one ReSA cycle of {wl['f']} tokens through {wl['layers']} layers",
-                   "note": "each step is a bounded sample extrapolated to a full cycle"},
+        "config": bench_config(args.workload, wl),
+        "sample_note": "each step is a bounded sample extrapolated to a full cycle",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.num_threads(),
                          "kind": "oracle", "sample": s.describe()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -657,10 +664,8 @@ def run_resa(args):
         "warmup": W, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16 (K/V/q), fp32 accumulate and output",
         "data": "synthetic (seeded N(0,1) q/K/V, LogNormal K channel scale, needle blocks)",
-        "config": {"workload": args.workload, "description": wl["text"],
-                   "step": f"one ReSA cycle of {wl['f']} tokens through {wl['layers']} layers",
-                   "l2": "working set larger than L2 (cache > 126 MB per layer set); no flush",
-                   "parallelism": f"replicas x{world}", "graph": "one CUDA graph per cycle"},
+        "config": bench_config(args.workload, wl),
+        "execution": f"one CUDA graph per cycle; {world} replica(s)",
         "us_per_token": per_token_us,
         "roofline": roofline,
         "step_roofline": {"algorithmic_bytes_per_step": cyc_bytes / K, "achieved": step_gbs,
