@@ -469,17 +469,23 @@ def run_reference(args):
     s = OracleSample(wl, args.seed)
     for _ in range(args.warmup):
         s.run()
-    times = [s.run()[0] for _ in range(args.steps)]
-    total = sum(times)
+    runs = [s.run() for _ in range(args.steps)]
+    total = sum(r[0] for r in runs)
+    measured = sum(r[1] + r[2] for r in runs)
     value = args.steps * wl["f"] * wl["batch"] / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step_extrapolated": True,
+        "sample_ms_per_step": 1e3 * measured / args.steps,
         "vs_baseline": None, "dtype": "bf16 K/V, fp32 scores, fp64 attention (CPU oracle)",
         "data": "synthetic (seeded N(0,1) q/K/V, LogNormal K channel scale, needle blocks)",
         "config": bench_config(args.workload, wl),
-        "sample_note": "each step is a bounded sample extrapolated to a full cycle",
+        "sample_note": "each step times one decode step and one rectification row of one "
+                       "layer (sample_ms_per_step) and extrapolates them to the full cycle "
+                       f"(ms_per_step): {wl['layers']} layers x ({wl['f'] - 1} decode steps + "
+                       f"{wl['f']} rectification rows)",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.num_threads(),
                          "kind": "oracle", "sample": s.describe()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -620,6 +626,9 @@ def run_resa(args):
                 "frac": dec_gbs / hbm_peak, "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes_per_launch": dec_bytes,
                 "launch_us": dec_us, "peak_source": peak_src,
+                "isolated_launch_us": bd.get("decode_step_isolated_us") if fused else None,
+                "isolated_frac": (dec_bytes / (bd["decode_step_isolated_us"] * 1e-6) / 1e9 / hbm_peak
+                                  if fused else None),
                 "peak_kind": "burst copy (MEASURED_PEAKS hbm_gbs)"}
     # whole-step roofline: algorithmic bytes of every kernel in the cycle
     cyc_bytes = 0
@@ -738,6 +747,15 @@ def kernel_breakdown(w, stream, device, reps):
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
         w.topk_ptr(row), w.max_topk, w.out[0, w.f - 2, l], None, w.idx[l], w.cnt[l], w.ws)
         for l in range(n)], n)
+    # the same step with a plain kernel between launches (as a projection GEMM
+    # between layers would be): no overlap with the preceding launch's tail
+    z = torch.zeros(1, device=device)
+    t_pair = timed(lambda: [(R.resa_decode_step(
+        w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
+        w.topk_ptr(row), w.max_topk, w.out[0, w.f - 2, l], None, w.idx[l], w.cnt[l], w.ws),
+        z.add_(1.0)) for l in range(n)], n)
+    t_plain = timed(lambda: [z.add_(1.0) for _ in range(n)], n)
+    res["decode_step_isolated_us"] = t_pair - t_plain
     # dense decoding of the same step (append + attention over every position, Eq. 1)
     res["dense_decode_us"] = timed(lambda: [R.resa_dense_decode(
         w.cfg, w.cache(l, row), w.q[c, w.f - 2, l], w.kn[c, w.f - 2, l], w.vn[c, w.f - 2, l],
