@@ -308,6 +308,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 }
 
 constexpr int kSelCluster = 8;    // CTAs per (sequence, kv head): one thread-block cluster
+constexpr int kSelWideUnits = 64;  // from this many (sequence, kv head) units on, 2 or 4 CTAs
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelKeys = 4096;     // keys of its slice a CTA keeps in shared memory
@@ -396,8 +397,9 @@ __device__ __forceinline__ void radix_select(KeyFn key, int n, int bits_left, ui
     }
 }
 
-// Grid (kSelCluster, hkv, batch), clusters of kSelCluster CTAs along x: one
-// cluster per (sequence, kv head); CTA rank r owns keys [r*C, (r+1)*C).
+// Grid (CL, hkv, batch), clusters of CL CTAs along x: one cluster per
+// (sequence, kv head); CTA rank r owns keys [r*C, (r+1)*C).
+template <int CL>
 __global__ void __launch_bounds__(kSelThreads)
     select_kernel(const float *__restrict__ scores, uint32_t *__restrict__ hist,
                   uint32_t *__restrict__ hist_range, const int32_t *__restrict__ seq_len,
@@ -414,8 +416,8 @@ __global__ void __launch_bounds__(kSelThreads)
     __shared__ uint32_t warp_tot[kSelWarps], warp_gt[kSelWarps], warp_eq[kSelWarps];
     __shared__ uint32_t sh[4];
     __shared__ uint32_t lc_n;                   // candidates of this CTA
-    __shared__ uint32_t cta_gt[kSelCluster];    // keys > T / == T in each CTA's slice
-    __shared__ uint32_t cta_eq[kSelCluster];
+    __shared__ uint32_t cta_gt[CL];    // keys > T / == T in each CTA's slice
+    __shared__ uint32_t cta_eq[CL];
 
     pdl_launch_next();
     const int rank = (int)cluster.block_rank();
@@ -435,7 +437,7 @@ __global__ void __launch_bounds__(kSelThreads)
         k = max_topk;
     }
     k = min(k, M);
-    const int C = (M + kSelCluster - 1) / kSelCluster;
+    const int C = (M + CL - 1) / CL;
     const int c0 = min(M, rank * C), c1 = min(M, c0 + C);
     pdl_wait();
 
@@ -562,16 +564,16 @@ __global__ void __launch_bounds__(kSelThreads)
     bool fallback = trivial ? false : !hist_ok;
     if (!trivial) {
         // Gather the cluster's candidates (distributed shared memory).
-        uint32_t nr[kSelCluster], offs[kSelCluster + 1];
+        uint32_t nr[CL], offs[CL + 1];
 #pragma unroll
-        for (int r = 0; r < kSelCluster; ++r) nr[r] = *cluster.map_shared_rank(&lc_n, r);
+        for (int r = 0; r < CL; ++r) nr[r] = *cluster.map_shared_rank(&lc_n, r);
         offs[0] = 0;
 #pragma unroll
-        for (int r = 0; r < kSelCluster; ++r) {
+        for (int r = 0; r < CL; ++r) {
             offs[r + 1] = offs[r] + nr[r];
             if (nr[r] > (uint32_t)kSelLocalCand) fallback = true;
         }
-        const uint32_t ntot = offs[kSelCluster];
+        const uint32_t ntot = offs[CL];
         if (ntot > (uint32_t)kSelCandCap) fallback = true;
         if (!fallback) {
             // one flattened loop over the cluster's candidates: the remote
@@ -580,7 +582,7 @@ __global__ void __launch_bounds__(kSelThreads)
                 int r = 0;
                 uint32_t base = 0;
 #pragma unroll
-                for (int q = 1; q < kSelCluster; ++q)
+                for (int q = 1; q < CL; ++q)
                     if (j >= offs[q]) {
                         r = q;
                         base = offs[q];
@@ -630,7 +632,7 @@ __global__ void __launch_bounds__(kSelThreads)
     // This CTA's counts go into every CTA's table (remote stores), so that
     // after the next cluster barrier no CTA reads a peer's shared memory and
     // each may leave when done.
-    if (tid < kSelCluster) {
+    if (tid < CL) {
         uint32_t g2 = 0, e2 = 0;
         for (int w = 0; w < kSelWarps; ++w) {
             g2 += warp_gt[w];
@@ -743,23 +745,35 @@ cudaError_t launch_select(const Shape &s, const float *scores, uint32_t *hist,
                           uint32_t *hist_range, const int32_t *seq_len, const int32_t *topk,
                           int max_topk, int32_t *block_idx, int32_t *block_cnt, uint32_t *err,
                           cudaStream_t st) {
+    // Large batches: fewer CTAs per (sequence, kv head), so that the grid
+    // stays near one wave, as long as a CTA's keys still fit its shared
+    // memory (kSelKeys).
+    int cl = kSelCluster;
+    if (s.batch * s.hkv >= kSelWideUnits) {
+        if ((s.max_pages + 1) / 2 <= kSelKeys) cl = 2;
+        else if ((s.max_pages + 3) / 4 <= kSelKeys) cl = 4;
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kSelCluster, s.hkv, s.batch);
+    cfg.gridDim = dim3(cl, s.hkv, s.batch);
     cfg.blockDim = dim3(kSelThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kSelCluster;
+    attr[0].val.clusterDim.x = cl;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, select_kernel, scores, hist, hist_range, seq_len, topk,
-                              max_topk, block_idx, block_cnt, s.hkv, s.max_pages, s.bs, s.rows,
-                              err);
+#define RESA_SELECT_LAUNCH(CL)                                                                \
+    cudaLaunchKernelEx(&cfg, select_kernel<CL>, scores, hist, hist_range, seq_len, topk, max_topk, \
+                       block_idx, block_cnt, s.hkv, s.max_pages, s.bs, s.rows, err)
+    if (cl == 2) return RESA_SELECT_LAUNCH(2);
+    if (cl == 4) return RESA_SELECT_LAUNCH(4);
+    return RESA_SELECT_LAUNCH(kSelCluster);
+#undef RESA_SELECT_LAUNCH
 }
 
 }  // namespace resa
