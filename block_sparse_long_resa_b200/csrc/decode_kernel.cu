@@ -2,10 +2,11 @@
 // split-execution kernel of §3.4.4, redone for sm_100a).
 //
 // Grid (splits, Hkv, batch), one 8-warp CTA per SM.  CTA (s, h, b) takes the
-// s-th contiguous slice of the group's selected block list; warp w takes
-// every eighth block of the slice and keeps its own online-softmax state for
-// the group's g query heads, so the K/V of a block are fetched once for the
-// whole group.  Each warp streams its blocks through a private ring of
+// s-th contiguous slice of the group's selected block list (or of every block
+// without a list); a block of b tokens is b / 16 tiles of 16 tokens, and warp
+// w takes every eighth tile of the slice and keeps its own online-softmax
+// state for the group's g query heads, so the K/V of a block are fetched once
+// for the whole group.  Each warp streams its tiles through a private ring of
 // kStages shared-memory stages with 16-byte cp.async copies (the (page,
 // head) K and V tiles of 16 x D bf16, laid out 128-byte swizzled for
 // ldmatrix): copies through the load/store path keep HBM busy with 4 KB

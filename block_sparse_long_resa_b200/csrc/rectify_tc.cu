@@ -6,14 +6,14 @@
 // Rows of one (sequence, kv head) are rho = r * g + j (chunk position r, group
 // head j; position L - f + r).  Grid (row groups of 256, splits, batch * Hkv):
 // a CTA owns 256 rows (two M = 128 MMA tiles) and one contiguous range of KV
-// blocks, streamed as tiles of 64 keys (four blocks).
+// blocks, streamed as tiles of 64 keys (64 / b blocks of b tokens).
 //
 // Warp roles (384 threads, one CTA per SM):
-//   warp 0      TMA producer: when a tile's four blocks sit on four
-//               consecutive pages, one 4-D tensor load per channel half of K
-//               and of V (64 channels x 16 tokens x 1 head x 4 pages, 8 KB,
-//               128-byte swizzled); otherwise one 2-D load (16 x 64) per
-//               block and half.  Both write the same shared-memory image;
+//   warp 0      TMA producer: when a tile's blocks sit on consecutive pages,
+//               one 4-D tensor load per channel half of K and of V (64
+//               channels x b tokens x 1 head x 64 / b pages, 8 KB, 128-byte
+//               swizzled); otherwise one 2-D load (b x 64) per block and
+//               half.  Both write the same shared-memory image;
 //   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into a
 //               double-buffered TMEM tile (kind::f16, bf16 inputs), then
 //               O += P V (kind::f16, fp16 inputs), commits on mbarriers;
