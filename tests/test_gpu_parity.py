@@ -343,8 +343,10 @@ def test_dense_decode_long_single_sequence(cuda_device):
     ((8, 1, 64), [40, 64, 300], 40, True),
     ((28, 4, 128), [4096, 1000], 32, False),
     ((4, 2, 64), [2049, 77], 32, False),
+    ((28, 4, 128), [3000, 700], 64, True),
+    ((4, 2, 64), [500, 37], 1, True),
 ], ids=["tiny", "qwen-aligned", "qwen-unaligned", "whole-seq", "qwen-contiguous",
-        "tiny-contiguous"])
+        "tiny-contiguous", "qwen-two-row-groups", "one-row-chunk"])
 def test_rectify_matches_oracle(cuda_device, shape, ctx, f, paged):
     """Random page order takes the per-block tensor loads; the contiguous
     layout takes the four-page loads wherever a tile's pages are consecutive
@@ -505,6 +507,36 @@ def test_rectification_beyond_one_wave(cuda_device):
         qc, kc, vc = inputs.make_rectify_chunk(13 + call, B, f, 4, 4, 128)
         out = torch.empty(B, f, 4, 128, device=cuda_device)
         lse = torch.empty(B, f, 4, device=cuda_device)
+        R.resa_rectify_attention(cfg, lc.struct(), f, dev(qc), dev(kc), dev(vc), out, lse, ws)
+        assert_no_device_error(ws)
+        res = o.rectify_rows(qc, kc, vc, L, f, rows)
+        np.testing.assert_array_equal(bits_of(lc.desc), o.desc)
+        for r in rows:
+            ref, ref_lse = res[r]
+            np.testing.assert_allclose(out[:, r].cpu().numpy(), ref, rtol=0, atol=OUT_ATOL)
+            np.testing.assert_allclose(lse[:, r].cpu().numpy(), ref_lse, rtol=0, atol=LSE_ATOL)
+
+
+def test_rectification_row_groups_beyond_one_wave(cuda_device):
+    """Two 256-row groups a (sequence, kv head) (f = 64 chunk rows x 7 heads =
+    448 rows) and two key splits (the longest sequence has more than 16384
+    keys) over 48 units: 192 CTAs, more than one wave, so each group's last
+    split merges it, group 1 included.  Sampled rows of both groups against
+    the oracle; a second call reuses the reset tickets."""
+    B, f, hq, hkv, d = 12, 64, 28, 4, 128
+    ctx = [17000] + [500 + (i * 733) % 2500 for i in range(1, B)]
+    p = inputs.make_decode_problem(14, B, hq, hkv, d, 16, ctx, paged=True, needles=0,
+                                   topk=[1] * B)
+    cfg, lc, ws = setup_layer(p, cuda_device, max_chunk=f)
+    L = p.ctx_len
+    o = oracle_of(p)
+    o.build_descriptors(p.ctx_len)
+    rows = [0, 36, 37, 63]  # rows 252-258 straddle the groups; 441-447 end group 1
+    dev = lambda t: t.to(cuda_device)
+    for call in range(2):
+        qc, kc, vc = inputs.make_rectify_chunk(15 + call, B, f, hq, hkv, d)
+        out = torch.empty(B, f, hq, d, device=cuda_device)
+        lse = torch.empty(B, f, hq, device=cuda_device)
         R.resa_rectify_attention(cfg, lc.struct(), f, dev(qc), dev(kc), dev(vc), out, lse, ws)
         assert_no_device_error(ws)
         res = o.rectify_rows(qc, kc, vc, L, f, rows)
