@@ -32,9 +32,10 @@ def oracle_of(p):
 
 # --------------------------------------------------------------------------- descriptors
 
-@pytest.mark.parametrize("paged", [False, True])
-def test_descriptors_match_numpy_minmax(paged):
-    p = small_problem(paged=paged, ctx=(37, 22))
+@pytest.mark.parametrize("paged,bs,ctx", [(False, 4, (37, 22)), (True, 4, (37, 22)),
+                                           (True, 32, (201, 64)), (False, 64, (150, 63))])
+def test_descriptors_match_numpy_minmax(paged, bs, ctx):
+    p = small_problem(paged=paged, bs=bs, ctx=ctx)
     c = oracle_of(p)
     c.build_descriptors(p.ctx_len)
     for b in range(p.batch):
@@ -172,8 +173,9 @@ def test_score_ranking_scale_invariant_sign_sensitive():
 
 # --------------------------------------------------------------------------- selection
 
-def test_select_matches_lexsort():
-    p = small_problem(seed=7, d=16, bs=4, ctx=(200, 150), topk=[9, 40])
+@pytest.mark.parametrize("bs,ctx,topk", [(4, (200, 150), [9, 40]), (32, (2000, 700), [7, 30])])
+def test_select_matches_lexsort(bs, ctx, topk):
+    p = small_problem(seed=7, d=16, bs=bs, ctx=ctx, topk=topk)
     c = oracle_of(p)
     L = p.ctx_len + 1
     c.append(p.k_new, p.v_new, L)
@@ -250,8 +252,9 @@ def test_all_blocks_selected_equals_dense_sdpa():
             assert r["lse"][b, qh] == pytest.approx(lse, abs=1e-10)
 
 
-def test_sparse_equals_masked_sdpa_and_weights_sum_to_one():
-    p = small_problem(seed=9, d=32, bs=8, ctx=(130, 61), hq=4, hkv=2, topk=[4, 2])
+@pytest.mark.parametrize("bs,ctx,topk", [(8, (130, 61), [4, 2]), (64, (700, 200), [3, 1])])
+def test_sparse_equals_masked_sdpa_and_weights_sum_to_one(bs, ctx, topk):
+    p = small_problem(seed=9, d=32, bs=bs, ctx=ctx, hq=4, hkv=2, topk=topk)
     c = oracle_of(p)
     L = p.ctx_len + 1
     r = c.decode_step(p.q, p.k_new, p.v_new, p.topk, L, 8)
