@@ -329,8 +329,9 @@ def test_rectify_whole_sequence_is_causal_sdpa():
     np.testing.assert_array_equal(c.desc, fresh.desc)
 
 
-def test_rectify_chunk_rows_against_dense_and_refresh():
-    p = small_problem(seed=13, d=32, bs=8, ctx=(100, 71), hq=6, hkv=2)
+@pytest.mark.parametrize("bs", [8, 32])
+def test_rectify_chunk_rows_against_dense_and_refresh(bs):
+    p = small_problem(seed=13, d=32, bs=bs, ctx=(100, 71), hq=6, hkv=2)
     c = oracle_of(p)
     c.build_descriptors(p.ctx_len)
     f = 12
@@ -351,10 +352,10 @@ def test_rectify_chunk_rows_against_dense_and_refresh():
         k = c.keys(b, 1, int(L[b]))
         np.testing.assert_array_equal(k[-f:], kc[b, :, 1].float().numpy())
     # descriptors equal a rebuild from scratch
-    fresh = O.OracleCache(c.K, c.V, c.page_table, 6, 2, 32, 8)
+    fresh = O.OracleCache(c.K, c.V, c.page_table, 6, 2, 32, bs)
     fresh.build_descriptors(L)
     for b in range(p.batch):
-        for blk in range((int(L[b]) + 7) // 8):
+        for blk in range((int(L[b]) + bs - 1) // bs):
             page = c.page_table[b, blk]
             np.testing.assert_array_equal(c.desc[page], fresh.desc[page])
 
