@@ -109,6 +109,31 @@ def test_host_validation_without_gpu(lib):
     assert lib.resa_check_device_status(None, 0, None, None) == 1
 
 
+def test_host_validation_of_the_other_entry_points(lib):
+    """Argument checks that return before anything is launched (status codes
+    of resa.h: 1 NULL, 3 RANGE, 4 UNSUPPORTED)."""
+    cfg, c, B = R.make_config(4, 2, 64, 16), _cache(), ctypes.byref
+
+    def step(q=0x600000, topk=0x630000, max_topk=8):
+        return lib.resa_decode_step(B(cfg), B(c), q, 0x610000, 0x620000, topk, max_topk,
+                                    0x640000, None, None, None, 0xa00000, 1 << 30, None)
+    assert step(max_topk=-1) == 3
+    assert step(max_topk=65) == 3          # above max_pages with the list in the workspace
+    assert step(q=None) == 1
+    assert step(topk=0x630004) == 4        # misaligned
+    assert lib.resa_append_token(B(cfg), B(c), None, 0x620000, 0xa00000, 1 << 30, None) == 1
+    assert lib.resa_build_descriptors(None, B(c), None, 0xa00000, 1 << 30, None) == 1
+    assert lib.resa_build_descriptors(B(R.make_config(4, 2, 64, 8)), B(c), None, 0xa00000,
+                                      1 << 30, None) == 4
+    # max_topk + 1 above the split merge's 1024 x 512 blocks
+    assert lib.resa_sparse_decode(B(cfg), B(c), 0x600000, 0x700000, 0x800000, 1024 * 512,
+                                  0x640000, None, 0xa00000, 1 << 30, None) == 3
+    assert lib.resa_sparse_decode_noalloc(B(cfg), B(c), 0x600000, 0x700000, 0x800000, 8,
+                                          0x640000, None, None, None) == 1
+    assert lib.resa_sparse_decode_noalloc(B(cfg), B(c), 0x600000, 0x700000, 0x800000,
+                                          1024 * 512, 0x640000, None, 0x650000, None) == 3
+
+
 def test_binding_raises_on_error(lib):
     cfg = R.make_config(4, 2, 64, 16)
     with pytest.raises(R.ResaError) as e:
